@@ -1,0 +1,33 @@
+"""Plain CPU oracle for the vocab-sliced logits projection and the per-row sampler.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
+package.  The product path (``vocab_sharded_logits_b200``) never imports it and
+shares no code with it: no kernels, helpers, tables or constants.
+
+Every function here restates a plain definition, in float64 unless the
+definition itself fixes another precision, with no blocking, fusion or
+reordering beyond what the definition states:
+
+* ``oracle.gemm``     - the vocab-slice projection with no gather
+  ("Qwen4Exp batch-sharded sampling: inside vLLM PR #61018", orcarouter.ai
+  blog, section "batch-sharded sampling in one paragraph" and section "why
+  three lines were the whole job": each rank returns only its own vocab slice
+  of ``lm_head(hidden)``).
+* ``oracle.philox``   - Philox4x32-10 written from its published description
+  (Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As Easy as 1, 2, 3",
+  SC'11, section 3.2 and Table 2).
+* ``oracle.sampler``  - temperature, top-k, top-p, Gumbel-max draw and top-n
+  logprobs over the concatenated vocab slices of one row.  The pages name the
+  sampler's top-k / top-p / logprob work and the batch x (spec+1) x vocab logits
+  (same page, section "batch-sharded sampling in one paragraph"); the draw
+  (Gumbel-max keyed by Philox4x32 on (seed, request, position, token)) and the
+  exact tie / threshold readings are the plainest readings stated in each
+  function's docstring.
+
+Pins (see ``tests/test_oracle_*.py``): the Philox known-answer vectors of the
+Random123 distribution, brute-force enumeration on tiny vocabularies, closed
+forms (greedy == argmax, top_k=1, top_p -> 0, top_p=1 keeps all, sum of
+probabilities == 1), exact integer GEMMs, and chi-square tests of the draw
+frequencies.  No function here is "parity unpinned".
+"""
