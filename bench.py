@@ -1,0 +1,367 @@
+"""Benchmark of the vocab-sliced logits projection + per-row sampler on B200.
+
+One step = one pass of the whole hot path over one batch: ``logits_local``
+(tcgen05 GEMM, every vocab slice, no gather) followed by ``sample``
+(temperature / top-k / top-p / Gumbel-max draw / top-n logprobs) on the
+"decode" workload by default: 64 requests x 1 row, hidden 4096, vocab 151936
+in 4 slices, bf16 hidden N(0,1) and lm_head N(0,0.02), per-request
+T ~ U[0.5,1.5], top_k in {off,20,50}, top_p ~ U[0.8,1.0], top-20 logprobs.
+
+Prints ONE JSON line (rank 0).  ``--impl reference`` times the CPU oracle on
+the same workload instead.  Multi-GPU (torchrun): every rank runs its own
+batch (weak scaling, no collective on the data path); the timed region is
+bracketed by barriers and the max over ranks is reported.
+"""
+import argparse
+import json
+import os
+import shutil
+import signal
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from vocab_sharded_logits_b200 import workloads as W  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+class ClockSampler:
+    """Samples nvidia-smi SM clocks and throttle reasons during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.idx = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        if shutil.which("nvidia-smi") is None:
+            return
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                                      "-i", str(self.idx), "-lms", "100"], stdout=open(self.path, "w"),
+                                     stderr=subprocess.DEVNULL)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.send_signal(signal.SIGTERM)
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def _dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def _max_over_ranks(x, world, device):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def cpu_oracle_rows(w, n_rows, seed=0):
+    """Times the oracle on ``n_rows`` rows of workload ``w`` (projection + sampler).
+
+    Returns (seconds, rows, threads).  Inputs are made on the CPU from the same
+    seeded recipe; only the oracle calls are timed.
+    """
+    from oracle.gemm import logits_local as ref_logits
+    from oracle.sampler import sample_row
+    hidden, ws = W.gemm_inputs(W.scaled(w, requests=max(1, n_rows // w.rows_per_request)), "cpu")
+    h = hidden.float().numpy()[:n_rows]
+    ws_np = [x.float().numpy() for x in ws]
+    T, k, p, req, pos = W.row_params(w)
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        threads = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    logits = np.concatenate(ref_logits(h, ws_np), axis=1).astype(np.float32)
+    for r in range(n_rows):
+        sample_row(logits[r], T[r], int(k[r]), p[r], int(req[r]), int(pos[r]), seed, w.n_logprobs)
+    return time.perf_counter() - t0, n_rows, threads
+
+
+def run_reference(args, w):
+    world, rank, _ = _dist_setup(args.gpus)
+    if rank != 0:
+        return 0
+    for _ in range(args.warmup):
+        cpu_oracle_rows(w, 1)
+    times, rows = [], 0
+    for _ in range(args.steps):
+        t, n, threads = cpu_oracle_rows(w, args.reference_rows)
+        times.append(t)
+        rows += n
+    total = sum(times)
+    value = rows / total
+    line = {
+        "impl": "reference", "metric": _metric(w), "value": value, "unit": "rows/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": _config(w),
+        "cpu_baseline": {"value": value, "unit": "rows/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{args.reference_rows} rows per step of the {w.name} workload "
+                                   f"(float64 projection of those rows over all {w.V} tokens + the sampler oracle)"},
+        "e2e": {"value": value, "unit": "rows/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _metric(w):
+    return f"sampled rows/sec ({w.name}: logits_local GEMM + sampler, V={w.V})"
+
+
+def _config(w):
+    return {"workload": w.name, "requests": w.requests, "rows": w.R, "hidden": w.H, "vocab": w.V, "slices": w.S,
+            "n_logprobs": w.n_logprobs, "l2": "inputs larger than L2 (lm_head weights "
+            f"{w.V * w.H * 2 / 1e9:.3f} GB read per step); sampler-only figure flushes L2 between reps"}
+
+
+def run_gpu(args, w):
+    import vocab_sharded_logits_b200 as vsl
+    world, rank, local = _dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    hbm_peak, tf_peak, tf_sus, peak_kind = _peaks()
+
+    hidden, ws = W.gemm_inputs(w, dev)
+    T, k, p, req, pos = W.row_params(w)
+    params = vsl.make_row_params(T, k, p, req + rank * w.requests, pos, dev)
+    logits = [torch.empty(w.R, w.V_s, dtype=torch.float32, device=dev) for _ in range(w.S)]
+    n = w.n_logprobs
+    out = vsl.SampleResult(torch.empty(w.R, dtype=torch.int32, device=dev), torch.empty(w.R, device=dev),
+                           torch.empty(w.R, n, dtype=torch.int32, device=dev), torch.empty(w.R, n, device=dev),
+                           torch.empty(w.R, dtype=torch.int32, device=dev))
+
+    def step(seed):
+        vsl.logits_local(hidden, ws, out=logits, stream=stream)
+        vsl.sample(logits, params, seed, n, out=out, stream=stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+
+    # ---- timed region: K steps, per-kernel events on the launching stream
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    _barrier(world)
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        a, b, c = ev[i]
+        a.record(stream)
+        vsl.logits_local(hidden, ws, out=logits, stream=stream)
+        b.record(stream)
+        vsl.sample(logits, params, 1000 + i, n, out=out, stream=stream)
+        c.record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    _barrier(world)
+    clk = clocks.stop()
+    total_ms = t_start.elapsed_time(t_end)
+    gemm_ms = sum(a.elapsed_time(b) for a, b, _ in ev) / args.steps
+    samp_ms = sum(b.elapsed_time(c) for _, b, c in ev) / args.steps
+    total_ms = _max_over_ranks(total_ms, world, dev)
+    ms_per_step = total_ms / args.steps
+    value = world * w.R * args.steps / (total_ms / 1e3)
+
+    # ---- sampler alone with L2 flushed between reps (its HBM figure)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    s_times = []
+    for i in range(max(3, args.steps)):
+        flush.fill_(float(i))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        vsl.sample(logits, params, 2000 + i, n, out=out, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        s_times.append(e0.elapsed_time(e1))
+    samp_cold_ms = statistics.median(s_times)
+    del flush
+
+    # ---- end to end through the public API with host buffers
+    hidden_h = hidden.cpu().pin_memory()
+    params_h = params.cpu().pin_memory()
+    hidden_d = torch.empty_like(hidden)
+    params_d = torch.empty_like(params)
+    tok_h = torch.empty(w.R, dtype=torch.int32).pin_memory()
+    lp_h = torch.empty(w.R).pin_memory()
+    tid_h = torch.empty(w.R, n, dtype=torch.int32).pin_memory()
+    tlp_h = torch.empty(w.R, n).pin_memory()
+    flags_h = torch.empty(w.R, dtype=torch.int32).pin_memory()
+    h2d = hidden_h.numel() * hidden_h.element_size() + params_h.numel() * params_h.element_size()
+    d2h = sum(t.numel() * t.element_size() for t in (tok_h, lp_h, tid_h, tlp_h, flags_h))
+
+    def e2e_step(seed):
+        hidden_d.copy_(hidden_h, non_blocking=True)
+        params_d.copy_(params_h, non_blocking=True)
+        vsl.logits_local(hidden_d, ws, out=logits, stream=stream)
+        vsl.sample(logits, params_d, seed, n, out=out, stream=stream)
+        tok_h.copy_(out.token_ids, non_blocking=True)
+        lp_h.copy_(out.token_logprob, non_blocking=True)
+        tid_h.copy_(out.topn_ids, non_blocking=True)
+        tlp_h.copy_(out.topn_logprob, non_blocking=True)
+        flags_h.copy_(out.row_flags, non_blocking=True)
+
+    for i in range(args.warmup):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    _barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        e2e_step(3000 + i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = _max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e_value = world * w.R * args.steps / (e2e_ms / 1e3)
+    _barrier(world)
+
+    status = vsl.device_error()
+    if status != (0, 0):
+        print(f"device error word set: {status}", file=sys.stderr)
+
+    # ---- roofline of the dominant kernel
+    gemm_bytes = w.V * w.H * 2 + w.R * w.H * 2 + w.R * w.V * 4
+    gemm_flops = 2.0 * w.R * w.H * w.V
+    samp_bytes = w.R * w.V * 4
+    intensity = gemm_flops / gemm_bytes
+    ridge = tf_peak * 1e12 / (hbm_peak * 1e9)
+    if gemm_ms >= samp_ms:
+        if intensity < ridge:
+            roof = {"kernel": "logits_local_kernel", "bound": "hbm", "achieved": gemm_bytes / (gemm_ms / 1e3) / 1e9,
+                    "peak": hbm_peak, "unit": "GB/s"}
+        else:
+            roof = {"kernel": "logits_local_kernel", "bound": "tensor", "achieved": gemm_flops / (gemm_ms / 1e3) / 1e12,
+                    "peak": tf_sus, "unit": "TFLOP/s"}
+    else:
+        roof = {"kernel": "sample_kernel", "bound": "hbm", "achieved": samp_bytes / (samp_ms / 1e3) / 1e9,
+                "peak": hbm_peak, "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["peak_source"] = peak_kind
+    roof["traffic"] = None
+
+    line = {
+        "metric": _metric(w), "value": value, "unit": "rows/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": _config(w),
+        "roofline": roof,
+        "kernels": {
+            "logits_local_ms": gemm_ms, "sample_ms": samp_ms, "sample_cold_l2_ms": samp_cold_ms,
+            "gemm_tflops": gemm_flops / (gemm_ms / 1e3) / 1e12,
+            "gemm_hbm_gbs": gemm_bytes / (gemm_ms / 1e3) / 1e9,
+            "sampler_rows_per_s": w.R / (samp_ms / 1e3),
+            "sampler_hbm_gbs_cold_l2": samp_bytes / (samp_cold_ms / 1e3) / 1e9,
+            "sampler_hbm_gbs_in_step": samp_bytes / (samp_ms / 1e3) / 1e9,
+        },
+        "e2e": {"value": e2e_value, "unit": "rows/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk,
+        "cpu_baseline": None,
+    }
+    if rank == 0 and world == 1 and not args.skip_cpu:
+        secs, rows, threads = cpu_oracle_rows(w, args.cpu_rows)
+        line["cpu_baseline"] = {"value": rows / secs, "unit": "rows/s", "cores": threads, "kind": "oracle",
+                                "sample": f"{rows} rows of the {w.name} workload: float64 projection of those rows "
+                                          f"over all {w.V} tokens + the sampler oracle ({secs:.1f} s)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["vsl", "reference"], default="vsl")
+    ap.add_argument("--workload", default="decode", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--cpu-rows", type=int, default=4)
+    ap.add_argument("--reference-rows", type=int, default=2)
+    ap.add_argument("--skip-cpu", action="store_true")
+    args = ap.parse_args()
+    w = W.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    if not torch.cuda.is_available():
+        print(json.dumps({"error": "no CUDA device"}))
+        return 1
+    return run_gpu(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

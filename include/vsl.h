@@ -1,0 +1,155 @@
+/*
+ * vsl.h - C ABI of libvsl: vocab-sliced logits and the per-row sampler on one
+ * NVIDIA B200 (sm_100a).
+ *
+ * The two calls mirror the hot path of batch-sharded sampling as described in
+ * "Qwen4Exp batch-sharded sampling: inside vLLM PR #61018" (orcarouter.ai blog):
+ *
+ *   - vsl_logits_local: the rank-local vocab-slice projection with no gather
+ *     (section "why three lines were the whole job": the model's
+ *     compute_logits_local returns logits_processor(lm_head, hidden_states,
+ *     skip_gather=True), i.e. only the rank's own vocab shard; section
+ *     "batch-sharded sampling in one paragraph": each rank computes only its
+ *     own slice of the vocabulary projection).  On one GPU the S slices are
+ *     kept as an input / output layout; nothing is gathered or exchanged.
+ *   - vsl_sample: the sampler's per-request work over batch x (spec+1) x
+ *     vocab logits (same page, section "batch-sharded sampling in one
+ *     paragraph": top-k and top-p per request, logprobs under a non-negative
+ *     max_logprobs), with temperature and a Philox4x32-keyed Gumbel-max draw.
+ *
+ * Conventions for every call:
+ *   - The caller owns every buffer.  "device" pointers are CUDA device
+ *     memory of the current device; "host" arrays are ordinary host memory
+ *     read during the call only.  The library never allocates device
+ *     memory and never synchronises the stream.
+ *   - stream is a cudaStream_t (NULL = legacy default stream).  Work is
+ *     enqueued asynchronously; host-side argument errors are returned before
+ *     anything is enqueued, launch errors as VSL_ERR_CUDA.
+ *   - Row r of the logits is the concatenation of its S slices: the token
+ *     with index j in slice s has global id s * V_s + j.
+ */
+#ifndef VSL_H
+#define VSL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define VSL_API __attribute__((visibility("default")))
+#else
+#define VSL_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  VSL_OK = 0,
+  VSL_ERR_INVALID_ARG = 1,          /* null pointer, non-positive size, out-of-range value */
+  VSL_ERR_ALIGNMENT = 2,            /* pointer or row pitch not 16-byte aligned            */
+  VSL_ERR_UNSUPPORTED = 3,          /* size beyond what this build handles (see limits)    */
+  VSL_ERR_WORKSPACE_TOO_SMALL = 4,  /* workspace_bytes below vsl_sample_workspace_bytes()  */
+  VSL_ERR_CUDA = 5,                 /* a CUDA runtime / driver call failed                 */
+  VSL_ERR_DEVICE_TIMEOUT = 6        /* a kernel gave up a bounded wait (reported later by
+                                       vsl_device_error)                                    */
+} vsl_status;
+
+/* Limits of this build. */
+#define VSL_MAX_SLICES 16       /* S <= 16                                  */
+#define VSL_MAX_LOGPROBS 20     /* 0 <= n_logprobs <= 20 (and <= S * V_s)   */
+
+/* Row flags written by vsl_sample (bit set = the row was not sampled).  A
+ * flagged row gets token -1, logprob NaN, top-n ids -1 and top-n logprobs NaN;
+ * other rows are unaffected. */
+#define VSL_ROW_NONFINITE        (1u << 0)  /* a logit is NaN or +inf                   */
+#define VSL_ROW_ALL_NEG_INF      (1u << 1)  /* every logit is -inf                      */
+#define VSL_ROW_BAD_TEMPERATURE  (1u << 2)  /* temperature < 0, NaN or inf              */
+#define VSL_ROW_BAD_TOP_P        (1u << 3)  /* top_p <= 0 or NaN                        */
+#define VSL_ROW_BAD_TOP_K        (1u << 4)  /* top_k < 0                                */
+#define VSL_ROW_SCALE_OVERFLOW   (1u << 5)  /* some finite logit / temperature overflows */
+
+/* Per-row sampling parameters (20 bytes, device memory, one entry per row;
+ * a request's (spec + 1) rows normally repeat its entry with consecutive
+ * positions).
+ *   temperature : 0 = greedy (argmax of the raw logits, lowest id on ties;
+ *                 top_k and top_p are then ignored); otherwise > 0 and finite.
+ *                 Sampling uses x = fl(logit / temperature) in float32.
+ *   top_k       : 0 or >= S * V_s = off; otherwise keep every token whose x is
+ *                 >= the top_k-th largest x (ties at the boundary kept).
+ *   top_p       : >= 1 = off; otherwise in (0, 1): over the top-k survivors,
+ *                 with probabilities renormalised over them, keep a token iff
+ *                 the probability mass of strictly larger x is < top_p.
+ *   request_id, position : Philox counter words of the draw.
+ * The draw is token = argmax over kept i of x_i - log(-log(u_i)), lowest id on
+ * exact ties, with u_i = ((w >> 9) + 0.5) * 2^-23 and w the word (i mod 4) of
+ * Philox4x32-10(counter = {i / 4, position, request_id, 0},
+ *               key = {seed & 0xffffffff, seed >> 32}). */
+typedef struct {
+  float temperature;
+  int32_t top_k;
+  float top_p;
+  uint32_t request_id;
+  uint32_t position;
+} vsl_row_params;
+
+/* vsl_logits_local - logits_s[r][j] = sum_h hidden[r][h] * W_s[j][h] for every
+ * slice s, bf16 inputs, fp32 accumulation and output, no gather.
+ *   hidden_bf16   : device, [R][H] bf16 row-major, 16-byte aligned.
+ *   w_slices_bf16 : host array of S device pointers, slice s = [V_s][H] bf16
+ *                   row-major (nn.Linear out x in), each 16-byte aligned.
+ *   logits_slices : host array of S device pointers, slice s = [R][V_s] fp32
+ *                   row-major, each 16-byte aligned; fully overwritten.
+ *   R >= 1, H >= 8 with H % 8 == 0 (16-byte rows), 1 <= S <= VSL_MAX_SLICES,
+ *   V_s >= 1 with V_s % 4 == 0.
+ * Errors: VSL_ERR_INVALID_ARG (null / sizes), VSL_ERR_ALIGNMENT,
+ *         VSL_ERR_CUDA (tensor-map encode or launch failure). */
+VSL_API vsl_status vsl_logits_local(const void* hidden_bf16, const void* const* w_slices_bf16,
+                            float* const* logits_slices, int32_t R, int32_t H, int32_t S,
+                            int32_t V_s, void* stream);
+
+/* Bytes of device workspace vsl_sample needs for these sizes (0 if none). */
+VSL_API size_t vsl_sample_workspace_bytes(int32_t R, int32_t S, int32_t V_s, int32_t n_logprobs);
+
+/* vsl_sample - per-row temperature, top-k, top-p, Gumbel-max draw and top-n
+ * raw logprobs.
+ *   logits_slices : host array of S device pointers, slice s = [R][V_s] fp32
+ *                   row-major, each 16-byte aligned (read only).
+ *   params_dev    : device, R entries.
+ *   seed          : 64-bit Philox key.
+ *   n_logprobs    : 0 <= n <= VSL_MAX_LOGPROBS and n <= S * V_s.
+ *   token_ids     : device int32 [R]          (output)
+ *   token_logprob : device fp32 [R]           (output) raw log-softmax of the token
+ *   topn_ids      : device int32 [R][n]       (output; may be NULL when n == 0)
+ *   topn_logprob  : device fp32 [R][n]        (output; may be NULL when n == 0)
+ *                   the n largest raw logits' ids and log-softmax values,
+ *                   descending, lower id first on ties
+ *   row_flags     : device uint32 [R]         (output) VSL_ROW_* bits, 0 = sampled
+ *   workspace     : device, workspace_bytes >= vsl_sample_workspace_bytes()
+ *                   (may be NULL when that is 0)
+ * Logprobs are of the raw (unscaled) logits over the full vocabulary.
+ * Errors: VSL_ERR_INVALID_ARG, VSL_ERR_ALIGNMENT, VSL_ERR_UNSUPPORTED,
+ *         VSL_ERR_WORKSPACE_TOO_SMALL, VSL_ERR_CUDA. */
+VSL_API vsl_status vsl_sample(const float* const* logits_slices, int32_t R, int32_t S, int32_t V_s,
+                      const vsl_row_params* params_dev, uint64_t seed, int32_t n_logprobs,
+                      int32_t* token_ids, float* token_logprob, int32_t* topn_ids,
+                      float* topn_logprob, uint32_t* row_flags, void* workspace,
+                      size_t workspace_bytes, void* stream);
+
+/* Reads and clears the device error word the kernels set when a bounded wait
+ * gives up (a bug, never expected).  Synchronises the current device.
+ * Returns VSL_OK, VSL_ERR_DEVICE_TIMEOUT (with *code_out = the site bits) or
+ * VSL_ERR_CUDA. code_out may be NULL. */
+VSL_API vsl_status vsl_device_error(uint32_t* code_out);
+
+/* Static, human-readable name of a status code. */
+VSL_API const char* vsl_status_string(vsl_status status);
+
+/* Library version string. */
+VSL_API const char* vsl_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VSL_H */

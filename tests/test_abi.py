@@ -1,0 +1,85 @@
+"""CPU checks of the C ABI: the library loads, exports every declared symbol,
+and rejects bad arguments on the host before touching the device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "vsl.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"VSL_API\s+[\w\s\*]+?\b(vsl_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for n in ["vsl_logits_local", "vsl_sample", "vsl_sample_workspace_bytes", "vsl_status_string",
+              "vsl_device_error", "vsl_version"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    import vocab_sharded_logits_b200 as v
+    out = subprocess.run(["nm", "-D", "--defined-only", v.LIB_PATH], capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s(vsl_\w+)", out))
+    for n in _declared_functions():
+        assert n in exported, n
+        assert hasattr(v.lib, n)
+
+
+def test_status_strings_and_version():
+    import vocab_sharded_logits_b200 as v
+    assert v.status_string(0) == "ok"
+    for s in range(1, 7):
+        assert v.status_string(s) and v.status_string(s) != "unknown status"
+    assert v.status_string(99) == "unknown status"
+    assert b"sm_100a" in v.lib.vsl_version()
+
+
+def test_host_validation_rejects_bad_arguments_without_a_device():
+    import vocab_sharded_logits_b200 as v
+    L = v.lib
+    vp = ctypes.c_void_p
+    fake = vp(0x10000)                       # never dereferenced: validation fails first
+    arr1 = (vp * 1)(0x10000)
+    null_arr = (vp * 1)(0)
+    # vsl_logits_local
+    assert L.vsl_logits_local(None, arr1, arr1, 4, 64, 1, 512, None) == 1
+    assert L.vsl_logits_local(fake, arr1, arr1, 0, 64, 1, 512, None) == 1
+    assert L.vsl_logits_local(fake, arr1, arr1, 4, 64, 0, 512, None) == 1
+    assert L.vsl_logits_local(fake, arr1, arr1, 4, 64, 17, 512, None) == 3
+    assert L.vsl_logits_local(fake, arr1, arr1, 4, 60, 1, 512, None) == 2      # H % 8
+    assert L.vsl_logits_local(fake, arr1, arr1, 4, 64, 1, 510, None) == 2      # V_s % 4
+    assert L.vsl_logits_local(vp(0x10004), arr1, arr1, 4, 64, 1, 512, None) == 2
+    assert L.vsl_logits_local(fake, null_arr, arr1, 4, 64, 1, 512, None) == 1
+    # vsl_sample
+    args = lambda R=4, S=1, V_s=512, n=5, params=fake, topn=fake, ws=0: (
+        arr1, R, S, V_s, params, ctypes.c_uint64(0), n, fake, fake, topn, topn, fake, None, ws, None)
+    assert L.vsl_sample(*args(R=0)) == 1
+    assert L.vsl_sample(*args(n=-1)) == 1
+    assert L.vsl_sample(*args(n=21)) == 3
+    assert L.vsl_sample(*args(S=1, V_s=4, n=5)) == 1          # n > V
+    assert L.vsl_sample(*args(params=None)) == 1
+    assert L.vsl_sample(*args(topn=None)) == 1
+    assert L.vsl_sample(*args(V_s=514)) == 2
+    assert L.vsl_sample(*args(S=17)) == 3
+    assert L.vsl_sample(*args(V_s=1 << 20, S=1)) == 3         # beyond the largest vocabulary
+    assert L.vsl_sample_workspace_bytes(2048, 8, 18992, 20) == 0
+
+
+def test_binding_has_no_cpu_fallback(monkeypatch, tmp_path):
+    """The binding raises at import when the library is absent."""
+    import importlib.util
+    import shutil
+    pkg = os.path.join(ROOT, "vocab_sharded_logits_b200")
+    dst = tmp_path / "vocab_sharded_logits_b200"
+    shutil.copytree(pkg, dst, ignore=shutil.ignore_patterns("*.so", "csrc", "__pycache__"))
+    spec = importlib.util.spec_from_file_location("vsl_nolib", dst / "__init__.py")
+    mod = importlib.util.module_from_spec(spec)
+    with pytest.raises(ImportError):
+        spec.loader.exec_module(mod)

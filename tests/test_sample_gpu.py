@@ -1,0 +1,170 @@
+"""Parity of the CUDA sampler with the oracle (GPU), on the same seeded fp32
+logits: flags and token ids bit-exact (except near-ties / cut-ties, counted),
+top-n ids exact, logprobs within 1e-4."""
+import numpy as np
+import pytest
+import torch
+
+import vocab_sharded_logits_b200 as vsl
+from vocab_sharded_logits_b200 import workloads as W
+from parity_helpers import compare, run_sampler
+
+pytestmark = pytest.mark.gpu
+
+
+def _case(w, device, seed_offset=0, rows=None, S=None, seed=0):
+    logits = W.sampler_logits(w, device, seed_offset)
+    params = W.row_params(w, seed_offset)
+    gpu = run_sampler(logits, params, seed, w.n_logprobs, S or w.S, device)
+    rows = range(w.R) if rows is None else rows
+    return compare(gpu, logits.cpu().numpy(), params, seed, w.n_logprobs, rows), gpu
+
+
+def test_tiny_config_all_rows(cuda_device):
+    st, _ = _case(W.WORKLOADS["tiny"], cuda_device)
+    assert st["rows"] == 4
+
+
+@pytest.mark.parametrize("name", ["decode", "spec", "large", "peaked"])
+def test_small_vocab_versions_all_rows(cuda_device, name):
+    # the configs' parameter recipes at a vocabulary the oracle handles in seconds,
+    # still several CTAs per row and a ragged tail
+    w = W.scaled(W.WORKLOADS[name], V=8 * 1500, requests=max(4, 64 // W.WORKLOADS[name].rows_per_request))
+    st, _ = _case(w, cuda_device)
+    assert st["mismatch_allowed"] <= max(1, st["rows"] // 50)
+
+
+@pytest.mark.parametrize("name,nrows", [("decode", 64), ("spec", 48), ("large", 24), ("peaked", 24)])
+def test_full_size_configs_sampled_rows(cuda_device, name, nrows):
+    w = W.WORKLOADS[name]
+    rows = np.random.default_rng(5).choice(w.R, min(nrows, w.R), replace=False)
+    st, _ = _case(w, cuda_device, rows=sorted(rows.tolist()))
+    assert st["rows"] == len(rows)
+
+
+@pytest.mark.parametrize("S", [1, 2, 4, 8])
+def test_results_do_not_depend_on_slicing(cuda_device, S):
+    w = W.scaled(W.WORKLOADS["decode"], V=8 * 1024, requests=32)
+    logits = W.sampler_logits(w, cuda_device)
+    params = W.row_params(w)
+    ref = run_sampler(logits, params, 3, w.n_logprobs, 1, cuda_device)
+    got = run_sampler(logits, params, 3, w.n_logprobs, S, cuda_device)
+    for key in ref:
+        assert np.array_equal(ref[key], got[key], equal_nan=True), key
+
+
+def test_run_twice_bitwise_equal(cuda_device):
+    w = W.WORKLOADS["decode"]
+    logits = W.sampler_logits(w, cuda_device)
+    params = W.row_params(w)
+    a = run_sampler(logits, params, 11, 20, w.S, cuda_device)
+    b = run_sampler(logits, params, 11, 20, w.S, cuda_device)
+    for key in a:
+        assert np.array_equal(a[key], b[key], equal_nan=True), key
+
+
+def _edge_rows(V, rng):
+    rows, params = [], []
+    base = lambda: rng.normal(0, 1.5, V).astype(np.float32)
+    add = lambda l, T, k, p: (rows.append(l), params.append((T, k, p)))
+    add(base(), 0.0, 0, 1.0)                           # greedy
+    add(base(), 1.0, 1, 1.0)                           # top_k = 1
+    add(base(), 1.0, V, 1.0)                           # k >= V: off
+    add(base(), 1.0, V + 7, 0.5)                       # k > V with top-p
+    add(base(), 1.0, 0, 1.0)                           # pure sampling, full vocab
+    add(base(), 0.7, 0, 0.3)                           # top-p only
+    add(base(), 1.3, 3000, 0.9)                        # large k: narrowing path
+    add(base(), 0.05, 0, 0.9)                          # very peaked
+    add(base(), 50.0, 0, 0.95)                         # very flat
+    add(np.zeros(V, np.float32), 1.0, 10, 0.5)         # all equal: ties everywhere
+    add(np.zeros(V, np.float32), 0.0, 0, 1.0)          # all equal, greedy
+    l = base(); l[::3] = -np.inf; add(l, 1.0, 50, 0.9)  # -inf mixed in
+    l = np.full(V, -np.inf, np.float32); l[17] = 2.0; add(l, 1.0, 5, 0.9)  # one finite token
+    l = np.full(V, -np.inf, np.float32); l[5:9] = 1.0; add(l, 1.0, 100, 1.0)  # k > #finite
+    l = np.round(base() * 4) / 4; add(l.astype(np.float32), 1.0, 40, 0.8)    # quantised ties
+    l = base(); l[100] = np.nan; add(l, 1.0, 0, 1.0)   # NaN -> flagged
+    l = base(); l[3] = np.inf; add(l, 1.0, 0, 1.0)     # +inf -> flagged
+    add(np.full(V, -np.inf, np.float32), 1.0, 0, 1.0)  # all -inf -> flagged
+    add(base(), -1.0, 0, 1.0)                          # bad temperature
+    add(base(), float("nan"), 0, 1.0)                  # bad temperature
+    add(base(), 1.0, 0, 0.0)                           # bad top_p
+    add(base(), 1.0, -3, 1.0)                          # bad top_k
+    l = base(); l[0] = 3e38; add(l, 0.5, 0, 1.0)       # l / T overflows
+    l = base(); l[::2] = -0.0; l[1::2] = 0.0; add(l, 1.0, 2, 1.0)  # signed zeros tie
+    return np.stack(rows), params
+
+
+@pytest.mark.parametrize("V,S", [(1024, 2), (12000, 4), (151936, 8), (8, 2)])
+def test_edge_cases(cuda_device, V, S):
+    rng = np.random.default_rng(V)
+    logits, prm = _edge_rows(V, rng)
+    R = logits.shape[0]
+    T = np.array([p[0] for p in prm], np.float32)
+    k = np.array([p[1] for p in prm], np.int32)
+    p = np.array([p[2] for p in prm], np.float32)
+    req = np.arange(R)
+    pos = np.arange(R) * 3 + 1
+    n = min(20, V)
+    params = (T, k, p, req, pos)
+    gpu = run_sampler(torch.from_numpy(logits), params, 1234, n, S, cuda_device)
+    compare(gpu, logits, params, 1234, n, range(R))
+
+
+def test_no_logprobs_requested(cuda_device):
+    w = W.scaled(W.WORKLOADS["decode"], V=4 * 2048, requests=16)
+    logits = W.sampler_logits(w, cuda_device)
+    params = W.row_params(w)
+    gpu = run_sampler(logits, params, 5, 0, w.S, cuda_device)
+    compare(gpu, logits.cpu().numpy(), params, 5, 0, range(w.R))
+
+
+def test_outputs_fully_written_over_poison(cuda_device):
+    w = W.scaled(W.WORKLOADS["spec"], V=4 * 2048, requests=16)
+    logits = W.sampler_logits(w, cuda_device)
+    T, k, p, req, pos = W.row_params(w)
+    slices = [t.contiguous() for t in torch.tensor_split(logits, w.S, dim=1)]
+    prm = vsl.make_row_params(T, k, p, req, pos, cuda_device)
+    out = vsl.SampleResult(torch.full((w.R,), -7, dtype=torch.int32, device=cuda_device),
+                           torch.full((w.R,), float("nan"), device=cuda_device),
+                           torch.full((w.R, w.n_logprobs), -7, dtype=torch.int32, device=cuda_device),
+                           torch.full((w.R, w.n_logprobs), float("nan"), device=cuda_device),
+                           torch.full((w.R,), 0x7777, dtype=torch.int32, device=cuda_device))
+    vsl.sample(slices, prm, 0, w.n_logprobs, out=out)
+    torch.cuda.synchronize()
+    assert bool((out.token_ids >= 0).all()) and bool(torch.isfinite(out.token_logprob).all())
+    assert bool((out.topn_ids >= 0).all()) and bool(torch.isfinite(out.topn_logprob).all())
+    assert bool((out.row_flags == 0).all())
+    assert vsl.device_error() == (0, 0)
+
+
+def test_draw_frequencies_chi_square(cuda_device):
+    """GPU draw frequencies over many positions match the oracle's truncated,
+    renormalised distribution (chi-square, significance 1e-3, fixed seeds)."""
+    from scipy import stats
+    from oracle import sampler as S
+    rng = np.random.default_rng(77)
+    V = 1024
+    l = rng.normal(0, 1.4, V).astype(np.float32)
+    T, k, p = 0.9, 30, 0.9
+    ref = S.sample_row(l, T, k, p, 0, 0, 0, 0)
+    ids = np.nonzero(ref.kept)[0]
+    x = S.scale(l, T).astype(np.float64)
+    probs = np.exp(x[ids] - x[ids].max())
+    probs /= probs.sum()
+    R = 1 << 17
+    logits = torch.from_numpy(np.tile(l, (R, 1)))
+    params = (np.full(R, T, np.float32), np.full(R, k, np.int32), np.full(R, p, np.float32),
+              np.full(R, 9), np.arange(R))
+    counts = np.zeros(V, np.int64)
+    for seed in (0, 1, 2, 3, 4, 5, 6, 7):
+        gpu = run_sampler(logits, params, seed, 0, 2, cuda_device)
+        counts += np.bincount(gpu["token"], minlength=V)
+    assert counts[~ref.kept].sum() == 0
+    obs = counts[ids]
+    exp = probs * obs.sum()
+    big = exp >= 5
+    obs_m = np.append(obs[big], obs[~big].sum())
+    exp_m = np.append(exp[big], exp[~big].sum())
+    if exp_m[-1] == 0:
+        obs_m, exp_m = obs_m[:-1], exp_m[:-1]
+    assert stats.chisquare(obs_m, exp_m).pvalue > 1e-3

@@ -1,0 +1,180 @@
+"""Vocab-sliced logits and per-row sampler for one NVIDIA B200 (sm_100a).
+
+A thin binding over the C ABI of ``libvsl.so`` (``include/vsl.h``): argument
+marshalling only; every step of the path runs in the library's CUDA kernels.
+PyTorch is used for device memory and streams.  There is no fallback: if the
+library is missing, importing the binding raises.
+"""
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "logits_local", "sample", "make_row_params", "SampleResult", "lib", "status_string",
+    "device_error", "VslError", "ROW_NONFINITE", "ROW_ALL_NEG_INF", "ROW_BAD_TEMPERATURE",
+    "ROW_BAD_TOP_P", "ROW_BAD_TOP_K", "ROW_SCALE_OVERFLOW", "MAX_SLICES", "MAX_LOGPROBS",
+]
+
+_PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG_DIR, "libvsl.so")
+
+MAX_SLICES = 16
+MAX_LOGPROBS = 20
+ROW_NONFINITE = 1 << 0
+ROW_ALL_NEG_INF = 1 << 1
+ROW_BAD_TEMPERATURE = 1 << 2
+ROW_BAD_TOP_P = 1 << 3
+ROW_BAD_TOP_K = 1 << 4
+ROW_SCALE_OVERFLOW = 1 << 5
+
+_STATUS_NAMES = {0: "VSL_OK", 1: "VSL_ERR_INVALID_ARG", 2: "VSL_ERR_ALIGNMENT", 3: "VSL_ERR_UNSUPPORTED",
+                 4: "VSL_ERR_WORKSPACE_TOO_SMALL", 5: "VSL_ERR_CUDA", 6: "VSL_ERR_DEVICE_TIMEOUT"}
+
+
+class VslError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__(f"{where}: {_STATUS_NAMES.get(status, status)} ({status_string(status)})")
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libvsl.so not built at {LIB_PATH}; run vocab_sharded_logits_b200/build.py")
+    l = ctypes.CDLL(LIB_PATH)
+    vp, i32, u32, u64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_uint32, ctypes.c_uint64, ctypes.c_size_t
+    l.vsl_logits_local.restype = ctypes.c_int
+    l.vsl_logits_local.argtypes = [vp, ctypes.POINTER(vp), ctypes.POINTER(vp), i32, i32, i32, i32, vp]
+    l.vsl_sample_workspace_bytes.restype = sz
+    l.vsl_sample_workspace_bytes.argtypes = [i32, i32, i32, i32]
+    l.vsl_sample.restype = ctypes.c_int
+    l.vsl_sample.argtypes = [ctypes.POINTER(vp), i32, i32, i32, vp, u64, i32, vp, vp, vp, vp, vp, vp, sz, vp]
+    l.vsl_device_error.restype = ctypes.c_int
+    l.vsl_device_error.argtypes = [ctypes.POINTER(u32)]
+    l.vsl_status_string.restype = ctypes.c_char_p
+    l.vsl_status_string.argtypes = [ctypes.c_int]
+    l.vsl_version.restype = ctypes.c_char_p
+    l.vsl_version.argtypes = []
+    return l
+
+
+lib = _load()
+
+
+def status_string(status):
+    return lib.vsl_status_string(int(status)).decode()
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _ptr_array(ts):
+    arr = (ctypes.c_void_p * len(ts))()
+    for i, t in enumerate(ts):
+        arr[i] = t.data_ptr()
+    return arr
+
+
+def _stream_handle(stream, device):
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(status, where):
+    if status != 0:
+        raise VslError(status, where)
+
+
+def logits_local(hidden, w_slices, out=None, stream=None):
+    """Vocab-slice projection with no gather: ``out[s] = hidden @ w_slices[s].T`` in fp32.
+
+    hidden: bf16 [R, H] CUDA tensor; w_slices: list of bf16 [V_s, H] CUDA tensors.
+    Returns the list of fp32 [R, V_s] slices (``out`` if given).
+    """
+    R, H = hidden.shape
+    S = len(w_slices)
+    V_s = w_slices[0].shape[0]
+    if out is None:
+        out = [torch.empty(R, V_s, dtype=torch.float32, device=hidden.device) for _ in range(S)]
+    for t in [hidden, *w_slices, *out]:
+        if not t.is_contiguous():
+            raise ValueError("logits_local needs contiguous tensors")
+    if hidden.dtype != torch.bfloat16 or any(w.dtype != torch.bfloat16 for w in w_slices):
+        raise TypeError("hidden and weights must be bfloat16")
+    status = lib.vsl_logits_local(_ptr(hidden), _ptr_array(w_slices), _ptr_array(out), R, H, S, V_s,
+                                  _stream_handle(stream, hidden.device))
+    _check(status, "vsl_logits_local")
+    return out
+
+
+def make_row_params(temperature, top_k, top_p, request_id, position, device):
+    """Pack per-row parameters into the 20-byte ``vsl_row_params`` layout (int32 [R, 5])."""
+    t = torch.as_tensor(temperature, dtype=torch.float32).reshape(-1)
+    R = t.numel()
+    k = torch.as_tensor(top_k, dtype=torch.int32).reshape(-1).expand(R)
+    p = torch.as_tensor(top_p, dtype=torch.float32).reshape(-1).expand(R)
+    req = torch.as_tensor(request_id, dtype=torch.int64).reshape(-1).expand(R)
+    pos = torch.as_tensor(position, dtype=torch.int64).reshape(-1).expand(R)
+    packed = torch.empty(R, 5, dtype=torch.int32)
+    packed[:, 0] = t.view(torch.int32)
+    packed[:, 1] = k
+    packed[:, 2] = p.contiguous().view(torch.int32)
+    packed[:, 3] = _u32_to_i32(req)
+    packed[:, 4] = _u32_to_i32(pos)
+    return packed.to(device)
+
+
+def _u32_to_i32(x):
+    x = x & 0xFFFFFFFF
+    return torch.where(x >= 2 ** 31, x - 2 ** 32, x).to(torch.int32)
+
+
+class SampleResult:
+    """Outputs of ``sample``: token ids, their raw logprobs, top-n ids / logprobs, row flags."""
+
+    def __init__(self, token_ids, token_logprob, topn_ids, topn_logprob, row_flags):
+        self.token_ids = token_ids
+        self.token_logprob = token_logprob
+        self.topn_ids = topn_ids
+        self.topn_logprob = topn_logprob
+        self.row_flags = row_flags
+
+
+def sample(logits_slices, params, seed, n_logprobs, out=None, stream=None):
+    """Per-row temperature / top-k / top-p / Gumbel-max draw / top-n raw logprobs.
+
+    logits_slices: list of fp32 [R, V_s] CUDA tensors (row r = concatenation over slices).
+    params: int32 [R, 5] CUDA tensor from ``make_row_params``.
+    """
+    R, V_s = logits_slices[0].shape
+    S = len(logits_slices)
+    dev = logits_slices[0].device
+    for t in logits_slices:
+        if t.dtype != torch.float32 or not t.is_contiguous() or tuple(t.shape) != (R, V_s):
+            raise ValueError("logits slices must be contiguous fp32 [R, V_s]")
+    if params.dtype != torch.int32 or tuple(params.shape) != (R, 5) or not params.is_contiguous():
+        raise ValueError("params must be a contiguous int32 [R, 5] tensor (make_row_params)")
+    if out is None:
+        n = max(n_logprobs, 1)
+        out = SampleResult(torch.empty(R, dtype=torch.int32, device=dev),
+                           torch.empty(R, dtype=torch.float32, device=dev),
+                           torch.empty(R, n, dtype=torch.int32, device=dev)[:, :n_logprobs],
+                           torch.empty(R, n, dtype=torch.float32, device=dev)[:, :n_logprobs],
+                           torch.empty(R, dtype=torch.int32, device=dev))
+    ws_bytes = lib.vsl_sample_workspace_bytes(R, S, V_s, n_logprobs)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev) if ws_bytes else None
+    topn_ids = out.topn_ids if n_logprobs > 0 else None
+    topn_lp = out.topn_logprob if n_logprobs > 0 else None
+    status = lib.vsl_sample(_ptr_array(logits_slices), R, S, V_s, _ptr(params), ctypes.c_uint64(seed & (2 ** 64 - 1)),
+                            n_logprobs, _ptr(out.token_ids), _ptr(out.token_logprob), _ptr(topn_ids),
+                            _ptr(topn_lp), _ptr(out.row_flags), _ptr(ws), ws_bytes, _stream_handle(stream, dev))
+    _check(status, "vsl_sample")
+    return out
+
+
+def device_error():
+    """Reads and clears the kernels' error word (synchronises the device)."""
+    code = ctypes.c_uint32(0)
+    status = lib.vsl_device_error(ctypes.byref(code))
+    return status, code.value

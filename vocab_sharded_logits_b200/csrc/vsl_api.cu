@@ -1,0 +1,104 @@
+// vsl_api.cu - the extern "C" entry points of libvsl: host-side argument
+// validation, then a launch of the projection or the sampler kernel.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "vsl_internal.h"
+
+namespace vsl {
+
+// Device error word: kernels OR a site bit into it when a bounded wait gives up.
+__device__ uint32_t g_device_error = 0;
+
+uint32_t* device_error_word() {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+  return static_cast<uint32_t*>(p);
+}
+
+namespace {
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+}  // namespace
+
+}  // namespace vsl
+
+extern "C" {
+
+const char* vsl_version(void) { return "libvsl 0.1 (sm_100a)"; }
+
+const char* vsl_status_string(vsl_status status) {
+  switch (status) {
+    case VSL_OK: return "ok";
+    case VSL_ERR_INVALID_ARG: return "invalid argument";
+    case VSL_ERR_ALIGNMENT: return "pointer or row pitch not 16-byte aligned";
+    case VSL_ERR_UNSUPPORTED: return "size not supported by this build";
+    case VSL_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case VSL_ERR_CUDA: return "CUDA call failed";
+    case VSL_ERR_DEVICE_TIMEOUT: return "a kernel gave up a bounded wait";
+  }
+  return "unknown status";
+}
+
+vsl_status vsl_logits_local(const void* hidden_bf16, const void* const* w_slices_bf16, float* const* logits_slices,
+                            int32_t R, int32_t H, int32_t S, int32_t V_s, void* stream) {
+  if (hidden_bf16 == nullptr || w_slices_bf16 == nullptr || logits_slices == nullptr) return VSL_ERR_INVALID_ARG;
+  if (R <= 0 || H <= 0 || S <= 0 || V_s <= 0) return VSL_ERR_INVALID_ARG;
+  if (S > VSL_MAX_SLICES) return VSL_ERR_UNSUPPORTED;
+  if (H % 8 != 0 || V_s % 4 != 0) return VSL_ERR_ALIGNMENT;
+  if (!vsl::aligned16(hidden_bf16)) return VSL_ERR_ALIGNMENT;
+  for (int s = 0; s < S; ++s) {
+    if (w_slices_bf16[s] == nullptr || logits_slices[s] == nullptr) return VSL_ERR_INVALID_ARG;
+    if (!vsl::aligned16(w_slices_bf16[s]) || !vsl::aligned16(logits_slices[s])) return VSL_ERR_ALIGNMENT;
+  }
+  const cudaError_t e = vsl::launch_logits_local(hidden_bf16, w_slices_bf16, logits_slices, R, H, S, V_s,
+                                                 static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? VSL_OK : VSL_ERR_CUDA;
+}
+
+size_t vsl_sample_workspace_bytes(int32_t R, int32_t S, int32_t V_s, int32_t n_logprobs) {
+  (void)R;
+  (void)S;
+  (void)V_s;
+  (void)n_logprobs;
+  return 0;  // every intermediate lives in shared memory
+}
+
+vsl_status vsl_sample(const float* const* logits_slices, int32_t R, int32_t S, int32_t V_s,
+                      const vsl_row_params* params_dev, uint64_t seed, int32_t n_logprobs, int32_t* token_ids,
+                      float* token_logprob, int32_t* topn_ids, float* topn_logprob, uint32_t* row_flags,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+  (void)workspace;
+  if (logits_slices == nullptr || params_dev == nullptr || token_ids == nullptr || token_logprob == nullptr ||
+      row_flags == nullptr)
+    return VSL_ERR_INVALID_ARG;
+  if (R <= 0 || S <= 0 || V_s <= 0 || n_logprobs < 0) return VSL_ERR_INVALID_ARG;
+  if (S > VSL_MAX_SLICES || n_logprobs > VSL_MAX_LOGPROBS) return VSL_ERR_UNSUPPORTED;
+  const long long V = static_cast<long long>(S) * V_s;
+  if (n_logprobs > V) return VSL_ERR_INVALID_ARG;
+  if (n_logprobs > 0 && (topn_ids == nullptr || topn_logprob == nullptr)) return VSL_ERR_INVALID_ARG;
+  if (V_s % 4 != 0) return VSL_ERR_ALIGNMENT;
+  for (int s = 0; s < S; ++s) {
+    if (logits_slices[s] == nullptr) return VSL_ERR_INVALID_ARG;
+    if (!vsl::aligned16(logits_slices[s])) return VSL_ERR_ALIGNMENT;
+  }
+  int c = 0, part = 0;
+  if (!vsl::sample_geometry(V, &c, &part) || V > 0x7FFFFFFFLL) return VSL_ERR_UNSUPPORTED;
+  if (workspace_bytes < vsl_sample_workspace_bytes(R, S, V_s, n_logprobs)) return VSL_ERR_WORKSPACE_TOO_SMALL;
+  const cudaError_t e = vsl::launch_sample(logits_slices, R, S, V_s, params_dev, seed, n_logprobs, token_ids,
+                                           token_logprob, topn_ids, topn_logprob, row_flags,
+                                           static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? VSL_OK : VSL_ERR_CUDA;
+}
+
+vsl_status vsl_device_error(uint32_t* code_out) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return VSL_ERR_CUDA;
+  uint32_t v = 0;
+  if (cudaMemcpyFromSymbol(&v, vsl::g_device_error, sizeof(v)) != cudaSuccess) return VSL_ERR_CUDA;
+  const uint32_t zero = 0;
+  if (cudaMemcpyToSymbol(vsl::g_device_error, &zero, sizeof(zero)) != cudaSuccess) return VSL_ERR_CUDA;
+  if (code_out) *code_out = v;
+  return v ? VSL_ERR_DEVICE_TIMEOUT : VSL_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,282 @@
+// vsl_gemm.cu - vocab-slice lm_head projection on sm_100a tensor cores.
+//
+// logits_s[r][j] = sum_h hidden[r][h] * W_s[j][h] for every vocab slice s, with
+// no gather ("Qwen4Exp batch-sharded sampling: inside vLLM PR #61018",
+// orcarouter.ai blog, sections "batch-sharded sampling in one paragraph" and
+// "why three lines were the whole job").
+//
+// Design (one CTA per output tile):
+//   * The MMA M side is the vocabulary (128 rows of W_s per tile) and the N side
+//     is the batch rows (BN in {16, 32, 64, 128, 256}), so a small batch still
+//     issues full-height tcgen05.mma instructions ("swap-AB").
+//   * Warp 0 (one lane) streams K-slabs of 64 bf16 (one 128-byte swizzle row)
+//     of W_s and hidden into a STAGES-deep shared-memory ring with 2-D TMA
+//     loads (128B swizzle, zero fill past the edges, no multicast).
+//   * Warp 1 (one lane) issues tcgen05.mma.kind::f16 (bf16 x bf16 -> fp32) into
+//     a 128 x BN fp32 accumulator in tensor memory, releasing each ring slot
+//     with tcgen05.commit.
+//   * Warps 2..5 read the accumulator with tcgen05.ld (one TMEM lane = one
+//     vocab row per thread) and store fp32 logits; for each batch row a warp
+//     writes 32 consecutive floats (128 coalesced bytes).
+// Every wait is bounded; a wait that gives up sets the device error word and
+// the CTA drains its own copies, frees its tensor memory and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "vsl_internal.h"
+#include "vsl_ptx.cuh"
+
+namespace vsl {
+
+constexpr int kBM = 128;        // vocab rows per tile (MMA M)
+constexpr int kBK = 64;         // bf16 elements per K slab = 128 bytes
+constexpr int kUmmaK = 16;      // K per tcgen05.mma.kind::f16
+constexpr int kGemmThreads = 192;
+
+struct GemmArgs {
+  CUtensorMap tmap_w[VSL_MAX_SLICES];
+  CUtensorMap tmap_h;
+  float* out[VSL_MAX_SLICES];
+  int R, H, V_s;
+  int m_tiles;       // vocab tiles per slice
+  int n_tiles;       // batch tiles
+  int k_iters;       // K slabs
+  int w_evict_first; // W read once (single batch tile): stream it through L2
+  uint32_t* err;
+};
+
+// Shared-memory matrix descriptor for a K-major tile whose rows are 128 bytes,
+// stored as TMA writes it with 128-byte swizzle: 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFF) >> 4);      // start address
+  d |= static_cast<uint64_t>(1) << 16;                      // leading offset (unused, swizzled)
+  d |= static_cast<uint64_t>(1024 >> 4) << 32;              // stride between 8-row groups
+  d |= static_cast<uint64_t>(1) << 46;                      // descriptor version (sm_100)
+  d |= static_cast<uint64_t>(2) << 61;                      // 128-byte swizzle
+  return d;
+}
+
+// Instruction descriptor: D fp32, A and B bf16, both K-major, M = 128, N = BN.
+template <int BN>
+__device__ __forceinline__ uint32_t idesc_bf16_f32() {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(BN >> 3) << 17) |
+         (static_cast<uint32_t>(kBM >> 4) << 24);
+}
+
+template <int BN>
+__host__ __device__ constexpr int tmem_cols() {
+  return BN < 32 ? 32 : BN;
+}
+
+template <int BN, int STAGES>
+constexpr size_t gemm_smem_bytes() {
+  return 1024 /*alignment slack*/ + static_cast<size_t>(STAGES) * (kBM + BN) * kBK * 2 +
+         (2 * STAGES + 1) * 8 + 16;
+}
+
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(kGemmThreads, 1) logits_local_kernel(const __grid_constant__ GemmArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  constexpr uint32_t kABytes = kBM * kBK * 2;
+  constexpr uint32_t kBBytes = BN * kBK * 2;
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * kABytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * (kABytes + kBBytes));
+  uint64_t* empty = full + STAGES;
+  uint64_t* accf = empty + STAGES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n_tile = blockIdx.x % a.n_tiles;
+  const int mt = blockIdx.x / a.n_tiles;
+  const int slice = mt / a.m_tiles;
+  const int m0 = (mt % a.m_tiles) * kBM;
+  const int n0 = n_tile * BN;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    mbar_init(smem_u32(accf), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), tmem_cols<BN>());
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer
+    prefetch_tmap(&a.tmap_w[slice]);
+    prefetch_tmap(&a.tmap_h);
+    const uint64_t pol_w = a.w_evict_first ? policy_evict_first() : policy_evict_last();
+    const uint64_t pol_h = policy_evict_last();
+    int issued = 0;
+    for (int k = 0; k < a.k_iters; ++k) {
+      const int s = k % STAGES;
+      const uint32_t ph = (k / STAGES) & 1;
+      if (k >= STAGES && !mbar_wait_bounded(smem_u32(&empty[s]), ph ^ 1)) {
+        atomicOr(a.err, kErrGemmProducer);
+        *abort_flag = 1;
+        break;
+      }
+      if (*abort_flag) break;
+      mbar_arrive_expect_tx(smem_u32(&full[s]), kABytes + kBBytes);
+      tma_load_2d(smem_u32(sA + s * kABytes), &a.tmap_w[slice], k * kBK, m0, smem_u32(&full[s]), pol_w);
+      tma_load_2d(smem_u32(sB + s * kBBytes), &a.tmap_h, k * kBK, n0, smem_u32(&full[s]), pol_h);
+      issued = k + 1;
+    }
+    if (*abort_flag) {
+      // drain our own copies: the last load issued to each slot must land
+      for (int k = issued - 1; k >= 0 && k >= issued - STAGES; --k)
+        mbar_wait_bounded(smem_u32(&full[k % STAGES]), (k / STAGES) & 1);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer
+    const uint32_t idesc = idesc_bf16_f32<BN>();
+    for (int k = 0; k < a.k_iters; ++k) {
+      const int s = k % STAGES;
+      const uint32_t ph = (k / STAGES) & 1;
+      if (!mbar_wait_bounded(smem_u32(&full[s]), ph)) {
+        atomicOr(a.err, kErrGemmMma);
+        *abort_flag = 1;
+        break;
+      }
+      if (*abort_flag) break;
+      tc_fence_after();
+      const uint64_t da = sw128_desc(smem_u32(sA + s * kABytes));
+      const uint64_t db = sw128_desc(smem_u32(sB + s * kBBytes));
+#pragma unroll
+      for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
+        // advancing K by 16 bf16 = 32 bytes moves the start address by 2 (16-byte units)
+        umma_f16(tmem, da + 2 * kk, db + 2 * kk, idesc, (k | kk) != 0);
+      }
+      umma_commit(smem_u32(&empty[s]));
+    }
+    umma_commit(smem_u32(accf));
+    // the accumulator must be complete before tensor memory is freed below
+    mbar_wait_bounded(smem_u32(accf), 0);
+  } else if (warp >= 2) {
+    // ---------------- epilogue: TMEM -> registers -> global fp32
+    const bool ok = mbar_wait_bounded(smem_u32(accf), 0);
+    if (!ok) {
+      atomicOr(a.err, kErrGemmEpilogue);
+      *abort_flag = 1;
+    }
+    tc_fence_after();
+    // tcgen05.ld is warp-collective: decide for the whole warp
+    if (__all_sync(0xFFFFFFFFu, ok && !*abort_flag)) {
+      const int q = warp & 3;                  // TMEM lane quarter this warp may access
+      const int m = m0 + q * 32 + lane;        // vocab row of this thread
+      float* out = a.out[slice];
+      const bool m_ok = m < a.V_s;
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 16) {
+        uint32_t r[16];
+        tmem_ld_x16(tmem + (static_cast<uint32_t>(q * 32) << 16) + c, r);
+        tmem_ld_wait();
+        if (m_ok) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int n = n0 + c + i;
+            if (n < a.R) out[static_cast<size_t>(n) * a.V_s + m] = __uint_as_float(r[i]);
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, tmem_cols<BN>());
+  }
+}
+
+// ------------------------------------------------------------------ host side
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool get_encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode != nullptr;
+}
+
+// 2-D bf16 row-major [rows][cols] map with a box of 64 columns x box_rows rows.
+bool encode_bf16_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int BN, int STAGES>
+cudaError_t launch_bn(GemmArgs& args, const void* hidden, const void* const* w, int S, int H, int R,
+                      int V_s, cudaStream_t stream) {
+  for (int s = 0; s < S; ++s)
+    if (!encode_bf16_2d(&args.tmap_w[s], w[s], V_s, H, kBM)) return cudaErrorInvalidValue;
+  if (!encode_bf16_2d(&args.tmap_h, hidden, R, H, BN)) return cudaErrorInvalidValue;
+  args.n_tiles = (R + BN - 1) / BN;
+  args.w_evict_first = args.n_tiles == 1;
+  constexpr size_t smem = gemm_smem_bytes<BN, STAGES>();
+  auto kern = logits_local_kernel<BN, STAGES>;
+  static bool attr_set = false;  // per template instance; idempotent if raced
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const long long grid = static_cast<long long>(S) * args.m_tiles * args.n_tiles;
+  if (grid > 0x7FFFFFFF) return cudaErrorInvalidConfiguration;
+  kern<<<static_cast<unsigned>(grid), kGemmThreads, smem, stream>>>(args);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_logits_local(const void* hidden, const void* const* w_slices, float* const* logits,
+                                int R, int H, int S, int V_s, cudaStream_t stream) {
+  if (!get_encoder()) return cudaErrorNotSupported;
+  GemmArgs args{};
+  for (int s = 0; s < S; ++s) args.out[s] = logits[s];
+  args.R = R;
+  args.H = H;
+  args.V_s = V_s;
+  args.m_tiles = (V_s + kBM - 1) / kBM;
+  args.k_iters = (H + kBK - 1) / kBK;
+  args.err = device_error_word();
+  if (args.err == nullptr) return cudaErrorUnknown;
+  if (R <= 16) return launch_bn<16, 8>(args, hidden, w_slices, S, H, R, V_s, stream);
+  if (R <= 32) return launch_bn<32, 8>(args, hidden, w_slices, S, H, R, V_s, stream);
+  if (R <= 64) return launch_bn<64, 4>(args, hidden, w_slices, S, H, R, V_s, stream);
+  if (R <= 128) return launch_bn<128, 6>(args, hidden, w_slices, S, H, R, V_s, stream);
+  return launch_bn<256, 4>(args, hidden, w_slices, S, H, R, V_s, stream);
+}
+
+}  // namespace vsl
