@@ -55,15 +55,27 @@ class ClockSampler:
         self.idx = device_index
         self.proc = None
         self.path = None
+        self.skip = 0
 
     def start(self):
+        """Starts sampling and waits (up to 5 s) until the first sample is written."""
         if shutil.which("nvidia-smi") is None:
             return
         fd, self.path = tempfile.mkstemp(suffix=".csv")
         os.close(fd)
         self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
-                                      "-i", str(self.idx), "-lms", "100"], stdout=open(self.path, "w"),
+                                      "-i", str(self.idx), "-lms", "50"], stdout=open(self.path, "w"),
                                      stderr=subprocess.DEVNULL)
+        t0 = time.time()
+        while time.time() - t0 < 5 and os.path.getsize(self.path) == 0:
+            time.sleep(0.02)
+        self.skip = self.count()
+
+    def count(self):
+        if self.path is None:
+            return 0
+        with open(self.path) as f:
+            return sum(1 for _ in f)
 
     def stop(self):
         if self.proc is None:
@@ -75,7 +87,8 @@ class ClockSampler:
             self.proc.kill()
         sm, smax, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
+        lines = open(self.path).read().splitlines()[self.skip:]   # samples taken while the steps ran
+        for line in lines:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
                 continue
@@ -227,6 +240,13 @@ def run_gpu(args, w):
         c.record(stream)
     t_end.record(stream)
     torch.cuda.synchronize()
+    # a timed region shorter than the sampling period still gets samples: keep
+    # running the same step (untimed) until three samples under load exist
+    t0 = time.time()
+    while clocks.proc is not None and clocks.count() - clocks.skip < 3 and time.time() - t0 < 10:
+        for i in range(20):
+            step(5000 + i)
+        torch.cuda.synchronize()
     _barrier(world)
     clk = clocks.stop()
     total_ms = t_start.elapsed_time(t_end)

@@ -79,7 +79,7 @@ def _edge_rows(V, rng):
     add(np.zeros(V, np.float32), 1.0, 10, 0.5)         # all equal: ties everywhere
     add(np.zeros(V, np.float32), 0.0, 0, 1.0)          # all equal, greedy
     l = base(); l[::3] = -np.inf; add(l, 1.0, 50, 0.9)  # -inf mixed in
-    l = np.full(V, -np.inf, np.float32); l[17] = 2.0; add(l, 1.0, 5, 0.9)  # one finite token
+    l = np.full(V, -np.inf, np.float32); l[min(17, V - 1)] = 2.0; add(l, 1.0, 5, 0.9)  # one finite token
     l = np.full(V, -np.inf, np.float32); l[5:9] = 1.0; add(l, 1.0, 100, 1.0)  # k > #finite
     l = np.round(base() * 4) / 4; add(l.astype(np.float32), 1.0, 40, 0.8)    # quantised ties
     l = base(); l[100] = np.nan; add(l, 1.0, 0, 1.0)   # NaN -> flagged

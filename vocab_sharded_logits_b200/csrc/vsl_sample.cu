@@ -84,7 +84,7 @@ struct SampleArgs {
 
 // Per-CTA results the leader reads through distributed shared memory.
 struct CtaStats {
-  uint32_t kmax, kmin, kminf;
+  uint32_t kmax, kmin, kminf, bad;
   float m, s;           // online softmax partial: max finite logit, sum exp(l - m)
   double z;             // MASS_HIST: sum of survivor masses
   double best_sd;       // GUMBEL: float64 score of this CTA's best
@@ -170,15 +170,23 @@ constexpr size_t kScratchBytes = kHistBins * 8 + kHistBins * 4;
 constexpr size_t kListBytes = kListCap * 8;
 
 // ------------------------------------------------------------------ small helpers
-__device__ __forceinline__ uint32_t fkey(float v) {  // order-preserving key; v must be canonical (+0 for -0)
-  const uint32_t b = __float_as_uint(v);
+// Order-preserving key of a float, computed on its bits with integer operations
+// only (no float arithmetic, so NaN payloads cannot change the result): -0 and
+// +0 share one key, larger keys are larger values, -inf < finite < +inf.
+__device__ __forceinline__ uint32_t fkey_bits(uint32_t b) {
+  b = (b == 0x80000000u) ? 0u : b;
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ uint32_t fkey(float v) { return fkey_bits(__float_as_uint(v)); }
+// NaN of either sign, or +inf (-inf is a legal logit).
+__device__ __forceinline__ bool nan_or_pos_inf(uint32_t b) {
+  return (b & 0x7FFFFFFFu) > 0x7F800000u || b == 0x7F800000u;
 }
 __device__ __forceinline__ float key_value(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 __device__ __forceinline__ bool key_finite(uint32_t k) { return k > kKeyNegInf && k < kKeyPosInf; }
-__device__ __forceinline__ float scale_x(float l, float T) { return __fdiv_rn(l, T) + 0.0f; }
+__device__ __forceinline__ float scale_x(float l, float T) { return __fdiv_rn(l, T); }
 
 __device__ __forceinline__ float fast_exp2(float t) {
   float r;
@@ -407,7 +415,7 @@ __device__ uint32_t raw_prefilter(float theta, float T) {
   const double lo = static_cast<double>(t2) * static_cast<double>(T);
   const float lo32 = __double2float_rd(lo);
   if (!(lo32 > -INFINITY)) return kKeyNegInf + 1;
-  return fkey(lo32 + 0.0f);
+  return fkey(lo32);
 }
 
 // Warp-aggregated append of sort keys to the leader's list.
@@ -429,7 +437,7 @@ __device__ __forceinline__ void list_append(const Ctx& cx, bool pred, uint64_t k
 // ---- pass 1: stats + level-1 raw histogram
 __device__ void pass_stats(const Ctx& cx) {
   uint32_t* hist = reinterpret_cast<uint32_t*>(cx.scratch);
-  uint32_t kmax = 0, kmin = 0xFFFFFFFFu, kminf = 0xFFFFFFFFu;
+  uint32_t kmax = 0, kmin = 0xFFFFFFFFu, kminf = 0xFFFFFFFFu, bad = 0;
   float m = -INFINITY, s = 0.0f;
   constexpr float kLog2e = 1.4426950408889634f;
   for (int q = threadIdx.x; q < cx.n4; q += kThreads) {
@@ -439,10 +447,12 @@ __device__ void pass_stats(const Ctx& cx) {
     bool fin[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint32_t k = fkey(v[i] + 0.0f);
+      const uint32_t raw = __float_as_uint(v[i]);
+      bad |= nan_or_pos_inf(raw) ? 1u : 0u;
+      const uint32_t k = fkey_bits(raw);
       kmax = max(kmax, k);
       kmin = min(kmin, k);
-      fin[i] = key_finite(k);
+      fin[i] = key_finite(k) && !nan_or_pos_inf(raw);
       if (fin[i]) {
         kminf = min(kminf, k);
         mx = fmaxf(mx, v[i]);
@@ -464,6 +474,7 @@ __device__ void pass_stats(const Ctx& cx) {
     kmax = max(kmax, __shfl_xor_sync(0xFFFFFFFFu, kmax, o));
     kmin = min(kmin, __shfl_xor_sync(0xFFFFFFFFu, kmin, o));
     kminf = min(kminf, __shfl_xor_sync(0xFFFFFFFFu, kminf, o));
+    bad |= __shfl_xor_sync(0xFFFFFFFFu, bad, o);
     const float om = __shfl_xor_sync(0xFFFFFFFFu, m, o);
     const float os = __shfl_xor_sync(0xFFFFFFFFu, s, o);
     const float nm = fmaxf(m, om);
@@ -476,14 +487,16 @@ __device__ void pass_stats(const Ctx& cx) {
     H->red_u[warp * 4 + 0] = kmax;
     H->red_u[warp * 4 + 1] = kmin;
     H->red_u[warp * 4 + 2] = kminf;
+    H->red_u[warp * 4 + 3] = bad;
     H->red_f[warp * 2 + 0] = m;
     H->red_f[warp * 2 + 1] = s;
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    uint32_t a = 0, b = 0xFFFFFFFFu, c = 0xFFFFFFFFu;
+    uint32_t a = 0, b = 0xFFFFFFFFu, c = 0xFFFFFFFFu, d = 0;
     float M = -INFINITY;
     for (int i = 0; i < kWarps; ++i) {
+      d |= H->red_u[i * 4 + 3];
       a = max(a, H->red_u[i * 4 + 0]);
       b = min(b, H->red_u[i * 4 + 1]);
       c = min(c, H->red_u[i * 4 + 2]);
@@ -496,6 +509,7 @@ __device__ void pass_stats(const Ctx& cx) {
     H->stats.kmax = a;
     H->stats.kmin = b;
     H->stats.kminf = c;
+    H->stats.bad = d;
     H->stats.m = M;
     H->stats.s = S;
   }
@@ -510,7 +524,7 @@ __device__ void op_collect_raw(const Ctx& cx, const Plan& p) {
     const float v[4] = {v4.x, v4.y, v4.z, v4.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint32_t k = fkey(v[i] + 0.0f);
+      const uint32_t k = fkey(v[i]);
       const bool pred = valid && k >= p.lo && k <= p.hi;
       const uint32_t gid = static_cast<uint32_t>(cx.g0 + 4 * q + i);
       list_append(cx, pred, (static_cast<uint64_t>(~k) << 32) | gid);
@@ -529,7 +543,7 @@ __device__ void op_collect_x(const Ctx& cx, const Plan& p) {
     for (int i = 0; i < 4; ++i) {
       bool pred = false;
       uint32_t xk = 0;
-      const uint32_t k = fkey(v[i] + 0.0f);
+      const uint32_t k = fkey(v[i]);
       if (valid && key_finite(k) && k >= p.raw_lo) {
         const float x = scale_x(v[i], cx.T);
         xk = fkey(x);
@@ -557,7 +571,7 @@ __device__ void op_mass_hist(const Ctx& cx, const Plan& p) {
     const float v[4] = {v4.x, v4.y, v4.z, v4.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint32_t k = fkey(v[i] + 0.0f);
+      const uint32_t k = fkey(v[i]);
       if (key_finite(k) && k >= p.raw_lo) {
         const float x = scale_x(v[i], cx.T);
         if (x >= p.theta) {
@@ -584,7 +598,7 @@ __device__ void op_narrow_count(const Ctx& cx, const Plan& p) {
     const float v[4] = {v4.x, v4.y, v4.z, v4.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint32_t k = fkey(v[i] + 0.0f);
+      const uint32_t k = fkey(v[i]);
       if (k >= p.lo && k <= p.hi) atomicAdd(&cnt[(p.hi - k) >> p.shift], 1u);
     }
   }
@@ -605,7 +619,7 @@ __device__ void op_narrow_mass(const Ctx& cx, const Plan& p) {
     const float v[4] = {v4.x, v4.y, v4.z, v4.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint32_t k = fkey(v[i] + 0.0f);
+      const uint32_t k = fkey(v[i]);
       if (key_finite(k) && k >= p.raw_lo) {
         const float x = scale_x(v[i], cx.T);
         const uint32_t xk = fkey(x);
@@ -629,7 +643,7 @@ __device__ void op_next_max(const Ctx& cx, const Plan& p) {
     const float v[4] = {v4.x, v4.y, v4.z, v4.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint32_t k = fkey(v[i] + 0.0f);
+      const uint32_t k = fkey(v[i]);
       const int32_t id = static_cast<int32_t>(cx.g0 + 4 * q + i);
       const bool after = k < p.nm_key || (k == p.nm_key && id > p.nm_id);
       if (after && (!have || k > bk || (k == bk && id < bid))) {
@@ -684,7 +698,7 @@ __device__ void op_gumbel(const Ctx& cx, const Plan& p) {
     float xmax = -INFINITY;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint32_t k = fkey(v[i] + 0.0f);
+      const uint32_t k = fkey(v[i]);
       kept[i] = false;
       x[i] = -INFINITY;
       if (key_finite(k) && k >= p.raw_lo) {
@@ -971,9 +985,10 @@ __device__ Plan leader_step(const Ctx& cx) {
   switch (L.phase) {
     case PH_START: {
       if (threadIdx.x == 0) {
-        uint32_t kmax = 0, kmin = 0xFFFFFFFFu, kminf = 0xFFFFFFFFu;
+        uint32_t kmax = 0, kmin = 0xFFFFFFFFu, kminf = 0xFFFFFFFFu, bad = 0;
         float M = -INFINITY;
         for (uint32_t r = 0; r < cx.C; ++r) {
+          bad |= remote_u32(cx, &cx.H->stats.bad, r);
           kmax = max(kmax, remote_u32(cx, &cx.H->stats.kmax, r));
           kmin = min(kmin, remote_u32(cx, &cx.H->stats.kmin, r));
           kminf = min(kminf, remote_u32(cx, &cx.H->stats.kminf, r));
@@ -987,7 +1002,7 @@ __device__ Plan leader_step(const Ctx& cx) {
         }
         const vsl_row_params prm = a.params[cx.row];
         uint32_t flags = 0;
-        if (kmax >= kKeyPosInf || kmin < kKeyNegInf) flags |= VSL_ROW_NONFINITE;
+        if (bad) flags |= VSL_ROW_NONFINITE;
         else if (kmax == kKeyNegInf) flags |= VSL_ROW_ALL_NEG_INF;
         if (!(prm.temperature >= 0.0f && prm.temperature < INFINITY)) flags |= VSL_ROW_BAD_TEMPERATURE;
         if (!(prm.top_p > 0.0f)) flags |= VSL_ROW_BAD_TOP_P;
