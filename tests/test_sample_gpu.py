@@ -82,7 +82,7 @@ def _edge_rows(V, rng):
     l = np.full(V, -np.inf, np.float32); l[min(17, V - 1)] = 2.0; add(l, 1.0, 5, 0.9)  # one finite token
     l = np.full(V, -np.inf, np.float32); l[5:9] = 1.0; add(l, 1.0, 100, 1.0)  # k > #finite
     l = np.round(base() * 4) / 4; add(l.astype(np.float32), 1.0, 40, 0.8)    # quantised ties
-    l = base(); l[100] = np.nan; add(l, 1.0, 0, 1.0)   # NaN -> flagged
+    l = base(); l[min(100, V - 1)] = np.nan; add(l, 1.0, 0, 1.0)   # NaN -> flagged
     l = base(); l[3] = np.inf; add(l, 1.0, 0, 1.0)     # +inf -> flagged
     add(np.full(V, -np.inf, np.float32), 1.0, 0, 1.0)  # all -inf -> flagged
     add(base(), -1.0, 0, 1.0)                          # bad temperature

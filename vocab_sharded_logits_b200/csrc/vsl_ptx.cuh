@@ -110,6 +110,15 @@ __device__ __forceinline__ uint32_t mapa(uint32_t local, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
   return r;
 }
+// Generic pointer to the same shared variable in CTA `rank` of this cluster.
+// Plain loads and stores through it are ordinary memory operations the
+// compiler can batch; cluster barriers order them across CTAs.
+template <typename T>
+__device__ __forceinline__ T* cluster_ptr(T* local, uint32_t rank) {
+  uint64_t r;
+  asm("mapa.u64 %0, %1, %2;" : "=l"(r) : "l"(reinterpret_cast<uint64_t>(local)), "r"(rank));
+  return reinterpret_cast<T*>(r);
+}
 __device__ __forceinline__ uint32_t ld_dsmem_u32(uint32_t addr) {
   uint32_t v;
   asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");

@@ -8,29 +8,33 @@
 // top-k / top-p per request over batch x (spec+1) x vocab logits, logprobs
 // under a non-negative max_logprobs).
 //
-// Execution model: one thread-block cluster of C CTAs per row.  CTA c copies
-// its contiguous part of the row (global ids [c*part, (c+1)*part)) from HBM
-// into shared memory with 1-D bulk copies, once; every later pass re-reads
-// shared memory, so each logit crosses HBM exactly once.  CTA rank 0 (the
-// leader) merges the CTAs' partial results through distributed shared memory
-// and plans the next pass ("op"); the cluster runs ops until the row is done:
+// Execution model: one thread-block cluster of C CTAs per row, several
+// clusters resident at once.  CTA c copies its contiguous part of the row
+// (global ids [c*part, (c+1)*part)) from HBM into shared memory with chunked
+// 1-D bulk copies, once, and starts its first pass on the chunks that have
+// landed; every later pass re-reads shared memory, so each logit crosses HBM
+// exactly once.  CTA rank 0 (the leader) merges partial results through
+// distributed shared memory and plans the next pass ("op"):
 //
-//   pass 1 (always)  max / min keys, online sum exp(l - M), and a 4096-bin
-//                    histogram of order-preserving keys of the raw logits
-//   COLLECT_RAW      candidates with key >= lo go to the leader's list: the
-//                    top-n, the argmax, and (when it fits) all top-k
-//                    survivors, resolved exactly by a sort in shared memory
-//   MASS_HIST        (top-k off / too large) float64 masses exp(x - m) of the
-//                    survivors, histogrammed on keys of x, and their sum Z
-//   COLLECT_X        survivors with x-key in [lo, hi] to the leader's list
-//   NARROW_COUNT/MASS  256-bin refinement of a key range (counts or masses)
-//   NEXT_MAX         the next largest (key, lowest id) after a given pair
-//   GUMBEL           Philox + Gumbel scores over every kept logit, per-CTA best
+//   pass 1 (always)  max key, NaN and +inf, online sum exp(l - M) and a
+//                    4096-bin histogram of order-preserving keys of raw logits
+//   COLLECT_RAW      keys >= lo go to the leader's list: the top-n and, when
+//                    every top-k survivor fits, all of them; the leader then
+//                    resolves top-n, top-k, top-p and the draw on the sorted
+//                    list alone while the other CTAs leave
+//   NEXT_MAX         the next (key desc, id asc) element: top-n under ties
+//   NARROW_COUNT     256-bin refinement of the top-k rank inside a key range
+//   MASS             x = fl(l / T) written in place, and the float64 masses
+//                    exp(x - m) of the survivors summed exactly in 76-bit
+//                    fixed point on 240 bins of equal width in x below m,
+//                    whose edges are exact key boundaries
+//   NARROW_MASS      256-bin refinement of the top-p cut inside an x-key range
+//   GUMBEL           Philox + Gumbel scores over every kept x, per-CTA best
 //
-// Exactness: x = fl(l / T) uses IEEE division; top-k / top-p thresholds are
-// found by exact integer selection on keys and float64 masses; the draw's
-// float32 scores are re-compared in float64 whenever two candidates are
-// closer than the float32 error bound, so the result is the float64 argmax.
+// Exactness: x uses IEEE division; the top-k threshold is an exact integer
+// rank selection on keys; the top-p cut compares exact sums of float64 masses
+// (fixed point, independent of summation order); the draw's float32 scores are
+// re-compared in float64 whenever float32 cannot separate two candidates.
 #include <cuda_runtime.h>
 
 #include <cfloat>
@@ -42,14 +46,16 @@
 
 namespace vsl {
 
-constexpr int kThreads = 512;
+constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kHistBins = 4096;      // level-1 bins: key >> 20
-constexpr int kListCap = 4096;       // leader candidate list capacity
-constexpr int kSubBins = 256;        // narrowing bins
+constexpr int kHistBins = 4096;        // pass-1 bins: raw key >> 20 (1/8 octave)
+constexpr int kMassBins = 240;         // mass bins: equal steps of x below the max
+constexpr int kSubBins = 256;          // narrowing bins
+constexpr int kListCap = 2048;         // leader candidate list capacity
 constexpr int kMaxCluster = 16;
-constexpr int kMaxPart = 32768;      // floats per CTA (128 KB)
-constexpr int kPreferredPart = 20480;  // floats per CTA (80 KB) when the cluster allows it
+constexpr int kMaxPart = 32768;        // floats per CTA (128 KB)
+constexpr int kPreferredPart = 12288;  // floats per CTA (48 KB) when the cluster size allows it
+constexpr int kLoadChunks = 4;
 
 constexpr uint32_t kKeyNegInf = 0x007FFFFFu;  // key(-inf)
 constexpr uint32_t kKeyPosInf = 0xFF800000u;  // key(+inf)
@@ -61,13 +67,14 @@ constexpr uint32_t kPhiloxW0 = 0x9E3779B9u, kPhiloxW1 = 0xBB67AE85u;
 enum Op : uint32_t {
   OP_END = 0,
   OP_COLLECT_RAW,
-  OP_COLLECT_X,
-  OP_MASS_HIST,
-  OP_NARROW_COUNT,
-  OP_NARROW_MASS,
   OP_NEXT_MAX,
+  OP_NARROW_COUNT,
+  OP_MASS,
+  OP_NARROW_MASS,
   OP_GUMBEL,
 };
+
+enum Tail : uint32_t { TAIL_NONE = 0, TAIL_LIST_GREEDY, TAIL_LIST_SAMPLE, TAIL_STREAM_DONE };
 
 struct SampleArgs {
   const float* slices[VSL_MAX_SLICES];
@@ -84,36 +91,40 @@ struct SampleArgs {
 
 // Per-CTA results the leader reads through distributed shared memory.
 struct CtaStats {
-  uint32_t kmax, kmin, kminf, bad;
+  uint32_t kmax, kminf, bad, pad;
   float m, s;           // online softmax partial: max finite logit, sum exp(l - m)
-  double z;             // MASS_HIST: sum of survivor masses
-  double best_sd;       // GUMBEL: float64 score of this CTA's best
-  int32_t best_id;
-  float best_l;
   uint32_t nm_key;      // NEXT_MAX result
   int32_t nm_id;
+};
+
+// GUMBEL result pushed by each CTA into the leader's slot [rank].
+struct BestSlot {
+  double sd;
+  int32_t id;
+  float l;
 };
 
 struct Plan {
   uint32_t op;
   uint32_t lo, hi, shift;  // key range and narrowing bin shift
-  uint32_t raw_lo;         // raw-key prefilter: elements below cannot be survivors / kept
-  float theta;             // survivor (MASS, NARROW_MASS, COLLECT_X) or kept (GUMBEL) threshold on x
+  float theta;             // survivor (MASS, NARROW_MASS) or kept (GUMBEL) threshold on x
   float m;                 // max x (masses are exp(x - m))
   uint32_t nm_key;         // NEXT_MAX: previous (key, id)
   int32_t nm_id;
+  uint32_t part_is_x;      // shared memory holds x = fl(l / T) instead of l
+  uint32_t last;           // the cluster's last op for this row
+  float step;              // MASS: width in x of one bin
+  uint32_t pad;
 };
 
 enum Phase : uint32_t {
   PH_START = 0,
-  PH_AFTER_COLLECT_RAW,
   PH_TOPN_NEXT_MAX,
+  PH_AFTER_TOPN_COLLECT,
   PH_TOPK_NARROW,
   PH_AFTER_MASS,
   PH_MASS_NARROW,
-  PH_AFTER_COLLECT_X,
   PH_AFTER_GUMBEL,
-  PH_DONE,
 };
 
 // Leader-only working state.
@@ -124,49 +135,45 @@ struct LeaderState {
   int32_t top_k;
   uint32_t req, pos;
   int r_n, r_k;
-  bool greedy, k_listed, topn_done;
+  int greedy, topn_listed, part_is_x, mode;
   uint32_t collect_lo;
   float theta_k, theta_p, m;
-  uint32_t surv_raw_lo;     // raw prefilter for survivors of top-k
-  double Z;
   // narrowing state
-  uint32_t nlo, nhi, nshift;
-  uint32_t nrank;
-  double cum_above;
+  uint32_t nlo, nhi, nshift, nrank;
+  unsigned long long cum_hi, cum_lo;   // exact mass strictly above the range (fixed point)
+  unsigned long long z_hi, z_lo;       // exact total mass (fixed point)
   int topn_count;
   uint32_t prev_key;
   int32_t prev_id;
-  // result
   int32_t token;
   float token_l;
   // scratch for block-wide searches
   int found_bin;
   uint32_t found_cum;
-  double found_mass;
-  int sstar, send;
-  int last_bin;
-  double last_before;
-  uint32_t last_cumc;
-  bool x_from_top;          // the x-key list starts at the top of the row
+  uint32_t found_cnt;
+  unsigned long long found_hi, found_lo;
 };
 
 struct __align__(16) SharedHeader {
   CtaStats stats;
+  CtaStats all[kMaxCluster];   // leader only: every CTA's stats, pushed before a cluster barrier
   Plan plan;
   LeaderState L;
+  BestSlot best[kMaxCluster];
   uint32_t list_count;
   uint32_t pad;
-  unsigned long long mbar;
+  unsigned long long mbar[kLoadChunks];
   double red_d[kWarps];
   uint32_t red_u[kWarps * 4];
   float red_f[kWarps * 2];
   int32_t red_i[kWarps];
   double scan_d[kWarps];
   uint32_t scan_u[kWarps];
+  unsigned long long scan_h[kWarps], scan_l[kWarps];
+  double exp_tab[64];
 };
 
-// Scratch union (48 KB).
-constexpr size_t kScratchBytes = kHistBins * 8 + kHistBins * 4;
+constexpr size_t kScratchBytes = kHistBins * 4;  // 16 KB: raw histogram, later mass / narrowing bins
 constexpr size_t kListBytes = kListCap * 8;
 
 // ------------------------------------------------------------------ small helpers
@@ -178,12 +185,12 @@ __device__ __forceinline__ uint32_t fkey_bits(uint32_t b) {
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 __device__ __forceinline__ uint32_t fkey(float v) { return fkey_bits(__float_as_uint(v)); }
+__device__ __forceinline__ float key_value(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
 // NaN of either sign, or +inf (-inf is a legal logit).
 __device__ __forceinline__ bool nan_or_pos_inf(uint32_t b) {
   return (b & 0x7FFFFFFFu) > 0x7F800000u || b == 0x7F800000u;
-}
-__device__ __forceinline__ float key_value(uint32_t k) {
-  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 __device__ __forceinline__ bool key_finite(uint32_t k) { return k > kKeyNegInf && k < kKeyPosInf; }
 __device__ __forceinline__ float scale_x(float l, float T) { return __fdiv_rn(l, T); }
@@ -192,6 +199,58 @@ __device__ __forceinline__ float fast_exp2(float t) {
   float r;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(t));
   return r;
+}
+
+// Mass-bin edges: bin j holds the x-keys in (edge[j + 1], edge[j]], with
+// edge[j] = key(fl(m - j * step)) (non-increasing in j) and the last bin
+// open below.  Computed the same way by every CTA, so the bins agree exactly.
+__device__ __forceinline__ uint32_t mass_edge(float m, float step, int j) {
+  return fkey(__fsub_rn(m, __fmul_rn(static_cast<float>(j), step)));
+}
+__device__ __forceinline__ int mass_bin(const uint32_t* edge, float m, float inv_step, float x, uint32_t k) {
+  int j = static_cast<int>(fminf(fmaxf(__fmul_rn(__fsub_rn(m, x), inv_step), 0.0f), static_cast<float>(kMassBins - 1)));
+  while (j > 0 && k > edge[j]) --j;
+  while (j < kMassBins - 1 && k <= edge[j + 1]) ++j;
+  return j;
+}
+
+// exp(d) for d <= 0 in float64, table-driven (P. T. P. Tang, "Table-driven
+// implementation of the exponential function in IEEE floating-point
+// arithmetic", ACM TOMS 15(2), 1989): d = (64 m + j) ln2/64 + r with
+// |r| <= ln2/128, exp(d) = 2^m * 2^(j/64) * p(r), p the degree-5 Taylor
+// polynomial of exp (truncation < 4e-17).  tab[j] = 2^(j/64).  ln2/64 is split
+// in a 35-bit high part (so n * hi is exact) and the rest.
+__device__ __forceinline__ double exp_neg64(double d, const double* tab) {
+  if (d < -708.0) return 0.0;  // below 1e-307: no mass that a sum of < 2^20 terms resolves
+  constexpr double kInvLn2x64 = 92.33248261689366;           // 64 / ln 2
+  constexpr double kLn2d64Hi = 0.010830424695996044;         // ln2 / 64, 35 significant bits
+  constexpr double kLn2d64Lo = 2.5310172166650877e-13;       // ln2 / 64 - high part
+  const int n = __double2int_rn(d * kInvLn2x64);
+  const double nd = static_cast<double>(n);
+  double r = fma(-nd, kLn2d64Hi, d);
+  r = fma(-nd, kLn2d64Lo, r);
+  double p = 1.0 / 120.0;
+  p = fma(p, r, 1.0 / 24.0);
+  p = fma(p, r, 1.0 / 6.0);
+  p = fma(p, r, 0.5);
+  p = fma(p, r, 1.0);
+  p = fma(p, r, 1.0);
+  const double v = tab[n & 63] * p;
+  const int m = n >> 6;  // floor(n / 64)
+  if (m < -1020) return ldexp(v, m);
+  return __hiloint2double(__double2hiint(v) + (m << 20), __double2loint(v));
+}
+
+// Fixed-point mass: e in (0, 1] as e * 2^76 = hi * 2^32 + lo, both exact integers
+// (hi <= 2^44, lo <= 2^32), so sums of up to 2^18 masses are exact in 64 bits.
+__device__ __forceinline__ void mass_fixed(double e, unsigned long long& hi, unsigned long long& lo) {
+  const double s = e * 0x1p44;
+  const double h = floor(s);
+  hi = static_cast<unsigned long long>(h);
+  lo = __double2ull_rn((s - h) * 0x1p32);
+}
+__device__ __forceinline__ double fixed_to_double(unsigned long long hi, unsigned long long lo) {
+  return static_cast<double>(hi) * 0x1p-44 + static_cast<double>(lo) * 0x1p-76;
 }
 
 __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
@@ -224,6 +283,10 @@ __device__ __forceinline__ double gumbel64(uint32_t w) {
   const double u = (static_cast<double>(w >> 9) + 0.5) * 0x1p-23;
   return -log(-log(u));
 }
+// 1 - u for the word, exact in float32.
+__device__ __forceinline__ float one_minus_u(uint32_t w) {
+  return (static_cast<float>(0x7FFFFFu - (w >> 9)) + 0.5f) * 0x1p-23f;
+}
 // Bound on |float32 score - exact score| for score s (logf / log1pf are within
 // 1 ulp; |g| < 17), with a 3x safety factor.
 __device__ __forceinline__ float score_tol(float s) { return 8e-6f + 3e-7f * fabsf(s); }
@@ -241,6 +304,9 @@ struct Best {
     s = -INFINITY;
     id = 0x7FFFFFFF;
     sd = -INFINITY;
+    x = 0.f;
+    l = 0.f;
+    w = 0;
   }
   __device__ double exact() {
     if (!have_sd) {
@@ -249,7 +315,15 @@ struct Best {
     }
     return sd;
   }
-  __device__ void offer(float cx, float cl, uint32_t cw, int32_t cid) {
+  // Offers candidate (x, raw l, Philox word, id).  A cheap test rejects most
+  // candidates first: beating the best needs -log u < exp(x - bound) with
+  // bound below the best's exact score, and -log u >= 1 - u.
+  __device__ __forceinline__ void offer(float cx, float cl, uint32_t cw, int32_t cid) {
+    if (valid) {
+      const float bound = s - score_tol(s) - 3e-5f;
+      const float q = fast_exp2((cx - bound) * 1.4426950408889634f);
+      if (one_minus_u(cw) > q * 1.0001f + 1e-30f) return;
+    }
     const float cs = cx + gumbel32(cw);
     if (!valid) {
       s = cs; x = cx; l = cl; w = cw; id = cid; valid = true; have_sd = false;
@@ -276,17 +350,6 @@ __device__ __forceinline__ T warp_reduce(T v, F f) {
   return v;
 }
 
-__device__ __forceinline__ double block_sum_d(double v, SharedHeader* H) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  v = warp_reduce(v, [](double a, double b) { return a + b; });
-  __syncthreads();
-  if (lane == 0) H->red_d[warp] = v;
-  __syncthreads();
-  double t = 0.0;
-  for (int i = 0; i < kWarps; ++i) t += H->red_d[i];  // fixed order: deterministic
-  return t;
-}
-
 __device__ __forceinline__ int block_max_i(int v, SharedHeader* H) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   v = warp_reduce(v, [](int a, int b) { return a > b ? a : b; });
@@ -297,9 +360,7 @@ __device__ __forceinline__ int block_max_i(int v, SharedHeader* H) {
   for (int i = 1; i < kWarps; ++i) t = max(t, H->red_i[i]);
   return t;
 }
-__device__ __forceinline__ int block_min_i(int v, SharedHeader* H) {
-  return -block_max_i(-v, H);
-}
+__device__ __forceinline__ int block_min_i(int v, SharedHeader* H) { return -block_max_i(-v, H); }
 
 // Inclusive prefix sum over threads (thread order), u32; also returns the block total.
 __device__ __forceinline__ uint32_t block_scan_u(uint32_t v, uint32_t* total, SharedHeader* H) {
@@ -339,6 +400,30 @@ __device__ __forceinline__ double block_scan_d(double v, double* total, SharedHe
   }
   *total = tot;
   return x + off;
+}
+// Inclusive prefix sum of a fixed-point pair (hi, lo) over threads: exact.
+__device__ __forceinline__ void block_scan_fixed(unsigned long long& hi, unsigned long long& lo, SharedHeader* H) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long yh = __shfl_up_sync(0xFFFFFFFFu, hi, o);
+    const unsigned long long yl = __shfl_up_sync(0xFFFFFFFFu, lo, o);
+    if (lane >= o) {
+      hi += yh;
+      lo += yl;
+    }
+  }
+  __syncthreads();
+  if (lane == 31) {
+    H->scan_h[warp] = hi;
+    H->scan_l[warp] = lo;
+  }
+  __syncthreads();
+  for (int i = 0; i < warp; ++i) {
+    hi += H->scan_h[i];
+    lo += H->scan_l[i];
+  }
+  __syncthreads();
 }
 
 // Block argmax of (sd desc, id asc); every thread gets the winner's (sd, id, l).
@@ -394,11 +479,11 @@ __device__ void bitonic_sort(uint64_t* a, int n) {
   }
 }
 
-// ------------------------------------------------------------------ the kernel
+// ------------------------------------------------------------------ per-CTA context
 struct Ctx {
   const SampleArgs* a;
   SharedHeader* H;
-  const float4* part4;
+  float4* part4;
   uint8_t* scratch;
   uint64_t* list;
   int row, n4;
@@ -407,6 +492,18 @@ struct Ctx {
   float T;
   uint32_t req, pos;
 };
+
+// Sum over the cluster's CTAs of one shared variable (loads issued together).
+template <typename T>
+__device__ __forceinline__ T cluster_sum(const Ctx& cx, const T* local) {
+  T v[kMaxCluster];
+#pragma unroll
+  for (int r = 0; r < kMaxCluster; ++r) v[r] = r < static_cast<int>(cx.C) ? *cluster_ptr(local, r) : T(0);
+  T t = 0;
+#pragma unroll
+  for (int r = 0; r < kMaxCluster; ++r) t += v[r];
+  return t;
+}
 
 // Raw-key lower bound for l such that fl(l / T) >= theta is possible.
 __device__ uint32_t raw_prefilter(float theta, float T) {
@@ -429,50 +526,55 @@ __device__ __forceinline__ void list_append(const Ctx& cx, bool pred, uint64_t k
   base = __shfl_sync(0xFFFFFFFFu, base, __ffs(mask) - 1);
   if (pred) {
     const uint32_t idx = base + __popc(mask & ((1u << lane) - 1u));
-    if (idx < static_cast<uint32_t>(kListCap))
-      st_dsmem_u64(mapa(smem_u32(cx.list + idx), 0), key);
+    if (idx < static_cast<uint32_t>(kListCap)) st_dsmem_u64(mapa(smem_u32(cx.list + idx), 0), key);
   }
 }
 
-// ---- pass 1: stats + level-1 raw histogram
-__device__ void pass_stats(const Ctx& cx) {
+// ---- pass 1: stats + raw-key histogram, chunk by chunk as the bulk copies land
+__device__ void pass_stats(const Ctx& cx, const int* chunk_q) {
   uint32_t* hist = reinterpret_cast<uint32_t*>(cx.scratch);
-  uint32_t kmax = 0, kmin = 0xFFFFFFFFu, kminf = 0xFFFFFFFFu, bad = 0;
+  uint32_t kmax = 0, kminf = 0xFFFFFFFFu, bad = 0;
   float m = -INFINITY, s = 0.0f;
+  bool load_ok = true;
   constexpr float kLog2e = 1.4426950408889634f;
-  for (int q = threadIdx.x; q < cx.n4; q += kThreads) {
-    const float4 v4 = cx.part4[q];
-    const float v[4] = {v4.x, v4.y, v4.z, v4.w};
-    float mx = -INFINITY;
-    bool fin[4];
+  for (int c = 0; c < kLoadChunks; ++c) {
+    if (load_ok && !mbar_wait_bounded(smem_u32(&cx.H->mbar[c]), 0)) {
+      if (threadIdx.x == 0) atomicOr(cx.a->err, kErrSampleLoad);
+      load_ok = false;
+    }
+    for (int q = chunk_q[c] + threadIdx.x; q < chunk_q[c + 1]; q += kThreads) {
+      const float4 v4 = cx.part4[q];
+      const float v[4] = {v4.x, v4.y, v4.z, v4.w};
+      float mx = -INFINITY;
+      bool fin[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint32_t raw = __float_as_uint(v[i]);
-      bad |= nan_or_pos_inf(raw) ? 1u : 0u;
-      const uint32_t k = fkey_bits(raw);
-      kmax = max(kmax, k);
-      kmin = min(kmin, k);
-      fin[i] = key_finite(k) && !nan_or_pos_inf(raw);
-      if (fin[i]) {
-        kminf = min(kminf, k);
-        mx = fmaxf(mx, v[i]);
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t raw = __float_as_uint(v[i]);
+        const bool nb = nan_or_pos_inf(raw);
+        bad |= nb ? 1u : 0u;
+        const uint32_t k = fkey_bits(raw);
+        kmax = max(kmax, k);
+        fin[i] = key_finite(k) && !nb;
+        if (fin[i]) {
+          kminf = min(kminf, k);
+          mx = fmaxf(mx, v[i]);
+        }
+        atomicAdd(&hist[k >> 20], 1u);
       }
-      atomicAdd(&hist[k >> 20], 1u);
-    }
-    if (mx > m) {
-      s = (m == -INFINITY) ? 0.0f : s * fast_exp2((m - mx) * kLog2e);
-      m = mx;
-    }
+      if (mx > m) {
+        s = (m == -INFINITY) ? 0.0f : s * fast_exp2((m - mx) * kLog2e);
+        m = mx;
+      }
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      if (fin[i]) s += fast_exp2((v[i] - m) * kLog2e);
+      for (int i = 0; i < 4; ++i)
+        if (fin[i]) s += fast_exp2((v[i] - m) * kLog2e);
+    }
   }
   // block reduce
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     kmax = max(kmax, __shfl_xor_sync(0xFFFFFFFFu, kmax, o));
-    kmin = min(kmin, __shfl_xor_sync(0xFFFFFFFFu, kmin, o));
     kminf = min(kminf, __shfl_xor_sync(0xFFFFFFFFu, kminf, o));
     bad |= __shfl_xor_sync(0xFFFFFFFFu, bad, o);
     const float om = __shfl_xor_sync(0xFFFFFFFFu, m, o);
@@ -485,20 +587,18 @@ __device__ void pass_stats(const Ctx& cx) {
   SharedHeader* H = cx.H;
   if (lane == 0) {
     H->red_u[warp * 4 + 0] = kmax;
-    H->red_u[warp * 4 + 1] = kmin;
     H->red_u[warp * 4 + 2] = kminf;
-    H->red_u[warp * 4 + 3] = bad;
+    H->red_u[warp * 4 + 3] = bad | (load_ok ? 0u : 1u);
     H->red_f[warp * 2 + 0] = m;
     H->red_f[warp * 2 + 1] = s;
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    uint32_t a = 0, b = 0xFFFFFFFFu, c = 0xFFFFFFFFu, d = 0;
+    uint32_t a = 0, c = 0xFFFFFFFFu, d = 0;
     float M = -INFINITY;
     for (int i = 0; i < kWarps; ++i) {
       d |= H->red_u[i * 4 + 3];
       a = max(a, H->red_u[i * 4 + 0]);
-      b = min(b, H->red_u[i * 4 + 1]);
       c = min(c, H->red_u[i * 4 + 2]);
       M = fmaxf(M, H->red_f[i * 2]);
     }
@@ -506,129 +606,35 @@ __device__ void pass_stats(const Ctx& cx) {
     if (M > -INFINITY)
       for (int i = 0; i < kWarps; ++i)
         if (H->red_f[i * 2] > -INFINITY) S += H->red_f[i * 2 + 1] * fast_exp2((H->red_f[i * 2] - M) * kLog2e);
-    H->stats.kmax = a;
-    H->stats.kmin = b;
-    H->stats.kminf = c;
-    H->stats.bad = d;
-    H->stats.m = M;
-    H->stats.s = S;
+    CtaStats* dst = cluster_ptr(&H->all[cx.rank], 0);
+    dst->kmax = a;
+    dst->kminf = c;
+    dst->bad = d;
+    dst->m = M;
+    dst->s = S;
   }
 }
 
-// ---- COLLECT_RAW: raw keys in [lo, hi] -> leader list (sort key: ~key, id)
+// ---- COLLECT_RAW: raw keys >= lo -> leader list (sort key: ~key, id)
 __device__ void op_collect_raw(const Ctx& cx, const Plan& p) {
   const int nq = (cx.n4 + kThreads - 1) / kThreads * kThreads;
   for (int q = threadIdx.x; q < nq; q += kThreads) {
     const bool valid = q < cx.n4;
     const float4 v4 = valid ? cx.part4[q] : make_float4(0.f, 0.f, 0.f, 0.f);
     const float v[4] = {v4.x, v4.y, v4.z, v4.w};
+    uint32_t k[4];
+    bool any = false;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint32_t k = fkey(v[i]);
-      const bool pred = valid && k >= p.lo && k <= p.hi;
+      k[i] = fkey(v[i]);
+      any |= valid && k[i] >= p.lo;
+    }
+    if (!__any_sync(0xFFFFFFFFu, any)) continue;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const bool pred = valid && k[i] >= p.lo;
       const uint32_t gid = static_cast<uint32_t>(cx.g0 + 4 * q + i);
-      list_append(cx, pred, (static_cast<uint64_t>(~k) << 32) | gid);
-    }
-  }
-}
-
-// ---- COLLECT_X: survivors with x-key in [lo, hi] -> leader list (sort key: ~xkey, id)
-__device__ void op_collect_x(const Ctx& cx, const Plan& p) {
-  const int nq = (cx.n4 + kThreads - 1) / kThreads * kThreads;
-  for (int q = threadIdx.x; q < nq; q += kThreads) {
-    const bool valid = q < cx.n4;
-    const float4 v4 = valid ? cx.part4[q] : make_float4(0.f, 0.f, 0.f, 0.f);
-    const float v[4] = {v4.x, v4.y, v4.z, v4.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      bool pred = false;
-      uint32_t xk = 0;
-      const uint32_t k = fkey(v[i]);
-      if (valid && key_finite(k) && k >= p.raw_lo) {
-        const float x = scale_x(v[i], cx.T);
-        xk = fkey(x);
-        pred = x >= p.theta && xk >= p.lo && xk <= p.hi;
-      }
-      const uint32_t gid = static_cast<uint32_t>(cx.g0 + 4 * q + i);
-      list_append(cx, pred, (static_cast<uint64_t>(~xk) << 32) | gid);
-    }
-  }
-}
-
-// ---- MASS_HIST: float64 masses of survivors on 4096 x-key bins, and their sum
-__device__ void op_mass_hist(const Ctx& cx, const Plan& p) {
-  double* mass = reinterpret_cast<double*>(cx.scratch);
-  uint32_t* cnt = reinterpret_cast<uint32_t*>(cx.scratch + kHistBins * 8);
-  for (int i = threadIdx.x; i < kHistBins; i += kThreads) {
-    mass[i] = 0.0;
-    cnt[i] = 0;
-  }
-  __syncthreads();
-  const double m = p.m;
-  double z = 0.0;
-  for (int q = threadIdx.x; q < cx.n4; q += kThreads) {
-    const float4 v4 = cx.part4[q];
-    const float v[4] = {v4.x, v4.y, v4.z, v4.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint32_t k = fkey(v[i]);
-      if (key_finite(k) && k >= p.raw_lo) {
-        const float x = scale_x(v[i], cx.T);
-        if (x >= p.theta) {
-          const double e = exp(static_cast<double>(x) - m);
-          const uint32_t b = fkey(x) >> 20;
-          atomicAdd(&mass[b], e);
-          atomicAdd(&cnt[b], 1u);
-          z += e;
-        }
-      }
-    }
-  }
-  const double zt = block_sum_d(z, cx.H);
-  if (threadIdx.x == 0) cx.H->stats.z = zt;
-}
-
-// ---- NARROW_COUNT: counts of raw keys in [lo, hi] on 256 bins from the top
-__device__ void op_narrow_count(const Ctx& cx, const Plan& p) {
-  uint32_t* cnt = reinterpret_cast<uint32_t*>(cx.scratch);
-  for (int i = threadIdx.x; i < kSubBins; i += kThreads) cnt[i] = 0;
-  __syncthreads();
-  for (int q = threadIdx.x; q < cx.n4; q += kThreads) {
-    const float4 v4 = cx.part4[q];
-    const float v[4] = {v4.x, v4.y, v4.z, v4.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint32_t k = fkey(v[i]);
-      if (k >= p.lo && k <= p.hi) atomicAdd(&cnt[(p.hi - k) >> p.shift], 1u);
-    }
-  }
-}
-
-// ---- NARROW_MASS: masses and counts of survivor x-keys in [lo, hi] on 256 bins from the top
-__device__ void op_narrow_mass(const Ctx& cx, const Plan& p) {
-  double* mass = reinterpret_cast<double*>(cx.scratch);
-  uint32_t* cnt = reinterpret_cast<uint32_t*>(cx.scratch + kHistBins * 8);
-  for (int i = threadIdx.x; i < kSubBins; i += kThreads) {
-    mass[i] = 0.0;
-    cnt[i] = 0;
-  }
-  __syncthreads();
-  const double m = p.m;
-  for (int q = threadIdx.x; q < cx.n4; q += kThreads) {
-    const float4 v4 = cx.part4[q];
-    const float v[4] = {v4.x, v4.y, v4.z, v4.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint32_t k = fkey(v[i]);
-      if (key_finite(k) && k >= p.raw_lo) {
-        const float x = scale_x(v[i], cx.T);
-        const uint32_t xk = fkey(x);
-        if (x >= p.theta && xk >= p.lo && xk <= p.hi) {
-          const uint32_t b = (p.hi - xk) >> p.shift;
-          atomicAdd(&mass[b], exp(static_cast<double>(x) - m));
-          atomicAdd(&cnt[b], 1u);
-        }
-      }
+      list_append(cx, pred, (static_cast<uint64_t>(~k[i]) << 32) | gid);
     }
   }
 }
@@ -653,7 +659,6 @@ __device__ void op_next_max(const Ctx& cx, const Plan& p) {
       }
     }
   }
-  // block reduce (key desc, id asc); "none" is (0, INT_MAX)
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     const uint32_t ok = __shfl_xor_sync(0xFFFFFFFFu, bk, o);
@@ -678,17 +683,108 @@ __device__ void op_next_max(const Ctx& cx, const Plan& p) {
         k = H->red_u[i];
         id = H->red_i[i];
       }
-    H->stats.nm_key = k;
-    H->stats.nm_id = id;
+    CtaStats* dst = cluster_ptr(&H->all[cx.rank], 0);
+    dst->nm_key = k;
+    dst->nm_id = id;
   }
 }
 
-// ---- GUMBEL: argmax of x + g over kept elements (x >= theta), float64-exact
+// ---- NARROW_COUNT: counts of raw keys in [lo, hi] on 256 bins from the top
+__device__ void op_narrow_count(const Ctx& cx, const Plan& p) {
+  uint32_t* cnt = reinterpret_cast<uint32_t*>(cx.scratch);
+  for (int i = threadIdx.x; i < kSubBins; i += kThreads) cnt[i] = 0;
+  __syncthreads();
+  for (int q = threadIdx.x; q < cx.n4; q += kThreads) {
+    const float4 v4 = cx.part4[q];
+    const float v[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t k = fkey(v[i]);
+      if (k >= p.lo && k <= p.hi) atomicAdd(&cnt[(p.hi - k) >> p.shift], 1u);
+    }
+  }
+}
+
+// Fixed-point mass bins in the scratch area: hi[256], lo[256], cnt[256], edge[256].
+struct MassBins {
+  unsigned long long* hi;
+  unsigned long long* lo;
+  uint32_t* cnt;
+  uint32_t* edge;
+};
+__device__ __forceinline__ MassBins mass_bins(uint8_t* scratch) {
+  MassBins b;
+  b.hi = reinterpret_cast<unsigned long long*>(scratch);
+  b.lo = b.hi + kSubBins;
+  b.cnt = reinterpret_cast<uint32_t*>(b.lo + kSubBins);
+  b.edge = b.cnt + kSubBins;
+  return b;
+}
+__device__ __forceinline__ void clear_mass_bins(const MassBins& b) {
+  for (int i = threadIdx.x; i < kSubBins; i += kThreads) {
+    b.hi[i] = 0;
+    b.lo[i] = 0;
+    b.cnt[i] = 0;
+  }
+  __syncthreads();
+}
+__device__ __forceinline__ void add_mass(const MassBins& b, uint32_t bin, double e) {
+  unsigned long long hi, lo;
+  mass_fixed(e, hi, lo);
+  atomicAdd(&b.hi[bin], hi);
+  atomicAdd(&b.lo[bin], lo);
+  atomicAdd(&b.cnt[bin], 1u);
+}
+
+// ---- MASS: x = fl(l / T) written in place; survivors' masses on bins of
+// equal width in x below m (exact key edges), exact fixed point.
+__device__ void op_mass(const Ctx& cx, const Plan& p) {
+  const MassBins b = mass_bins(cx.scratch);
+  for (int j = threadIdx.x; j <= kMassBins; j += kThreads) b.edge[j] = mass_edge(p.m, p.step, j);
+  clear_mass_bins(b);
+  const double m = p.m;
+  const float inv_step = 1.0f / p.step;
+  const double* tab = cx.H->exp_tab;
+  for (int q = threadIdx.x; q < cx.n4; q += kThreads) {
+    float4 v4 = cx.part4[q];
+    float v[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float x = key_finite(fkey(v[i])) ? scale_x(v[i], cx.T) : -INFINITY;
+      v[i] = x;
+      if (x >= p.theta && x > -INFINITY)
+        add_mass(b, mass_bin(b.edge, p.m, inv_step, x, fkey(x)), exp_neg64(static_cast<double>(x) - m, tab));
+    }
+    cx.part4[q] = make_float4(v[0], v[1], v[2], v[3]);
+  }
+}
+
+// ---- NARROW_MASS: survivors' masses of x-keys in [lo, hi] on 256 bins from the top
+__device__ void op_narrow_mass(const Ctx& cx, const Plan& p) {
+  const MassBins b = mass_bins(cx.scratch);
+  clear_mass_bins(b);
+  const double m = p.m;
+  const double* tab = cx.H->exp_tab;
+  for (int q = threadIdx.x; q < cx.n4; q += kThreads) {
+    const float4 v4 = cx.part4[q];
+    const float v[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t xk = fkey(v[i]);
+      if (xk >= p.lo && xk <= p.hi && v[i] >= p.theta && v[i] > -INFINITY)
+        add_mass(b, (p.hi - xk) >> p.shift, exp_neg64(static_cast<double>(v[i]) - m, tab));
+    }
+  }
+}
+
+// ---- GUMBEL: argmax of x + g over kept elements (x >= theta), float64-exact;
+// the CTA's best is pushed into the leader's slot [rank].
 __device__ void op_gumbel(const Ctx& cx, const Plan& p) {
   Best b;
   b.init();
   const uint32_t k0 = static_cast<uint32_t>(cx.a->seed), k1 = static_cast<uint32_t>(cx.a->seed >> 32);
   constexpr float kGMax = 16.7f;  // > -log(-log(1 - 2^-24)) = 16.63: the largest noise value
+  const uint32_t raw_lo = p.part_is_x ? 0u : raw_prefilter(p.theta, cx.T);
   for (int q = threadIdx.x; q < cx.n4; q += kThreads) {
     const float4 v4 = cx.part4[q];
     const float v[4] = {v4.x, v4.y, v4.z, v4.w};
@@ -698,15 +794,16 @@ __device__ void op_gumbel(const Ctx& cx, const Plan& p) {
     float xmax = -INFINITY;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint32_t k = fkey(v[i]);
-      kept[i] = false;
       x[i] = -INFINITY;
-      if (key_finite(k) && k >= p.raw_lo) {
-        x[i] = scale_x(v[i], cx.T);
-        kept[i] = x[i] >= p.theta;
-        if (kept[i]) xmax = fmaxf(xmax, x[i]);
-        any |= kept[i];
+      if (p.part_is_x) {
+        x[i] = v[i];
+      } else {
+        const uint32_t k = fkey(v[i]);
+        if (key_finite(k) && k >= raw_lo) x[i] = scale_x(v[i], cx.T);
       }
+      kept[i] = x[i] >= p.theta && x[i] > -INFINITY;
+      if (kept[i]) xmax = fmaxf(xmax, x[i]);
+      any |= kept[i];
     }
     // no kept element of this group can beat the current best, whatever its noise
     if (!any || (b.valid && xmax + kGMax < b.s - score_tol(b.s))) continue;
@@ -714,16 +811,17 @@ __device__ void op_gumbel(const Ctx& cx, const Plan& p) {
     const uint4 w = philox4x32_10(make_uint4(static_cast<uint32_t>(gid0 >> 2), cx.pos, cx.req, 0u), k0, k1);
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-      if (kept[i]) b.offer(x[i], v[i], word_of(w, i), static_cast<int32_t>(gid0 + i));
+      if (kept[i]) b.offer(x[i], p.part_is_x ? 0.0f : v[i], word_of(w, i), static_cast<int32_t>(gid0 + i));
   }
   double sd = b.valid ? b.exact() : -INFINITY;
   int32_t id = b.valid ? b.id : 0x7FFFFFFF;
   float l = b.valid ? b.l : 0.0f;
   block_best(sd, id, l, cx.H);
   if (threadIdx.x == 0) {
-    cx.H->stats.best_sd = sd;
-    cx.H->stats.best_id = id;
-    cx.H->stats.best_l = l;
+    const uint32_t slot = mapa(smem_u32(&cx.H->best[cx.rank]), 0);
+    st_dsmem_u64(slot, static_cast<uint64_t>(__double_as_longlong(sd)));
+    st_dsmem_u32(slot + 8, static_cast<uint32_t>(id));
+    st_dsmem_u32(slot + 12, __float_as_uint(l));
   }
 }
 
@@ -738,31 +836,28 @@ __device__ __forceinline__ void write_plan_all(const Ctx& cx, const Plan& p) {
   }
 }
 
-__device__ __forceinline__ uint32_t remote_u32(const Ctx& cx, const void* local, uint32_t rank) {
-  return ld_dsmem_u32(mapa(smem_u32(local), rank));
-}
-
-// Scan the C CTAs' histograms (u32 counts, bin b at cnt[b]) from bin `top`
-// downward; find the bin where the running count reaches `rank`.  Sets
-// L.found_bin (or -1) and L.found_cum (count strictly above that bin).
-__device__ void find_rank_bin(const Ctx& cx, const uint32_t* cnt_local, int top, int nbins_desc,
-                              bool desc_from_top, uint32_t rank, LeaderState& L) {
-  // nbins_desc bins, visited in order j = 0.. : bin index = desc_from_top ? top - j : j
+// Scan the C CTAs' u32 histograms (bin b at cnt[b]); visit bins j = 0.. as
+// bin(j) = desc ? top - j : j; find the bin where the running count reaches
+// `rank`.  Sets L.found_bin (or -1), L.found_cum (count strictly before it)
+// and L.found_cnt (its count).
+__device__ void find_rank_bin(const Ctx& cx, const uint32_t* cnt_local, int top, int nbins, bool desc,
+                              uint32_t rank, LeaderState& L) {
   uint32_t cum = 0;
   if (threadIdx.x == 0) L.found_bin = -1;
   __syncthreads();
-  for (int base = 0; base < nbins_desc; base += kThreads) {
+  for (int base = 0; base < nbins; base += kThreads) {
     const int j = base + threadIdx.x;
     uint32_t c = 0;
-    if (j < nbins_desc) {
-      const int b = desc_from_top ? top - j : j;
-      for (uint32_t r = 0; r < cx.C; ++r) c += remote_u32(cx, cnt_local + b, r);
+    if (j < nbins) {
+      const int b = desc ? top - j : j;
+      c = cluster_sum(cx, cnt_local + b);
     }
     uint32_t tot;
     const uint32_t incl = block_scan_u(c, &tot, cx.H);
-    if (j < nbins_desc && c > 0 && cum + incl >= rank && cum + incl - c < rank) {
-      L.found_bin = desc_from_top ? top - j : j;
+    if (j < nbins && c > 0 && cum + incl >= rank && cum + incl - c < rank) {
+      L.found_bin = desc ? top - j : j;
       L.found_cum = cum + incl - c;
+      L.found_cnt = c;
     }
     cum += tot;
     __syncthreads();
@@ -771,112 +866,44 @@ __device__ void find_rank_bin(const Ctx& cx, const uint32_t* cnt_local, int top,
   __syncthreads();
 }
 
-__device__ void finalize_row(const Ctx& cx, LeaderState& L) {
+// Mass bins merged over the cluster; finds the last non-empty bin whose exact
+// mass strictly above (cum_above + bins before it) is < top_p * Z.  Sets
+// L.found_bin, L.found_hi / found_lo (mass above it) and L.found_cnt.
+__device__ void find_mass_bin(const Ctx& cx, int nbins, LeaderState& L) {
+  const MassBins b = mass_bins(cx.scratch);
+  const int j = threadIdx.x;
+  unsigned long long h = 0, l = 0;
+  uint32_t c = 0;
+  if (j < nbins) {
+    h = cluster_sum(cx, b.hi + j);
+    l = cluster_sum(cx, b.lo + j);
+    c = cluster_sum(cx, b.cnt + j);
+  }
+  unsigned long long ih = h, il = l;
+  block_scan_fixed(ih, il, cx.H);
+  // exact mass strictly above bin j
+  const unsigned long long bh = L.cum_hi + ih - h, bl = L.cum_lo + il - l;
+  const double pz = static_cast<double>(L.top_p) * fixed_to_double(L.z_hi, L.z_lo);
+  const bool cand = j < nbins && c > 0 && fixed_to_double(bh, bl) < pz;
+  const int best = block_max_i(cand ? j : -1, cx.H);
+  if (threadIdx.x == 0) L.found_bin = -1;
+  __syncthreads();
+  if (best >= 0 && j == best) {
+    L.found_bin = j;
+    L.found_hi = bh;
+    L.found_lo = bl;
+    L.found_cnt = c;
+  }
+  __syncthreads();
+}
+
+__device__ void write_outputs(const Ctx& cx, LeaderState& L) {
   if (threadIdx.x == 0) {
     const SampleArgs& a = *cx.a;
     a.token_ids[cx.row] = L.token;
     a.token_logprob[cx.row] = L.token_l - L.lse;
     a.row_flags[cx.row] = 0;
   }
-}
-
-// Exact top-p on the leader's sorted list of survivors (entries 0..ns-1, x
-// descending), with `cum_above` mass strictly above the list.  Returns via L:
-// sstar (last kept group start) and send (kept prefix length).
-__device__ void list_top_p(const Ctx& cx, LeaderState& L, int ns, double Z, double cum_above, bool x_keys) {
-  const uint64_t* list = cx.list;
-  const double m = L.m;
-  constexpr int kPer = kListCap / kThreads;  // entries per thread (contiguous)
-  double e[kPer];
-  double tsum = 0.0;
-  const int j0 = threadIdx.x * kPer;
-#pragma unroll
-  for (int i = 0; i < kPer; ++i) {
-    const int j = j0 + i;
-    e[i] = 0.0;
-    if (j < ns) {
-      const uint32_t key = ~static_cast<uint32_t>(list[j] >> 32);
-      const float x = x_keys ? key_value(key) : scale_x(key_value(key), L.T);
-      e[i] = exp(static_cast<double>(x) - m);
-    }
-    tsum += e[i];
-  }
-  double total;
-  const double incl = block_scan_d(tsum, &total, cx.H);
-  if (Z <= 0.0) Z = total;  // survivors all listed: Z is their sum
-  const double pz = static_cast<double>(L.top_p);
-  double run = incl - tsum;  // exclusive prefix of this thread's first entry
-  int sstar = -1;
-#pragma unroll
-  for (int i = 0; i < kPer; ++i) {
-    const int j = j0 + i;
-    if (j < ns) {
-      const uint32_t kj = ~static_cast<uint32_t>(list[j] >> 32);
-      bool start = j == 0;
-      if (!start) {
-        const uint32_t kp = ~static_cast<uint32_t>(list[j - 1] >> 32);
-        start = x_keys ? kp != kj : scale_x(key_value(kp), L.T) != scale_x(key_value(kj), L.T);
-      }
-      if (start && (cum_above + run) / Z < pz) sstar = j;
-    }
-    run += e[i];
-  }
-  sstar = block_max_i(sstar, cx.H);
-  if (sstar < 0) sstar = 0;
-  // end of the kept group: the next group start after sstar
-  const uint32_t ks = ~static_cast<uint32_t>(list[sstar] >> 32);
-  const float xs = x_keys ? key_value(ks) : scale_x(key_value(ks), L.T);
-  int send = ns;
-  for (int j = threadIdx.x; j < ns; j += kThreads) {
-    if (j > sstar) {
-      const uint32_t kj = ~static_cast<uint32_t>(list[j] >> 32);
-      const float xj = x_keys ? key_value(kj) : scale_x(key_value(kj), L.T);
-      if (xj != xs) send = min(send, j);
-    }
-  }
-  send = block_min_i(send, cx.H);
-  if (threadIdx.x == 0) {
-    L.sstar = sstar;
-    L.send = send;
-    L.theta_p = xs;
-  }
-  __syncthreads();
-}
-
-// Gumbel draw over list entries [0, n) (keys raw or x); result into L.token / L.token_l.
-__device__ void list_gumbel(const Ctx& cx, LeaderState& L, int n, bool x_keys) {
-  Best b;
-  b.init();
-  const uint32_t k0 = static_cast<uint32_t>(cx.a->seed), k1 = static_cast<uint32_t>(cx.a->seed >> 32);
-  for (int j = threadIdx.x; j < n; j += kThreads) {
-    const uint64_t e = cx.list[j];
-    const uint32_t key = ~static_cast<uint32_t>(e >> 32);
-    const int32_t id = static_cast<int32_t>(e & 0xFFFFFFFFu);
-    float x, l;
-    if (x_keys) {
-      x = key_value(key);
-      l = -INFINITY;  // raw logit looked up below
-    } else {
-      l = key_value(key);
-      x = scale_x(l, L.T);
-    }
-    const uint4 w = philox4x32_10(make_uint4(static_cast<uint32_t>(id) >> 2, cx.pos, cx.req, 0u), k0, k1);
-    b.offer(x, l, word_of(w, id & 3), id);
-  }
-  double sd = b.valid ? b.exact() : -INFINITY;
-  int32_t id = b.valid ? b.id : 0x7FFFFFFF;
-  float l = b.valid ? b.l : 0.0f;
-  block_best(sd, id, l, cx.H);
-  if (threadIdx.x == 0) {
-    const bool ok = id >= 0 && id < cx.a->V;  // a kept set is never empty; guard anyway
-    L.token = ok ? id : -1;
-    if (x_keys && ok) {
-      const int s = id / cx.a->V_s, j = id - s * cx.a->V_s;
-      l = cx.a->slices[s][static_cast<size_t>(cx.row) * cx.a->V_s + j];
-    }
-    L.token_l = ok ? l : __int_as_float(0x7FC00000);
-  }
-  __syncthreads();
 }
 
 __device__ void write_topn_from_list(const Ctx& cx, const LeaderState& L) {
@@ -903,102 +930,179 @@ __device__ void sort_list(const Ctx& cx, int count) {
   bitonic_sort(cx.list, n);
 }
 
-// Plans the narrowing of the top-k rank search inside [lo, hi].
-__device__ Plan narrow_count_plan(LeaderState& L) {
-  Plan p{};
-  p.op = OP_NARROW_COUNT;
-  p.lo = L.nlo;
-  p.hi = L.nhi;
-  const uint32_t width = L.nhi - L.nlo;
-  const int bits = width == 0 ? 0 : 32 - __clz(width);
-  p.shift = bits > 8 ? bits - 8 : 0;
-  __syncthreads();
-  if (threadIdx.x == 0) L.nshift = p.shift;
-  __syncthreads();
-  return p;
-}
-__device__ Plan narrow_mass_plan(LeaderState& L) {
-  Plan p{};
-  p.op = OP_NARROW_MASS;
-  p.lo = L.nlo;
-  p.hi = L.nhi;
-  const uint32_t width = L.nhi - L.nlo;
-  const int bits = width == 0 ? 0 : 32 - __clz(width);
-  p.shift = bits > 8 ? bits - 8 : 0;
-  __syncthreads();
-  if (threadIdx.x == 0) L.nshift = p.shift;
-  __syncthreads();
-  p.theta = L.theta_k;
-  p.raw_lo = L.surv_raw_lo;
-  p.m = L.m;
-  return p;
-}
-
-// After the top-n / argmax is known: start the sampling part of the row.
-// Returns the next plan (or OP_END after finishing the row).
-__device__ Plan plan_sampling(const Ctx& cx, LeaderState& L);
-
-__device__ Plan plan_after_theta_k(const Ctx& cx, LeaderState& L) {
-  // survivors: finite with x >= theta_k (theta_k = -inf when top-k is off)
-  const uint32_t surv_raw_lo = raw_prefilter(L.theta_k, L.T);
-  __syncthreads();
-  if (threadIdx.x == 0) L.surv_raw_lo = surv_raw_lo;
-  __syncthreads();
-  Plan p{};
+// List resolution for a sampling row: the sorted raw list holds every top-k
+// survivor (and the top-n).  top-k threshold, exact top-p, the draw.
+__device__ void list_sample_tail(const Ctx& cx, LeaderState& L, int count) {
+  const uint64_t* list = cx.list;
+  // survivors: the prefix with x >= theta_k (x finite)
+  float theta_k = -INFINITY;
+  if (L.r_k > 0) theta_k = scale_x(key_value(~static_cast<uint32_t>(list[L.r_k - 1] >> 32)), L.T);
+  int ns = 0;
+  for (int j = threadIdx.x; j < count; j += kThreads) {
+    const float x = scale_x(key_value(~static_cast<uint32_t>(list[j] >> 32)), L.T);
+    if (x >= theta_k && x > -INFINITY) ns = max(ns, j + 1);
+  }
+  ns = block_max_i(ns, cx.H);
+  int nk = ns;
   if (L.top_p < 1.0f) {
-    p.op = OP_MASS_HIST;
+    // exact top-p over the survivors: float64 masses, fixed-order prefix sums
+    constexpr int kPer = kListCap / kThreads;
+    double e[kPer];
+    double tsum = 0.0;
+    const int j0 = threadIdx.x * kPer;
+    const double m = static_cast<double>(L.m);
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int j = j0 + i;
+      e[i] = 0.0;
+      if (j < ns)
+        e[i] = exp_neg64(static_cast<double>(scale_x(key_value(~static_cast<uint32_t>(list[j] >> 32)), L.T)) - m,
+                         cx.H->exp_tab);
+      tsum += e[i];
+    }
+    double Z;
+    const double incl = block_scan_d(tsum, &Z, cx.H);
+    const double pz = static_cast<double>(L.top_p);
+    double run = incl - tsum;
+    int sstar = -1;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int j = j0 + i;
+      if (j < ns) {
+        const float xj = scale_x(key_value(~static_cast<uint32_t>(list[j] >> 32)), L.T);
+        const bool start = j == 0 || scale_x(key_value(~static_cast<uint32_t>(list[j - 1] >> 32)), L.T) != xj;
+        if (start && run / Z < pz) sstar = j;
+      }
+      run += e[i];
+    }
+    sstar = max(block_max_i(sstar, cx.H), 0);
+    const float xs = scale_x(key_value(~static_cast<uint32_t>(list[sstar] >> 32)), L.T);
+    int send = ns;
+    for (int j = sstar + 1 + threadIdx.x; j < ns; j += kThreads)
+      if (scale_x(key_value(~static_cast<uint32_t>(list[j] >> 32)), L.T) != xs) send = min(send, j);
+    nk = block_min_i(send, cx.H);
+  }
+  // the draw over the kept prefix
+  Best b;
+  b.init();
+  const uint32_t k0 = static_cast<uint32_t>(cx.a->seed), k1 = static_cast<uint32_t>(cx.a->seed >> 32);
+  for (int j = threadIdx.x; j < nk; j += kThreads) {
+    const uint64_t e = list[j];
+    const float l = key_value(~static_cast<uint32_t>(e >> 32));
+    const int32_t id = static_cast<int32_t>(e & 0xFFFFFFFFu);
+    const uint4 w = philox4x32_10(make_uint4(static_cast<uint32_t>(id) >> 2, cx.pos, cx.req, 0u), k0, k1);
+    b.offer(scale_x(l, L.T), l, word_of(w, id & 3), id);
+  }
+  double sd = b.valid ? b.exact() : -INFINITY;
+  int32_t id = b.valid ? b.id : 0x7FFFFFFF;
+  float l = b.valid ? b.l : 0.0f;
+  block_best(sd, id, l, cx.H);
+  if (threadIdx.x == 0) {
+    const bool ok = id >= 0 && id < cx.a->V;
+    L.token = ok ? id : -1;
+    L.token_l = ok ? l : __int_as_float(0x7FC00000);
+  }
+  __syncthreads();
+}
+
+__device__ Plan narrow_plan(LeaderState& L, uint32_t op) {
+  Plan p{};
+  p.op = op;
+  p.lo = L.nlo;
+  p.hi = L.nhi;
+  const uint32_t width = L.nhi - L.nlo;
+  const int bits = width == 0 ? 0 : 32 - __clz(width);
+  p.shift = bits > 8 ? bits - 8 : 0;
+  p.theta = L.theta_k;
+  p.m = L.m;
+  p.part_is_x = L.part_is_x;
+  __syncthreads();
+  if (threadIdx.x == 0) L.nshift = p.shift;
+  __syncthreads();
+  return p;
+}
+
+// Narrows [nlo, nhi] to its sub-bin j (bins of 2^nshift keys from the top).
+__device__ __forceinline__ void narrow_range(LeaderState& L, int j) {
+  const uint32_t hi = L.nhi - (static_cast<uint32_t>(j) << L.nshift);
+  const uint32_t span = (static_cast<uint32_t>(j + 1) << L.nshift) - 1u;
+  const uint32_t lo = (L.nhi - L.nlo) > span ? L.nhi - span : L.nlo;
+  L.nlo = lo;
+  L.nhi = hi;
+}
+
+// Survivors known (theta_k): masses for top-p, or the draw directly.
+__device__ Plan plan_after_theta_k(const Ctx& cx, LeaderState& L) {
+  Plan p{};
+  __syncthreads();
+  if (L.top_p < 1.0f) {
+    p.op = OP_MASS;
     p.theta = L.theta_k;
-    p.raw_lo = L.surv_raw_lo;
     p.m = L.m;
-    if (threadIdx.x == 0) L.phase = PH_AFTER_MASS;
+    // bins span [x_low, m], x_low the smallest survivor x (at most 96 below m)
+    const float x_low = fmaxf(L.theta_k, scale_x(key_value(L.kminf), L.T));
+    float width = fminf(__fsub_rn(L.m, x_low), 96.0f);
+    if (!(width > 0.0f)) width = 1.0f;
+    p.step = width / static_cast<float>(kMassBins);
+    if (threadIdx.x == 0) {
+      L.phase = PH_AFTER_MASS;
+      L.part_is_x = 1;
+    }
   } else {
     p.op = OP_GUMBEL;
     p.theta = L.theta_k;
-    p.raw_lo = L.surv_raw_lo;
+    p.part_is_x = L.part_is_x;
     if (threadIdx.x == 0) L.phase = PH_AFTER_GUMBEL;
   }
+  __syncthreads();
   return p;
 }
 
-__device__ Plan plan_sampling(const Ctx& cx, LeaderState& L) {
-  Plan p{};
-  if (L.greedy) {
-    finalize_row(cx, L);
-    p.op = OP_END;
-    return p;
-  }
+// After the top-n is known (listed or extracted): the sampling part of a streamed row.
+__device__ Plan plan_stream_sampling(const Ctx& cx, LeaderState& L) {
+  __syncthreads();
   if (L.r_k == 0) {
-    __syncthreads();
     if (threadIdx.x == 0) L.theta_k = -INFINITY;
-    __syncthreads();
     return plan_after_theta_k(cx, L);
   }
-  // top-k rank search by narrowing inside the level-1 bin found at the start
-  return narrow_count_plan(L);
+  if (threadIdx.x == 0) L.phase = PH_TOPK_NARROW;
+  return narrow_plan(L, OP_NARROW_COUNT);
 }
 
-__device__ Plan leader_step(const Ctx& cx) {
+__device__ Plan gumbel_plan(LeaderState& L) {
+  __syncthreads();  // theta_p was just written by thread 0
+  Plan p{};
+  p.op = OP_GUMBEL;
+  p.theta = fmaxf(L.theta_k, L.theta_p);
+  p.part_is_x = 1;
+  __syncthreads();
+  if (threadIdx.x == 0) L.phase = PH_AFTER_GUMBEL;
+  __syncthreads();
+  return p;
+}
+
+__device__ Plan leader_step(const Ctx& cx, uint32_t& tail) {
   LeaderState& L = cx.H->L;
   const SampleArgs& a = *cx.a;
   Plan p{};
   p.op = OP_END;
+  tail = TAIL_NONE;
   switch (L.phase) {
     case PH_START: {
       if (threadIdx.x == 0) {
-        uint32_t kmax = 0, kmin = 0xFFFFFFFFu, kminf = 0xFFFFFFFFu, bad = 0;
+        uint32_t kmax = 0, kminf = 0xFFFFFFFFu, bad = 0;
         float M = -INFINITY;
         for (uint32_t r = 0; r < cx.C; ++r) {
-          bad |= remote_u32(cx, &cx.H->stats.bad, r);
-          kmax = max(kmax, remote_u32(cx, &cx.H->stats.kmax, r));
-          kmin = min(kmin, remote_u32(cx, &cx.H->stats.kmin, r));
-          kminf = min(kminf, remote_u32(cx, &cx.H->stats.kminf, r));
-          M = fmaxf(M, __uint_as_float(remote_u32(cx, &cx.H->stats.m, r)));
+          const CtaStats& st = cx.H->all[r];
+          bad |= st.bad;
+          kmax = max(kmax, st.kmax);
+          kminf = min(kminf, st.kminf);
+          M = fmaxf(M, st.m);
         }
         float S = 0.0f;
         for (uint32_t r = 0; r < cx.C; ++r) {
-          const float mr = __uint_as_float(remote_u32(cx, &cx.H->stats.m, r));
-          const float sr = __uint_as_float(remote_u32(cx, &cx.H->stats.s, r));
-          if (mr > -INFINITY) S += sr * fast_exp2((mr - M) * 1.4426950408889634f);
+          const CtaStats& st = cx.H->all[r];
+          if (st.m > -INFINITY) S += st.s * fast_exp2((st.m - M) * 1.4426950408889634f);
         }
         const vsl_row_params prm = a.params[cx.row];
         uint32_t flags = 0;
@@ -1028,8 +1132,9 @@ __device__ Plan leader_step(const Ctx& cx) {
         L.m = L.greedy ? 0.0f : scale_x(M, prm.temperature);
         L.theta_k = -INFINITY;
         L.theta_p = -INFINITY;
-        L.topn_done = false;
+        L.part_is_x = 0;
         L.token = -1;
+        L.cum_hi = L.cum_lo = 0;
       }
       __syncthreads();
       if (L.flags) {
@@ -1044,62 +1149,63 @@ __device__ Plan leader_step(const Ctx& cx) {
         }
         break;
       }
-      // level-1 search: bins of the raw histogram from the max key downward
+      // raw-histogram bins from the max key downward
       const uint32_t* hist = reinterpret_cast<const uint32_t*>(cx.scratch);
       const int top = static_cast<int>(L.kmax >> 20);
       find_rank_bin(cx, hist, top, top + 1, true, static_cast<uint32_t>(L.r_n), L);
-      const int bn = L.found_bin;
-      const uint32_t cnt_n_incl = L.found_cum + (bn >= 0 ? [&] {
-        uint32_t c = 0;
-        for (uint32_t r = 0; r < cx.C; ++r) c += remote_u32(cx, hist + bn, r);
-        return c;
-      }() : 0u);
-      int bk = -1;
-      uint32_t cnt_k_incl = 0, cum_k = 0;
+      const int bn = max(L.found_bin, 0);
+      const uint32_t need_n = L.found_cum + L.found_cnt;
+      int bk = 0;
+      uint32_t need_k = 0, cum_k = 0;
       if (L.r_k > 0) {
         find_rank_bin(cx, hist, top, top + 1, true, static_cast<uint32_t>(L.r_k), L);
-        bk = L.found_bin;
+        bk = max(L.found_bin, 0);
         cum_k = L.found_cum;
-        uint32_t c = 0, cbelow = 0;
-        for (uint32_t r = 0; r < cx.C; ++r) {
-          c += remote_u32(cx, hist + bk, r);
-          if (bk > 0) cbelow += remote_u32(cx, hist + bk - 1, r);
-        }
-        cnt_k_incl = cum_k + c + cbelow;
+        need_k = L.found_cum + L.found_cnt;
       }
-      __syncthreads();
       if (threadIdx.x == 0) {
-        uint32_t lo = static_cast<uint32_t>(bn) << 20;
-        uint32_t need = cnt_n_incl;
-        L.k_listed = false;
-        if (L.r_k > 0 && cnt_k_incl <= static_cast<uint32_t>(kListCap)) {
-          const uint32_t lo_k = bk > 0 ? static_cast<uint32_t>(bk - 1) << 20 : 0u;
-          lo = min(lo, lo_k);
-          need = max(need, cnt_k_incl);
-          L.k_listed = true;
+        const uint32_t lo_n = static_cast<uint32_t>(bn) << 20;
+        L.topn_listed = need_n <= static_cast<uint32_t>(kListCap);
+        uint32_t lo = lo_n;
+        int mode = 0;  // 0 = stream, 1 = list greedy, 2 = list sample
+        if (L.greedy) {
+          mode = L.topn_listed ? 1 : 0;
+        } else if (L.r_k > 0 && L.topn_listed && need_k <= static_cast<uint32_t>(kListCap)) {
+          // every survivor is listed when no value below the k-th key's bin can
+          // scale to that bin's lowest x: adjacent keys at the boundary stay apart
+          const uint32_t lo_k = static_cast<uint32_t>(bk) << 20;
+          bool ok = lo_k <= kKeyNegInf + 1;
+          if (!ok) ok = scale_x(key_value(lo_k - 1), L.T) < scale_x(key_value(lo_k), L.T);
+          if (ok) {
+            mode = 2;
+            lo = min(lo_n, lo_k);
+          }
         }
         // narrowing state for a top-k search outside the list
-        L.nlo = static_cast<uint32_t>(max(bk, 0)) << 20;
+        L.nlo = static_cast<uint32_t>(bk) << 20;
         L.nhi = L.nlo | 0xFFFFFu;
         L.nrank = static_cast<uint32_t>(L.r_k) - cum_k;
-        if (need <= static_cast<uint32_t>(kListCap)) {
-          L.collect_lo = lo;
-          cx.H->list_count = 0;
-          L.phase = PH_AFTER_COLLECT_RAW;
-        } else {
-          // top-n not listable (dense or tied top bins): extract it one by one
-          L.topn_count = 0;
-          L.prev_key = 0xFFFFFFFFu;
-          L.prev_id = -1;
-          L.k_listed = false;
-          L.phase = PH_TOPN_NEXT_MAX;
+        L.mode = mode;
+        L.collect_lo = lo;
+        cx.H->list_count = 0;
+        if (mode == 0) {
+          if (L.topn_listed) {
+            L.phase = PH_AFTER_TOPN_COLLECT;
+          } else {
+            L.topn_count = 0;
+            L.prev_key = 0xFFFFFFFFu;
+            L.prev_id = -1;
+            L.phase = PH_TOPN_NEXT_MAX;
+          }
         }
       }
       __syncthreads();
-      if (L.phase == PH_AFTER_COLLECT_RAW) {
+      if (L.mode != 0 || L.topn_listed) {
         p.op = OP_COLLECT_RAW;
         p.lo = L.collect_lo;
-        p.hi = 0xFFFFFFFFu;
+        if (L.mode == 1) tail = TAIL_LIST_GREEDY;
+        if (L.mode == 2) tail = TAIL_LIST_SAMPLE;
+        p.last = L.mode != 0;
       } else {
         p.op = OP_NEXT_MAX;
         p.nm_key = 0xFFFFFFFFu;
@@ -1114,8 +1220,8 @@ __device__ Plan leader_step(const Ctx& cx) {
         uint32_t bk = 0;
         int32_t bid = 0x7FFFFFFF;
         for (uint32_t r = 0; r < cx.C; ++r) {
-          const uint32_t k = remote_u32(cx, &cx.H->stats.nm_key, r);
-          const int32_t id = static_cast<int32_t>(remote_u32(cx, &cx.H->stats.nm_id, r));
+          const uint32_t k = cx.H->all[r].nm_key;
+          const int32_t id = cx.H->all[r].nm_id;
           if (k > bk || (k == bk && id < bid)) {
             bk = k;
             bid = id;
@@ -1141,264 +1247,92 @@ __device__ Plan leader_step(const Ctx& cx) {
         p.nm_id = L.prev_id;
         break;
       }
-      if (threadIdx.x == 0) {
-        L.topn_done = true;
-        if (L.r_k > 0) L.phase = PH_TOPK_NARROW;
+      if (L.greedy) {
+        write_outputs(cx, L);
+        break;
       }
-      __syncthreads();
-      p = plan_sampling(cx, L);
+      p = plan_stream_sampling(cx, L);
       break;
     }
 
-    case PH_AFTER_COLLECT_RAW: {
-      const int count = min(static_cast<int>(cx.H->list_count), kListCap);
-      sort_list(cx, count);
-      write_topn_from_list(cx, L);
-      if (L.greedy) {
-        if (threadIdx.x == 0) {
-          L.token = static_cast<int32_t>(cx.list[0] & 0xFFFFFFFFu);
-          L.token_l = key_value(~static_cast<uint32_t>(cx.list[0] >> 32));
-        }
-        __syncthreads();
-        finalize_row(cx, L);
-        break;
-      }
-      if (L.r_k > 0 && L.k_listed) {
-        // theta_k from the list; all survivors are listed iff the largest
-        // unlisted logit scales strictly below theta_k
-        const uint32_t kk = ~static_cast<uint32_t>(cx.list[L.r_k - 1] >> 32);
-        const float theta_k = scale_x(key_value(kk), L.T);
-        bool all_listed = true;
-        if (L.collect_lo > kKeyNegInf + 1) {
-          const float l_nc = key_value(L.collect_lo - 1);
-          all_listed = scale_x(l_nc, L.T) < theta_k;
-        }
-        if (threadIdx.x == 0) L.theta_k = theta_k;
-        __syncthreads();
-        if (all_listed) {
-          // survivors: the list prefix with x >= theta_k
-          int ns = 0;
-          for (int j = threadIdx.x; j < count; j += kThreads) {
-            const float x = scale_x(key_value(~static_cast<uint32_t>(cx.list[j] >> 32)), L.T);
-            if (x >= theta_k && x > -INFINITY) ns = max(ns, j + 1);
-          }
-          ns = block_max_i(ns, cx.H);
-          int nk = ns;
-          if (L.top_p < 1.0f) {
-            list_top_p(cx, L, ns, 0.0, 0.0, false);
-            nk = L.send;
-          }
-          list_gumbel(cx, L, nk, false);
-          finalize_row(cx, L);
-          break;
-        }
-        p = plan_after_theta_k(cx, L);
-        break;
-      }
-      if (L.r_k > 0) {
-        if (threadIdx.x == 0) L.phase = PH_TOPK_NARROW;
-        __syncthreads();
-        p = narrow_count_plan(L);
-        break;
-      }
-      if (threadIdx.x == 0) L.theta_k = -INFINITY;
-      __syncthreads();
-      p = plan_after_theta_k(cx, L);
+    case PH_AFTER_TOPN_COLLECT: {
+      // the top-n list stays in the leader's memory and is finished in its tail
+      p = plan_stream_sampling(cx, L);
       break;
     }
 
     case PH_TOPK_NARROW: {
-      // merge the 256 narrowing bins; find the rank's sub-bin
       const uint32_t* cnt = reinterpret_cast<const uint32_t*>(cx.scratch);
       const int nb = static_cast<int>(((L.nhi - L.nlo) >> L.nshift) + 1);
       find_rank_bin(cx, cnt, 0, nb, false, L.nrank, L);
       if (threadIdx.x == 0) {
-        const int j = max(L.found_bin, 0);
-        const uint32_t hi = L.nhi - (static_cast<uint32_t>(j) << L.nshift);
-        const uint32_t lo_c = (static_cast<uint32_t>(j + 1) << L.nshift) - 1;
-        const uint32_t lo = (L.nhi - L.nlo) > lo_c ? L.nhi - lo_c : L.nlo;
+        narrow_range(L, max(L.found_bin, 0));
         L.nrank -= L.found_cum;
-        L.nlo = lo;
-        L.nhi = hi;
       }
       __syncthreads();
       if (L.nlo != L.nhi) {
-        p = narrow_count_plan(L);
+        p = narrow_plan(L, OP_NARROW_COUNT);
         break;
       }
       if (threadIdx.x == 0) L.theta_k = scale_x(key_value(L.nlo), L.T);
-      __syncthreads();
       p = plan_after_theta_k(cx, L);
       break;
     }
 
     case PH_AFTER_MASS: {
-      // Z from the CTAs' deterministic sums; find the cut bin on the x-key histogram
-      if (threadIdx.x == 0) {
-        double Z = 0.0;
-        for (uint32_t r = 0; r < cx.C; ++r) Z += ld_dsmem_f64(mapa(smem_u32(&cx.H->stats.z), r));
-        L.Z = Z;
-        L.found_bin = -1;
-        L.last_bin = -1;
-      }
-      __syncthreads();
-      const double* mass = reinterpret_cast<const double*>(cx.scratch);
-      const uint32_t* cnt = reinterpret_cast<const uint32_t*>(cx.scratch + kHistBins * 8);
-      const int top = static_cast<int>(fkey(L.m) >> 20);
-      const double pz = static_cast<double>(L.top_p) * L.Z;
-      double cum = 0.0;
-      uint32_t cumc = 0;
-      for (int base = 0; base <= top; base += kThreads) {
-        const int j = base + threadIdx.x;
-        double mj = 0.0;
-        uint32_t cj = 0;
-        if (j <= top) {
-          for (uint32_t r = 0; r < cx.C; ++r) {
-            mj += ld_dsmem_f64(mapa(smem_u32(mass + (top - j)), r));
-            cj += remote_u32(cx, cnt + (top - j), r);
-          }
+      // exact total mass, then the log bin holding the cut
+      {
+        const MassBins b = mass_bins(cx.scratch);
+        const int j = threadIdx.x;
+        unsigned long long h = 0, l = 0;
+        if (j < kMassBins) {
+          h = cluster_sum(cx, b.hi + j);
+          l = cluster_sum(cx, b.lo + j);
         }
-        double mt;
-        uint32_t ct;
-        const double mincl = block_scan_d(mj, &mt, cx.H);
-        const uint32_t cincl = block_scan_u(cj, &ct, cx.H);
-        const double before = cum + mincl - mj;
-        if (cj > 0 && before < pz && cum + mincl >= pz) {
-          L.found_bin = top - j;
-          L.found_mass = before;
-          L.found_cum = cumc + cincl;  // elements from the top through this bin
+        block_scan_fixed(h, l, cx.H);
+        if (j == kThreads - 1) {
+          L.z_hi = h;
+          L.z_lo = l;
         }
-        const int ln = block_max_i(cj > 0 ? j : -1, cx.H);
-        if (ln >= 0 && threadIdx.x == ln - base) {
-          L.last_bin = top - ln;
-          L.last_before = before;
-          L.last_cumc = cumc + cincl;
-        }
-        cum += mt;
-        cumc += ct;
         __syncthreads();
-        if (L.found_bin >= 0) break;
       }
-      __syncthreads();
+      find_mass_bin(cx, kMassBins, L);
       if (threadIdx.x == 0) {
-        if (L.found_bin < 0) {
-          // rounding left pZ beyond the last bin: the cut is in the last non-empty bin
-          L.found_bin = L.last_bin;
-          L.found_mass = L.last_before;
-          L.found_cum = L.last_cumc;
-        }
-        L.nlo = static_cast<uint32_t>(L.found_bin) << 20;
-        L.nhi = L.nlo | 0xFFFFFu;
-        L.cum_above = L.found_mass;
-        L.x_from_top = L.found_cum <= static_cast<uint32_t>(kListCap);
-        if (L.x_from_top) {
-          // everything from the top through the cut bin fits: list it and finish exactly
-          L.cum_above = 0.0;
-          cx.H->list_count = 0;
-          L.phase = PH_AFTER_COLLECT_X;
-        } else {
-          L.phase = PH_MASS_NARROW;
-        }
+        const int bin = max(L.found_bin, 0);
+        // bin j holds x-keys in (edge[j + 1], edge[j]]; the last bin is open below
+        const uint32_t* edge = mass_bins(cx.scratch).edge;
+        L.nhi = edge[bin];
+        L.nlo = bin == kMassBins - 1 ? 0u : edge[bin + 1] + 1u;
+        L.cum_hi = L.found_hi;
+        L.cum_lo = L.found_lo;
+        L.phase = PH_MASS_NARROW;
       }
       __syncthreads();
-      if (L.x_from_top) {
-        p.op = OP_COLLECT_X;
-        p.lo = L.nlo;
-        p.hi = 0xFFFFFFFFu;
-        p.theta = L.theta_k;
-        p.raw_lo = L.surv_raw_lo;
-        p.m = L.m;
+      if (L.nlo == L.nhi) {
+        if (threadIdx.x == 0) L.theta_p = key_value(L.nlo);
+        p = gumbel_plan(L);
         break;
       }
-      p = narrow_mass_plan(L);
+      p = narrow_plan(L, OP_NARROW_MASS);
       break;
     }
 
     case PH_MASS_NARROW: {
-      const double* mass = reinterpret_cast<const double*>(cx.scratch);
-      const uint32_t* cnt = reinterpret_cast<const uint32_t*>(cx.scratch + kHistBins * 8);
       const int nb = static_cast<int>(((L.nhi - L.nlo) >> L.nshift) + 1);
-      const double pz = static_cast<double>(L.top_p) * L.Z;
-      if (threadIdx.x == 0) L.found_bin = -1;
-      __syncthreads();
-      const int j = threadIdx.x;
-      double mj = 0.0;
-      uint32_t cj = 0;
-      if (j < nb) {
-        for (uint32_t r = 0; r < cx.C; ++r) {
-          mj += ld_dsmem_f64(mapa(smem_u32(mass + j), r));
-          cj += remote_u32(cx, cnt + j, r);
-        }
-      }
-      double mt;
-      const double mincl = block_scan_d(mj, &mt, cx.H);
-      const double before = L.cum_above + mincl - mj;
-      // last non-empty sub-bin whose mass above is < pZ
-      int cand = (j < nb && cj > 0 && before < pz) ? j : -1;
-      cand = block_max_i(cand, cx.H);
-      if (cand < 0) cand = 0;
-      if (threadIdx.x == cand) {
-        L.found_bin = cand;
-        L.found_mass = before;
-        L.found_cum = cj;
-      }
-      __syncthreads();
+      find_mass_bin(cx, nb, L);
       if (threadIdx.x == 0) {
-        const uint32_t jj = static_cast<uint32_t>(L.found_bin);
-        const uint32_t hi = L.nhi - (jj << L.nshift);
-        const uint32_t lo_c = ((jj + 1) << L.nshift) - 1;
-        const uint32_t lo = (L.nhi - L.nlo) > lo_c ? L.nhi - lo_c : L.nlo;
-        L.nlo = lo;
-        L.nhi = hi;
-        L.cum_above = L.found_mass;
+        narrow_range(L, max(L.found_bin, 0));
+        L.cum_hi = L.found_hi;
+        L.cum_lo = L.found_lo;
       }
       __syncthreads();
-      if (L.nlo == L.nhi) {
-        // one x value: every survivor with it has the same mass above (< pZ): kept
-        Plan g{};
-        g.op = OP_GUMBEL;
-        g.theta = fmaxf(L.theta_k, key_value(L.nlo));
-        g.raw_lo = raw_prefilter(g.theta, L.T);
-        if (threadIdx.x == 0) L.phase = PH_AFTER_GUMBEL;
-        __syncthreads();
-        p = g;
+      if (L.nlo != L.nhi) {
+        p = narrow_plan(L, OP_NARROW_MASS);
         break;
       }
-      if (L.found_cum <= static_cast<uint32_t>(kListCap)) {
-        if (threadIdx.x == 0) {
-          cx.H->list_count = 0;
-          L.phase = PH_AFTER_COLLECT_X;
-        }
-        __syncthreads();
-        p.op = OP_COLLECT_X;
-        p.lo = L.nlo;
-        p.hi = L.nhi;
-        p.theta = L.theta_k;
-        p.raw_lo = L.surv_raw_lo;
-        p.m = L.m;
-        break;
-      }
-      p = narrow_mass_plan(L);
-      break;
-    }
-
-    case PH_AFTER_COLLECT_X: {
-      const int count = min(static_cast<int>(cx.H->list_count), kListCap);
-      sort_list(cx, count);
-      list_top_p(cx, L, count, L.Z, L.cum_above, true);
-      if (L.x_from_top) {
-        // the list holds every survivor above the cut: draw from it directly
-        list_gumbel(cx, L, L.send, true);
-        finalize_row(cx, L);
-        break;
-      }
-      Plan g{};
-      g.op = OP_GUMBEL;
-      g.theta = fmaxf(L.theta_k, L.theta_p);
-      g.raw_lo = raw_prefilter(g.theta, L.T);
-      if (threadIdx.x == 0) L.phase = PH_AFTER_GUMBEL;
-      __syncthreads();
-      p = g;
+      // one x value left: every survivor holding it has the same mass above (< pZ)
+      if (threadIdx.x == 0) L.theta_p = key_value(L.nlo);
+      p = gumbel_plan(L);
       break;
     }
 
@@ -1408,21 +1342,23 @@ __device__ Plan leader_step(const Ctx& cx) {
         int32_t bid = 0x7FFFFFFF;
         float bl = 0.0f;
         for (uint32_t r = 0; r < cx.C; ++r) {
-          const double sd = ld_dsmem_f64(mapa(smem_u32(&cx.H->stats.best_sd), r));
-          const int32_t id = static_cast<int32_t>(remote_u32(cx, &cx.H->stats.best_id, r));
-          const float l = __uint_as_float(remote_u32(cx, &cx.H->stats.best_l, r));
-          if (sd > bsd || (sd == bsd && id < bid)) {
-            bsd = sd;
-            bid = id;
-            bl = l;
+          const BestSlot& s = cx.H->best[r];
+          if (s.sd > bsd || (s.sd == bsd && s.id < bid)) {
+            bsd = s.sd;
+            bid = s.id;
+            bl = s.l;
           }
         }
         const bool ok = bid >= 0 && bid < a.V;
         L.token = ok ? bid : -1;
+        if (ok && L.part_is_x) {
+          const int s = bid / a.V_s, jj = bid - s * a.V_s;
+          bl = a.slices[s][static_cast<size_t>(cx.row) * a.V_s + jj];
+        }
         L.token_l = ok ? bl : __int_as_float(0x7FC00000);
       }
       __syncthreads();
-      finalize_row(cx, L);
+      tail = TAIL_STREAM_DONE;
       break;
     }
     default:
@@ -1431,7 +1367,34 @@ __device__ Plan leader_step(const Ctx& cx) {
   return p;
 }
 
-__global__ void __launch_bounds__(kThreads, 1) sample_kernel(const __grid_constant__ SampleArgs a) {
+// Leader work after the row's last cluster-wide step (the other CTAs have left).
+__device__ void leader_tail(const Ctx& cx, uint32_t tail) {
+  LeaderState& L = cx.H->L;
+  if (tail == TAIL_NONE) return;
+  const int count = min(static_cast<int>(cx.H->list_count), kListCap);
+  if (tail == TAIL_STREAM_DONE) {
+    if (L.topn_listed) {
+      sort_list(cx, count);
+      write_topn_from_list(cx, L);
+    }
+    write_outputs(cx, L);
+    return;
+  }
+  sort_list(cx, count);
+  write_topn_from_list(cx, L);
+  if (tail == TAIL_LIST_GREEDY) {
+    if (threadIdx.x == 0) {
+      L.token = static_cast<int32_t>(cx.list[0] & 0xFFFFFFFFu);
+      L.token_l = key_value(~static_cast<uint32_t>(cx.list[0] >> 32));
+    }
+    __syncthreads();
+  } else {
+    list_sample_tail(cx, L, count);
+  }
+  write_outputs(cx, L);
+}
+
+__global__ void __launch_bounds__(kThreads, 3) sample_kernel(const __grid_constant__ SampleArgs a) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   SharedHeader* H = reinterpret_cast<SharedHeader*>(smem_raw);
   uint8_t* scratch = smem_raw + ((sizeof(SharedHeader) + 127) & ~size_t(127));
@@ -1450,61 +1413,54 @@ __global__ void __launch_bounds__(kThreads, 1) sample_kernel(const __grid_consta
   const long long g1 = min(cx.g0 + a.part, static_cast<long long>(a.V));
   const int n = g1 > cx.g0 ? static_cast<int>(g1 - cx.g0) : 0;
   cx.n4 = n >> 2;
-  cx.part4 = reinterpret_cast<const float4*>(part);
+  cx.part4 = reinterpret_cast<float4*>(part);
 
-  // ---- load this CTA's part of the row (1-D bulk copies, one per slice segment)
-  const uint32_t bar = smem_u32(&H->mbar);
+  // ---- chunked load of this CTA's part (1-D bulk copies), one mbarrier per chunk
+  int chunk_q[kLoadChunks + 1];
+  for (int c = 0; c <= kLoadChunks; ++c) chunk_q[c] = static_cast<int>((static_cast<long long>(cx.n4) * c) / kLoadChunks);
   if (threadIdx.x == 0) {
-    mbar_init(bar, 1);
+    for (int c = 0; c < kLoadChunks; ++c) mbar_init(smem_u32(&H->mbar[c]), 1);
     fence_mbar_init();
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    mbar_arrive_expect_tx(bar, static_cast<uint32_t>(n) * 4u);
     const uint64_t pol = policy_evict_first();
-    long long g = cx.g0;
-    while (g < g1) {
-      const int s = static_cast<int>(g / a.V_s);
-      const long long s_end = min(static_cast<long long>(s + 1) * a.V_s, g1);
-      const float* src = a.slices[s] + static_cast<size_t>(cx.row) * a.V_s + (g - static_cast<long long>(s) * a.V_s);
-      long long off = g;
-      while (off < s_end) {
-        const long long chunk = min(s_end - off, 8192LL);  // 32 KB per copy
-        bulk_load(smem_u32(part + (off - cx.g0)), src + (off - g), static_cast<uint32_t>(chunk * 4), bar, pol);
-        off += chunk;
+    for (int c = 0; c < kLoadChunks; ++c) {
+      const long long e0 = cx.g0 + 4LL * chunk_q[c], e1 = cx.g0 + 4LL * chunk_q[c + 1];
+      const uint32_t bar = smem_u32(&H->mbar[c]);
+      mbar_arrive_expect_tx(bar, static_cast<uint32_t>((e1 - e0) * 4));
+      long long g = e0;
+      while (g < e1) {
+        const int s = static_cast<int>(g / a.V_s);
+        const long long s_end = min(static_cast<long long>(s + 1) * a.V_s, e1);
+        const float* src = a.slices[s] + static_cast<size_t>(cx.row) * a.V_s + (g - static_cast<long long>(s) * a.V_s);
+        bulk_load(smem_u32(part + (g - cx.g0)), src, static_cast<uint32_t>((s_end - g) * 4), bar, pol);
+        g = s_end;
       }
-      g = s_end;
     }
   }
   {
     uint32_t* hist = reinterpret_cast<uint32_t*>(scratch);
     for (int i = threadIdx.x; i < kHistBins; i += kThreads) hist[i] = 0;
+    for (int j = threadIdx.x; j < 64; j += kThreads) H->exp_tab[j] = exp2(static_cast<double>(j) / 64.0);
     if (threadIdx.x == 0) {
       H->L.phase = PH_START;
       H->list_count = 0;
     }
-  }
-  __syncthreads();
-  if (!mbar_wait_bounded(bar, 0)) {
-    // the copy never landed (a bug): report and leave the row unwritten
-    if (threadIdx.x == 0) atomicOr(a.err, kErrSampleLoad);
-  }
-
-  // ---- row params needed by every CTA
-  {
     const vsl_row_params prm = a.params[cx.row];
     cx.T = prm.temperature;
     cx.req = prm.request_id;
     cx.pos = prm.position;
   }
+  __syncthreads();
 
-  pass_stats(cx);
+  pass_stats(cx, chunk_q);
   cluster_sync();
 
+  uint32_t tail = TAIL_NONE;
   for (int iter = 0; iter < 64; ++iter) {
-    Plan next{};
     if (cx.rank == 0) {
-      next = leader_step(cx);
+      const Plan next = leader_step(cx, tail);
       __syncthreads();
       write_plan_all(cx, next);
     }
@@ -1513,17 +1469,18 @@ __global__ void __launch_bounds__(kThreads, 1) sample_kernel(const __grid_consta
     if (p.op == OP_END) break;
     switch (p.op) {
       case OP_COLLECT_RAW: op_collect_raw(cx, p); break;
-      case OP_COLLECT_X: op_collect_x(cx, p); break;
-      case OP_MASS_HIST: op_mass_hist(cx, p); break;
-      case OP_NARROW_COUNT: op_narrow_count(cx, p); break;
-      case OP_NARROW_MASS: op_narrow_mass(cx, p); break;
       case OP_NEXT_MAX: op_next_max(cx, p); break;
+      case OP_NARROW_COUNT: op_narrow_count(cx, p); break;
+      case OP_MASS: op_mass(cx, p); break;
+      case OP_NARROW_MASS: op_narrow_mass(cx, p); break;
       case OP_GUMBEL: op_gumbel(cx, p); break;
       default: break;
     }
     __syncthreads();
     cluster_sync();
+    if (p.last) break;  // what remains of the row is the leader's alone
   }
+  if (cx.rank == 0) leader_tail(cx, tail);
 }
 
 // ------------------------------------------------------------------ host side
@@ -1570,8 +1527,8 @@ static cudaError_t prepare_sample_kernel() {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, sample_kernel, &cfg) == cudaSuccess && n > 0) {
+    int nclusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&nclusters, sample_kernel, &cfg) == cudaSuccess && nclusters > 0) {
       g_max_cluster = c;
       break;
     }
