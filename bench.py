@@ -44,6 +44,31 @@ def _peaks():
         return 6650.0, 1590.0, 1400.0, "fallback"
 
 
+_KERNEL_SOURCES = {"logits_local_kernel": "vsl_gemm.cu", "sample_kernel": "vsl_sample.cu"}
+
+
+def _recorded_traffic(kernel, workload):
+    """DRAM bytes per launch recorded from an ncu capture in profiles/<kernel>_<workload>.md,
+    or None when there is none or the kernel source changed since (sha256 differs)."""
+    import hashlib
+    prof = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+    src = os.path.join(ROOT, "vocab_sharded_logits_b200", "csrc", _KERNEL_SOURCES[kernel])
+    if not (os.path.exists(prof) and os.path.exists(src)):
+        return None
+    fields = {}
+    for line in open(prof):
+        if ":" in line and line.split(":", 1)[0] in ("traffic_bytes_per_launch", "source_sha256"):
+            k, v = line.split(":", 1)
+            fields[k] = v.strip()
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    if fields.get("source_sha256") != sha:
+        return None
+    try:
+        return int(fields["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
 class ClockSampler:
     """Samples nvidia-smi SM clocks and throttle reasons during the timed region."""
 
@@ -330,7 +355,7 @@ def run_gpu(args, w):
                 "peak": hbm_peak, "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["peak_source"] = peak_kind
-    roof["traffic"] = None
+    roof["traffic"] = _recorded_traffic(roof["kernel"], w.name)
 
     line = {
         "metric": _metric(w), "value": value, "unit": "rows/s", "n_gpus": world, "steps": args.steps,
@@ -363,6 +388,41 @@ def run_gpu(args, w):
     return 0
 
 
+def run_sampler_only(args, w):
+    """Times ``sample`` alone on the workload's synthetic fp32 logits (the recipe of
+    the parity tests), L2 flushed before every rep; prints one JSON line."""
+    import vocab_sharded_logits_b200 as vsl
+    dev = torch.device("cuda", 0)
+    hbm_peak, _, _, peak_kind = _peaks()
+    logits = W.sampler_logits(w, dev)
+    slices = [t.contiguous() for t in torch.tensor_split(logits, w.S, dim=1)]
+    del logits
+    T, k, p, req, pos = W.row_params(w)
+    params = vsl.make_row_params(T, k, p, req, pos, dev)
+    out = vsl.sample(slices, params, 0, w.n_logprobs)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    for i in range(args.warmup):
+        vsl.sample(slices, params, i, w.n_logprobs, out=out)
+    times = []
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        vsl.sample(slices, params, 100 + i, w.n_logprobs, out=out)
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    ms = statistics.median(times)
+    nbytes = w.R * w.V * 4
+    print(json.dumps({"metric": f"sampler rows/sec ({w.name}, V={w.V}, L2 flushed)", "value": w.R / (ms / 1e3),
+                      "unit": "rows/s", "ms": ms, "hbm_gbs": nbytes / (ms / 1e3) / 1e9,
+                      "roofline": {"bound": "hbm", "achieved": nbytes / (ms / 1e3) / 1e9, "peak": hbm_peak,
+                                   "unit": "GB/s", "frac": nbytes / (ms / 1e3) / 1e9 / hbm_peak,
+                                   "peak_source": peak_kind},
+                      "config": {"workload": w.name, "rows": w.R, "vocab": w.V, "slices": w.S}}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -373,6 +433,8 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=4)
     ap.add_argument("--reference-rows", type=int, default=2)
     ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--sampler-only", action="store_true",
+                    help="time the sampler alone on the workload's synthetic logits (profiling aid)")
     args = ap.parse_args()
     w = W.WORKLOADS[args.workload]
     if args.impl == "reference":
@@ -380,6 +442,8 @@ def main():
     if not torch.cuda.is_available():
         print(json.dumps({"error": "no CUDA device"}))
         return 1
+    if args.sampler_only:
+        return run_sampler_only(args, w)
     return run_gpu(args, w)
 
 
