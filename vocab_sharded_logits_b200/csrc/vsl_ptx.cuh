@@ -104,6 +104,14 @@ __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
                "barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
+// Split cluster barrier: arrive (after this CTA's shared memory is initialised)
+// and wait (before the first access to another CTA's shared memory).
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
 // Address of the same shared variable in CTA `rank` of this cluster.
 __device__ __forceinline__ uint32_t mapa(uint32_t local, uint32_t rank) {
   uint32_t r;

@@ -56,6 +56,7 @@ constexpr int kMaxCluster = 16;
 constexpr int kMaxPart = 32768;        // floats per CTA (128 KB)
 constexpr int kPreferredPart = 12288;  // floats per CTA (48 KB) when the cluster size allows it
 constexpr int kLoadChunks = 4;
+constexpr int kLocalTopK = 64;         // top-k up to this is resolved from per-CTA candidate lists
 
 constexpr uint32_t kKeyNegInf = 0x007FFFFFu;  // key(-inf)
 constexpr uint32_t kKeyPosInf = 0xFF800000u;  // key(+inf)
@@ -71,6 +72,7 @@ enum Op : uint32_t {
   OP_NARROW_COUNT,
   OP_MASS,
   OP_NARROW_MASS,
+  OP_COLLECT_X,
   OP_GUMBEL,
 };
 
@@ -124,7 +126,14 @@ enum Phase : uint32_t {
   PH_TOPK_NARROW,
   PH_AFTER_MASS,
   PH_MASS_NARROW,
+  PH_AFTER_COLLECT_X,
   PH_AFTER_GUMBEL,
+};
+
+// Exact fixed-point mass: e * 2^60 held as four 16-bit limbs; a sum keeps each
+// limb's total separately in 64 bits (value = sum_k v[k] * 2^(16k - 60)).
+struct Fx4 {
+  unsigned long long v[4];
 };
 
 // Leader-only working state.
@@ -135,13 +144,13 @@ struct LeaderState {
   int32_t top_k;
   uint32_t req, pos;
   int r_n, r_k;
-  int greedy, topn_listed, part_is_x, mode;
+  int greedy, topn_listed, topn_done, part_is_x, mode;
   uint32_t collect_lo;
   float theta_k, theta_p, m;
   // narrowing state
   uint32_t nlo, nhi, nshift, nrank;
-  unsigned long long cum_hi, cum_lo;   // exact mass strictly above the range (fixed point)
-  unsigned long long z_hi, z_lo;       // exact total mass (fixed point)
+  Fx4 cum;                             // exact mass strictly above the range (fixed point)
+  Fx4 z;                               // exact total mass (fixed point)
   int topn_count;
   uint32_t prev_key;
   int32_t prev_id;
@@ -151,7 +160,7 @@ struct LeaderState {
   int found_bin;
   uint32_t found_cum;
   uint32_t found_cnt;
-  unsigned long long found_hi, found_lo;
+  Fx4 found_above;
 };
 
 struct __align__(16) SharedHeader {
@@ -160,6 +169,11 @@ struct __align__(16) SharedHeader {
   Plan plan;
   LeaderState L;
   BestSlot best[kMaxCluster];
+  uint32_t need_all[kMaxCluster];  // every CTA: each CTA's first-pass candidate count
+  uint32_t ok_all[kMaxCluster];    // every CTA: each CTA's list is usable for top-k
+  uint32_t listed;                 // the first-pass list holds the top-n (and top-k) union
+  uint32_t list_aux;               // staging count of a local collection / leader small-buffer counter
+  uint32_t list_base;              // reserved offset in the leader's list
   uint32_t list_count;
   uint32_t pad;
   unsigned long long mbar[kLoadChunks];
@@ -169,7 +183,7 @@ struct __align__(16) SharedHeader {
   int32_t red_i[kWarps];
   double scan_d[kWarps];
   uint32_t scan_u[kWarps];
-  unsigned long long scan_h[kWarps], scan_l[kWarps];
+  unsigned long long scan_fx[kWarps][4];
   double exp_tab[64];
 };
 
@@ -241,16 +255,39 @@ __device__ __forceinline__ double exp_neg64(double d, const double* tab) {
   return __hiloint2double(__double2hiint(v) + (m << 20), __double2loint(v));
 }
 
-// Fixed-point mass: e in (0, 1] as e * 2^76 = hi * 2^32 + lo, both exact integers
-// (hi <= 2^44, lo <= 2^32), so sums of up to 2^18 masses are exact in 64 bits.
-__device__ __forceinline__ void mass_fixed(double e, unsigned long long& hi, unsigned long long& lo) {
-  const double s = e * 0x1p44;
-  const double h = floor(s);
-  hi = static_cast<unsigned long long>(h);
-  lo = __double2ull_rn((s - h) * 0x1p32);
+// e in (0, 1] as the integer round(e * 2^60) (error <= 2^-61): exact sums of up
+// to 2^20 masses differ from the float64 sum by < 2^-41.  Each CTA adds the
+// four 16-bit limbs in u32 bins: a CTA holds at most 2^15 logits, so a limb
+// total stays below 2^31; the cluster-wide totals are kept per limb in 64 bits.
+__device__ __forceinline__ unsigned long long mass_q(double e) { return __double2ull_rn(e * 0x1p60); }
+__device__ __forceinline__ double fx_to_double(const Fx4& f) {
+  return static_cast<double>(f.v[0]) * 0x1p-60 + static_cast<double>(f.v[1]) * 0x1p-44 +
+         static_cast<double>(f.v[2]) * 0x1p-28 + static_cast<double>(f.v[3]) * 0x1p-12;
 }
-__device__ __forceinline__ double fixed_to_double(unsigned long long hi, unsigned long long lo) {
-  return static_cast<double>(hi) * 0x1p-44 + static_cast<double>(lo) * 0x1p-76;
+__device__ __forceinline__ Fx4 fx_zero() {
+  Fx4 f;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) f.v[k] = 0;
+  return f;
+}
+__device__ __forceinline__ Fx4 fx_add(const Fx4& a, const Fx4& b) {
+  Fx4 f;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) f.v[k] = a.v[k] + b.v[k];
+  return f;
+}
+__device__ __forceinline__ Fx4 fx_sub(const Fx4& a, const Fx4& b) {
+  Fx4 f;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) f.v[k] = a.v[k] - b.v[k];
+  return f;
+}
+__device__ __forceinline__ Fx4 fx_of(double e) {
+  const unsigned long long q = mass_q(e);
+  Fx4 f;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) f.v[k] = (q >> (16 * k)) & 0xFFFFull;
+  return f;
 }
 
 __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
@@ -401,28 +438,25 @@ __device__ __forceinline__ double block_scan_d(double v, double* total, SharedHe
   *total = tot;
   return x + off;
 }
-// Inclusive prefix sum of a fixed-point pair (hi, lo) over threads: exact.
-__device__ __forceinline__ void block_scan_fixed(unsigned long long& hi, unsigned long long& lo, SharedHeader* H) {
+// Inclusive prefix sum of fixed-point values over threads: exact.
+__device__ __forceinline__ void block_scan_fx(Fx4& x, SharedHeader* H) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const unsigned long long yh = __shfl_up_sync(0xFFFFFFFFu, hi, o);
-    const unsigned long long yl = __shfl_up_sync(0xFFFFFFFFu, lo, o);
-    if (lane >= o) {
-      hi += yh;
-      lo += yl;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const unsigned long long y = __shfl_up_sync(0xFFFFFFFFu, x.v[k], o);
+      if (lane >= o) x.v[k] += y;
     }
   }
   __syncthreads();
-  if (lane == 31) {
-    H->scan_h[warp] = hi;
-    H->scan_l[warp] = lo;
-  }
+  if (lane == 31)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) H->scan_fx[warp][k] = x.v[k];
   __syncthreads();
-  for (int i = 0; i < warp; ++i) {
-    hi += H->scan_h[i];
-    lo += H->scan_l[i];
-  }
+  for (int i = 0; i < warp; ++i)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) x.v[k] += H->scan_fx[i][k];
   __syncthreads();
 }
 
@@ -489,7 +523,8 @@ struct Ctx {
   int row, n4;
   long long g0;          // global id of the first element of this CTA's part
   uint32_t rank, C;
-  float T;
+  float T, top_p;
+  int top_k;
   uint32_t req, pos;
 };
 
@@ -528,6 +563,41 @@ __device__ __forceinline__ void list_append(const Ctx& cx, bool pred, uint64_t k
     const uint32_t idx = base + __popc(mask & ((1u << lane) - 1u));
     if (idx < static_cast<uint32_t>(kListCap)) st_dsmem_u64(mapa(smem_u32(cx.list + idx), 0), key);
   }
+}
+
+// Warp-aggregated append of sort keys to a list in this CTA's own shared memory.
+__device__ __forceinline__ void local_append(uint32_t* counter, uint64_t* list, bool pred, uint64_t key) {
+  const uint32_t mask = __ballot_sync(0xFFFFFFFFu, pred);
+  if (mask == 0) return;
+  const int lane = threadIdx.x & 31;
+  const int first = __ffs(mask) - 1;
+  uint32_t base = 0;
+  if (lane == first) base = atomicAdd(counter, static_cast<uint32_t>(__popc(mask)));
+  base = __shfl_sync(0xFFFFFFFFu, base, first);
+  if (pred) {
+    const uint32_t idx = base + __popc(mask & ((1u << lane) - 1u));
+    if (idx < static_cast<uint32_t>(kListCap)) list[idx] = key;
+  }
+}
+
+// After a local collection into this CTA's list (count in list_aux): a
+// non-leader reserves its exact count in the leader's list with one remote
+// atomic and copies its entries there.  The leader collects in place.
+__device__ void publish_local_list(const Ctx& cx) {
+  SharedHeader* H = cx.H;
+  if (cx.rank == 0) return;
+  __syncthreads();
+  const uint32_t cnt = min(H->list_aux, static_cast<uint32_t>(kListCap));
+  if (threadIdx.x == 0) H->list_base = atom_add_dsmem_u32(mapa(smem_u32(&H->list_count), 0), cnt);
+  __syncthreads();
+  const uint32_t base = H->list_base;
+  uint64_t* dst = cluster_ptr(cx.list, 0);
+  for (uint32_t i = threadIdx.x; i < cnt; i += kThreads)
+    if (base + i < static_cast<uint32_t>(kListCap)) dst[base + i] = cx.list[i];
+}
+// Counter and list a collection appends to: the leader's own, or a staging one.
+__device__ __forceinline__ uint32_t* collect_counter(const Ctx& cx) {
+  return cx.rank == 0 ? &cx.H->list_count : &cx.H->list_aux;
 }
 
 // ---- pass 1: stats + raw-key histogram, chunk by chunk as the bulk copies land
@@ -606,17 +676,22 @@ __device__ void pass_stats(const Ctx& cx, const int* chunk_q) {
     if (M > -INFINITY)
       for (int i = 0; i < kWarps; ++i)
         if (H->red_f[i * 2] > -INFINITY) S += H->red_f[i * 2 + 1] * fast_exp2((H->red_f[i * 2] - M) * kLog2e);
-    CtaStats* dst = cluster_ptr(&H->all[cx.rank], 0);
-    dst->kmax = a;
-    dst->kminf = c;
-    dst->bad = d;
-    dst->m = M;
-    dst->s = S;
+    H->stats.kmax = a;
+    H->stats.kminf = c;
+    H->stats.bad = d;
+    H->stats.m = M;
+    H->stats.s = S;
   }
+  __syncthreads();  // every thread reads the CTA's stats next (local_pick)
 }
 
 // ---- COLLECT_RAW: raw keys >= lo -> leader list (sort key: ~key, id)
 __device__ void op_collect_raw(const Ctx& cx, const Plan& p) {
+  uint32_t* counter = collect_counter(cx);
+  if (cx.rank != 0) {
+    if (threadIdx.x == 0) cx.H->list_aux = 0;
+    __syncthreads();
+  }
   const int nq = (cx.n4 + kThreads - 1) / kThreads * kThreads;
   for (int q = threadIdx.x; q < nq; q += kThreads) {
     const bool valid = q < cx.n4;
@@ -634,9 +709,10 @@ __device__ void op_collect_raw(const Ctx& cx, const Plan& p) {
     for (int i = 0; i < 4; ++i) {
       const bool pred = valid && k[i] >= p.lo;
       const uint32_t gid = static_cast<uint32_t>(cx.g0 + 4 * q + i);
-      list_append(cx, pred, (static_cast<uint64_t>(~k[i]) << 32) | gid);
+      local_append(counter, cx.list, pred, (static_cast<uint64_t>(~k[i]) << 32) | gid);
     }
   }
+  publish_local_list(cx);
 }
 
 // ---- NEXT_MAX: largest (key, lowest id) strictly after (nm_key, nm_id) in (key desc, id asc) order
@@ -705,35 +781,49 @@ __device__ void op_narrow_count(const Ctx& cx, const Plan& p) {
   }
 }
 
-// Fixed-point mass bins in the scratch area: hi[256], lo[256], cnt[256], edge[256].
+// Fixed-point mass bins in the scratch area: limb[4][256], cnt[256], edge[256]
+// (u32 only: the only shared-memory atomics that are native on this part).
 struct MassBins {
-  unsigned long long* hi;
-  unsigned long long* lo;
+  uint32_t* limb;   // limb[k * 256 + bin]
   uint32_t* cnt;
   uint32_t* edge;
 };
 __device__ __forceinline__ MassBins mass_bins(uint8_t* scratch) {
   MassBins b;
-  b.hi = reinterpret_cast<unsigned long long*>(scratch);
-  b.lo = b.hi + kSubBins;
-  b.cnt = reinterpret_cast<uint32_t*>(b.lo + kSubBins);
+  b.limb = reinterpret_cast<uint32_t*>(scratch);
+  b.cnt = b.limb + 4 * kSubBins;
   b.edge = b.cnt + kSubBins;
   return b;
 }
 __device__ __forceinline__ void clear_mass_bins(const MassBins& b) {
-  for (int i = threadIdx.x; i < kSubBins; i += kThreads) {
-    b.hi[i] = 0;
-    b.lo[i] = 0;
-    b.cnt[i] = 0;
-  }
+  for (int i = threadIdx.x; i < 5 * kSubBins; i += kThreads) b.limb[i] = 0;  // limbs and counts
   __syncthreads();
 }
 __device__ __forceinline__ void add_mass(const MassBins& b, uint32_t bin, double e) {
-  unsigned long long hi, lo;
-  mass_fixed(e, hi, lo);
-  atomicAdd(&b.hi[bin], hi);
-  atomicAdd(&b.lo[bin], lo);
+  const unsigned long long q = mass_q(e);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t limb = static_cast<uint32_t>((q >> (16 * k)) & 0xFFFFull);
+    if (limb) atomicAdd(&b.limb[k * kSubBins + bin], limb);
+  }
   atomicAdd(&b.cnt[bin], 1u);
+}
+// Sum over the cluster's CTAs of a u32 shared variable, widened to 64 bits.
+__device__ __forceinline__ unsigned long long cluster_sum_wide(const Ctx& cx, const uint32_t* local) {
+  unsigned long long v[kMaxCluster];
+#pragma unroll
+  for (int r = 0; r < kMaxCluster; ++r) v[r] = r < static_cast<int>(cx.C) ? *cluster_ptr(local, r) : 0ull;
+  unsigned long long t = 0;
+#pragma unroll
+  for (int r = 0; r < kMaxCluster; ++r) t += v[r];
+  return t;
+}
+// Cluster-wide fixed-point mass of bin j.
+__device__ __forceinline__ Fx4 bin_mass(const Ctx& cx, const MassBins& b, int j) {
+  Fx4 f;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) f.v[k] = cluster_sum_wide(cx, b.limb + k * kSubBins + j);
+  return f;
 }
 
 // ---- MASS: x = fl(l / T) written in place; survivors' masses on bins of
@@ -777,6 +867,70 @@ __device__ void op_narrow_mass(const Ctx& cx, const Plan& p) {
   }
 }
 
+// Pushes this CTA's best draw candidate into the leader's slot [rank].
+__device__ __forceinline__ void push_best(const Ctx& cx, Best& b) {
+  double sd = b.valid ? b.exact() : -INFINITY;
+  int32_t id = b.valid ? b.id : 0x7FFFFFFF;
+  float l = b.valid ? b.l : 0.0f;
+  block_best(sd, id, l, cx.H);
+  if (threadIdx.x == 0) {
+    const uint32_t slot = mapa(smem_u32(&cx.H->best[cx.rank]), 0);
+    st_dsmem_u64(slot, static_cast<uint64_t>(__double_as_longlong(sd)));
+    st_dsmem_u32(slot + 8, static_cast<uint32_t>(id));
+    st_dsmem_u32(slot + 12, __float_as_uint(l));
+  }
+}
+
+// ---- COLLECT_X: survivors (x >= theta, x in shared memory) with x-key in
+// [lo, hi] -> leader list (sort key: ~xkey, id).  Every survivor above the
+// range is kept whatever the cut inside it, so the same pass draws over them:
+// the CTA's best is pushed to the leader, which adds the range's kept entries.
+__device__ void op_collect_x(const Ctx& cx, const Plan& p) {
+  uint32_t* counter = collect_counter(cx);
+  if (cx.rank != 0) {
+    if (threadIdx.x == 0) cx.H->list_aux = 0;
+    __syncthreads();
+  }
+  Best b;
+  b.init();
+  const uint32_t k0 = static_cast<uint32_t>(cx.a->seed), k1 = static_cast<uint32_t>(cx.a->seed >> 32);
+  constexpr float kGMax = 16.7f;  // > the largest noise value, -log(-log(1 - 2^-24)) = 16.63
+  const int nq = (cx.n4 + kThreads - 1) / kThreads * kThreads;
+  for (int q = threadIdx.x; q < nq; q += kThreads) {
+    const bool valid = q < cx.n4;
+    const float4 v4 = valid ? cx.part4[q] : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+    const float v[4] = {v4.x, v4.y, v4.z, v4.w};
+    uint32_t k[4];
+    bool pred[4], above[4];
+    bool any = false, any_above = false;
+    float xmax = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      k[i] = fkey(v[i]);
+      const bool surv = valid && v[i] >= p.theta && v[i] > -INFINITY;
+      pred[i] = surv && k[i] >= p.lo && k[i] <= p.hi;
+      above[i] = surv && k[i] > p.hi;
+      any |= pred[i];
+      any_above |= above[i];
+      if (above[i]) xmax = fmaxf(xmax, v[i]);
+    }
+    if (__any_sync(0xFFFFFFFFu, any)) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        local_append(counter, cx.list, pred[i],
+                     (static_cast<uint64_t>(~k[i]) << 32) | static_cast<uint32_t>(cx.g0 + 4 * q + i));
+    }
+    if (!any_above || (b.valid && xmax + kGMax < b.s - score_tol(b.s))) continue;
+    const long long gid0 = cx.g0 + 4LL * q;
+    const uint4 w = philox4x32_10(make_uint4(static_cast<uint32_t>(gid0 >> 2), cx.pos, cx.req, 0u), k0, k1);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (above[i]) b.offer(v[i], 0.0f, word_of(w, i), static_cast<int32_t>(gid0 + i));
+  }
+  publish_local_list(cx);
+  push_best(cx, b);
+}
+
 // ---- GUMBEL: argmax of x + g over kept elements (x >= theta), float64-exact;
 // the CTA's best is pushed into the leader's slot [rank].
 __device__ void op_gumbel(const Ctx& cx, const Plan& p) {
@@ -813,16 +967,50 @@ __device__ void op_gumbel(const Ctx& cx, const Plan& p) {
     for (int i = 0; i < 4; ++i)
       if (kept[i]) b.offer(x[i], p.part_is_x ? 0.0f : v[i], word_of(w, i), static_cast<int32_t>(gid0 + i));
   }
-  double sd = b.valid ? b.exact() : -INFINITY;
-  int32_t id = b.valid ? b.id : 0x7FFFFFFF;
-  float l = b.valid ? b.l : 0.0f;
-  block_best(sd, id, l, cx.H);
-  if (threadIdx.x == 0) {
-    const uint32_t slot = mapa(smem_u32(&cx.H->best[cx.rank]), 0);
-    st_dsmem_u64(slot, static_cast<uint64_t>(__double_as_longlong(sd)));
-    st_dsmem_u32(slot + 8, static_cast<uint32_t>(id));
-    st_dsmem_u32(slot + 12, __float_as_uint(l));
+  push_best(cx, b);
+}
+
+// ---- per-CTA candidate threshold from this CTA's own histogram: the bin where
+// the running count from its max reaches `rank`.  Every element of the row's
+// top `rank` is in its CTA's local top `rank`, so the union of the per-CTA
+// collections holds the row's top `rank` (ties included: bins hold equal keys).
+struct LocalPick {
+  uint32_t lo, need, ok;
+};
+__device__ LocalPick local_pick(const Ctx& cx, uint32_t rank, bool check_T) {
+  const uint32_t* hist = reinterpret_cast<const uint32_t*>(cx.scratch);
+  SharedHeader* H = cx.H;
+  const int top = static_cast<int>(H->stats.kmax >> 20);
+  uint32_t cum = 0;
+  if (threadIdx.x == 0) H->L.found_bin = -1;  // scratch use in every CTA
+  __syncthreads();
+  for (int base = 0; base <= top; base += kThreads) {
+    const int j = base + threadIdx.x;
+    const uint32_t c = j <= top ? hist[top - j] : 0u;
+    uint32_t tot;
+    const uint32_t incl = block_scan_u(c, &tot, H);
+    if (c > 0 && cum + incl >= rank && cum + incl - c < rank) {
+      H->L.found_bin = top - j;
+      H->L.found_cum = cum + incl;
+    }
+    cum += tot;
+    __syncthreads();
+    if (H->L.found_bin >= 0) break;
   }
+  LocalPick lp;
+  if (H->L.found_bin < 0) {  // fewer than `rank` elements here: take them all
+    lp.lo = 0;
+    lp.need = cum;
+  } else {
+    lp.lo = static_cast<uint32_t>(H->L.found_bin) << 20;
+    lp.need = H->L.found_cum;
+  }
+  __syncthreads();
+  // top-k survivors: no element below the bin may scale to the bin's lowest x
+  lp.ok = 1;
+  if (check_T && lp.lo > kKeyNegInf + 1)
+    lp.ok = scale_x(key_value(lp.lo - 1), cx.T) < scale_x(key_value(lp.lo), cx.T) ? 1u : 0u;
+  return lp;
 }
 
 // ------------------------------------------------------------------ leader logic
@@ -867,31 +1055,28 @@ __device__ void find_rank_bin(const Ctx& cx, const uint32_t* cnt_local, int top,
 }
 
 // Mass bins merged over the cluster; finds the last non-empty bin whose exact
-// mass strictly above (cum_above + bins before it) is < top_p * Z.  Sets
-// L.found_bin, L.found_hi / found_lo (mass above it) and L.found_cnt.
+// mass strictly above (cum + bins before it) is < top_p * Z.  Sets
+// L.found_bin, L.found_above (mass above it) and L.found_cnt (its count).
 __device__ void find_mass_bin(const Ctx& cx, int nbins, LeaderState& L) {
   const MassBins b = mass_bins(cx.scratch);
   const int j = threadIdx.x;
-  unsigned long long h = 0, l = 0;
+  Fx4 own = fx_zero();
   uint32_t c = 0;
   if (j < nbins) {
-    h = cluster_sum(cx, b.hi + j);
-    l = cluster_sum(cx, b.lo + j);
-    c = cluster_sum(cx, b.cnt + j);
+    own = bin_mass(cx, b, j);
+    c = static_cast<uint32_t>(cluster_sum_wide(cx, b.cnt + j));
   }
-  unsigned long long ih = h, il = l;
-  block_scan_fixed(ih, il, cx.H);
-  // exact mass strictly above bin j
-  const unsigned long long bh = L.cum_hi + ih - h, bl = L.cum_lo + il - l;
-  const double pz = static_cast<double>(L.top_p) * fixed_to_double(L.z_hi, L.z_lo);
-  const bool cand = j < nbins && c > 0 && fixed_to_double(bh, bl) < pz;
+  Fx4 incl = own;
+  block_scan_fx(incl, cx.H);
+  const Fx4 above = fx_add(L.cum, fx_sub(incl, own));  // exact mass strictly above bin j
+  const double pz = static_cast<double>(L.top_p) * fx_to_double(L.z);
+  const bool cand = j < nbins && c > 0 && fx_to_double(above) < pz;
   const int best = block_max_i(cand ? j : -1, cx.H);
   if (threadIdx.x == 0) L.found_bin = -1;
   __syncthreads();
   if (best >= 0 && j == best) {
     L.found_bin = j;
-    L.found_hi = bh;
-    L.found_lo = bl;
+    L.found_above = above;
     L.found_cnt = c;
   }
   __syncthreads();
@@ -906,103 +1091,272 @@ __device__ void write_outputs(const Ctx& cx, LeaderState& L) {
   }
 }
 
-__device__ void write_topn_from_list(const Ctx& cx, const LeaderState& L) {
-  const SampleArgs& a = *cx.a;
-  for (int j = threadIdx.x; j < a.n_logprobs; j += kThreads) {
-    const uint64_t e = cx.list[j];
-    const float l = key_value(~static_cast<uint32_t>(e >> 32));
-    a.topn_ids[static_cast<size_t>(cx.row) * a.n_logprobs + j] = static_cast<int32_t>(e & 0xFFFFFFFFu);
-    a.topn_logprob[static_cast<size_t>(cx.row) * a.n_logprobs + j] = l - L.lse;
-  }
-}
-
 __device__ __forceinline__ int pow2_ceil(int n) {
   int p = 2;
   while (p < n) p <<= 1;
   return p;
 }
 
-// Sorts the list's first `count` entries (pads to a power of two).
-__device__ void sort_list(const Ctx& cx, int count) {
-  const int n = pow2_ceil(count);
-  for (int j = count + threadIdx.x; j < n; j += kThreads) cx.list[j] = ~0ull;
-  __syncthreads();
-  bitonic_sort(cx.list, n);
+// ---- leader list toolkit.  The list holds sort keys (~key << 32 | id), where
+// key is an order-preserving key (of l, or of x for x-lists).  Selections are
+// histogram narrowings over the list with native u32 shared atomics; only the
+// handful of top-n entries is ever sorted.
+__device__ __forceinline__ uint32_t entry_key(uint64_t e) { return ~static_cast<uint32_t>(e >> 32); }
+__device__ __forceinline__ int32_t entry_id(uint64_t e) { return static_cast<int32_t>(e & 0xFFFFFFFFu); }
+
+// x of a raw-list entry (or of an x-list entry).
+__device__ __forceinline__ float entry_x(uint64_t e, bool x_keys, float T) {
+  const float v = key_value(entry_key(e));
+  return x_keys ? v : scale_x(v, T);
 }
 
-// List resolution for a sampling row: the sorted raw list holds every top-k
-// survivor (and the top-n).  top-k threshold, exact top-p, the draw.
-__device__ void list_sample_tail(const Ctx& cx, LeaderState& L, int count) {
-  const uint64_t* list = cx.list;
-  // survivors: the prefix with x >= theta_k (x finite)
-  float theta_k = -INFINITY;
-  if (L.r_k > 0) theta_k = scale_x(key_value(~static_cast<uint32_t>(list[L.r_k - 1] >> 32)), L.T);
-  int ns = 0;
+// Key range [lo, hi] of the entries (all of them).
+__device__ void list_key_range(const Ctx& cx, int count, uint32_t& lo, uint32_t& hi) {
+  uint32_t mn = 0xFFFFFFFFu, mx = 0;
   for (int j = threadIdx.x; j < count; j += kThreads) {
-    const float x = scale_x(key_value(~static_cast<uint32_t>(list[j] >> 32)), L.T);
-    if (x >= theta_k && x > -INFINITY) ns = max(ns, j + 1);
+    const uint32_t k = entry_key(cx.list[j]);
+    mn = min(mn, k);
+    mx = max(mx, k);
   }
-  ns = block_max_i(ns, cx.H);
-  int nk = ns;
-  if (L.top_p < 1.0f) {
-    // exact top-p over the survivors: float64 masses, fixed-order prefix sums
-    constexpr int kPer = kListCap / kThreads;
-    double e[kPer];
-    double tsum = 0.0;
-    const int j0 = threadIdx.x * kPer;
-    const double m = static_cast<double>(L.m);
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-      const int j = j0 + i;
-      e[i] = 0.0;
-      if (j < ns)
-        e[i] = exp_neg64(static_cast<double>(scale_x(key_value(~static_cast<uint32_t>(list[j] >> 32)), L.T)) - m,
-                         cx.H->exp_tab);
-      tsum += e[i];
-    }
-    double Z;
-    const double incl = block_scan_d(tsum, &Z, cx.H);
-    const double pz = static_cast<double>(L.top_p);
-    double run = incl - tsum;
-    int sstar = -1;
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-      const int j = j0 + i;
-      if (j < ns) {
-        const float xj = scale_x(key_value(~static_cast<uint32_t>(list[j] >> 32)), L.T);
-        const bool start = j == 0 || scale_x(key_value(~static_cast<uint32_t>(list[j - 1] >> 32)), L.T) != xj;
-        if (start && run / Z < pz) sstar = j;
-      }
-      run += e[i];
-    }
-    sstar = max(block_max_i(sstar, cx.H), 0);
-    const float xs = scale_x(key_value(~static_cast<uint32_t>(list[sstar] >> 32)), L.T);
-    int send = ns;
-    for (int j = sstar + 1 + threadIdx.x; j < ns; j += kThreads)
-      if (scale_x(key_value(~static_cast<uint32_t>(list[j] >> 32)), L.T) != xs) send = min(send, j);
-    nk = block_min_i(send, cx.H);
+  mn = warp_reduce(mn, [](uint32_t a, uint32_t b) { return a < b ? a : b; });
+  mx = warp_reduce(mx, [](uint32_t a, uint32_t b) { return a > b ? a : b; });
+  SharedHeader* H = cx.H;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  __syncthreads();
+  if (lane == 0) {
+    H->red_u[warp * 2] = mn;
+    H->red_u[warp * 2 + 1] = mx;
   }
-  // the draw over the kept prefix
+  __syncthreads();
+  lo = 0xFFFFFFFFu;
+  hi = 0;
+  for (int i = 0; i < kWarps; ++i) {
+    lo = min(lo, H->red_u[i * 2]);
+    hi = max(hi, H->red_u[i * 2 + 1]);
+  }
+  __syncthreads();
+}
+
+// The r-th largest key among the list entries (1 <= r <= count), by 256-bin
+// rank narrowing on the key.
+__device__ uint32_t list_rank_key(const Ctx& cx, int count, uint32_t r) {
+  uint32_t lo, hi;
+  list_key_range(cx, count, lo, hi);
+  uint32_t* cnt = reinterpret_cast<uint32_t*>(cx.scratch);
+  SharedHeader* H = cx.H;
+  while (lo != hi) {
+    const uint32_t width = hi - lo;
+    const int bits = 32 - __clz(width);
+    const int shift = bits > 8 ? bits - 8 : 0;
+    for (int i = threadIdx.x; i < kSubBins; i += kThreads) cnt[i] = 0;
+    __syncthreads();
+    for (int j = threadIdx.x; j < count; j += kThreads) {
+      const uint32_t k = entry_key(cx.list[j]);
+      if (k >= lo && k <= hi) atomicAdd(&cnt[(hi - k) >> shift], 1u);
+    }
+    __syncthreads();
+    const uint32_t c = cnt[threadIdx.x];
+    uint32_t tot;
+    const uint32_t incl = block_scan_u(c, &tot, H);
+    if (threadIdx.x == 0) H->L.found_bin = 0;
+    __syncthreads();
+    if (c > 0 && incl >= r && incl - c < r) {
+      H->L.found_bin = threadIdx.x;
+      H->L.found_cum = incl - c;
+    }
+    __syncthreads();
+    const int jb = H->L.found_bin;
+    const uint32_t before = H->L.found_cum;
+    __syncthreads();
+    const uint32_t nhi = hi - (static_cast<uint32_t>(jb) << shift);
+    const uint32_t span = (static_cast<uint32_t>(jb + 1) << shift) - 1u;
+    lo = (hi - lo) > span ? hi - span : lo;
+    hi = nhi;
+    r -= before;
+  }
+  return lo;
+}
+
+// Writes the top-n (key desc, id asc) of a raw list that holds the row's top n.
+__device__ void list_topn(const Ctx& cx, const LeaderState& L, int count) {
+  const SampleArgs& a = *cx.a;
+  const int n = a.n_logprobs;
+  if (n <= 0) return;
+  const uint32_t kn = list_rank_key(cx, count, static_cast<uint32_t>(n));
+  // gather every entry with key >= the n-th key into a small buffer, sort it
+  uint64_t* buf = reinterpret_cast<uint64_t*>(cx.scratch);
+  uint32_t* nbuf = &cx.H->list_aux;
+  if (threadIdx.x == 0) *nbuf = 0;
+  __syncthreads();
+  for (int j = threadIdx.x; j < count; j += kThreads) {
+    const uint64_t e = cx.list[j];
+    if (entry_key(e) >= kn) {
+      const uint32_t i = atomicAdd(nbuf, 1u);
+      if (i < static_cast<uint32_t>(kListCap)) buf[i] = e;
+    }
+  }
+  __syncthreads();
+  const int m = min(static_cast<int>(*nbuf), kListCap);
+  const int np2 = pow2_ceil(m);
+  for (int j = m + threadIdx.x; j < np2; j += kThreads) buf[j] = ~0ull;
+  __syncthreads();
+  bitonic_sort(buf, np2);
+  for (int j = threadIdx.x; j < n; j += kThreads) {
+    const uint64_t e = buf[j];
+    a.topn_ids[static_cast<size_t>(cx.row) * n + j] = entry_id(e);
+    a.topn_logprob[static_cast<size_t>(cx.row) * n + j] = key_value(entry_key(e)) - L.lse;
+  }
+  __syncthreads();
+}
+
+// The list entry with the largest key (lowest id among equal keys).
+__device__ uint64_t list_max_entry(const Ctx& cx, int count) {
+  uint64_t best = ~0ull;  // sort keys: smaller = larger key, then lower id
+  for (int j = threadIdx.x; j < count; j += kThreads) best = min(best, cx.list[j]);
+  best = warp_reduce(best, [](uint64_t a, uint64_t b) { return a < b ? a : b; });
+  SharedHeader* H = cx.H;
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) reinterpret_cast<uint64_t*>(H->red_d)[threadIdx.x >> 5] = best;
+  __syncthreads();
+  uint64_t t = ~0ull;
+  for (int i = 0; i < kWarps; ++i) t = min(t, reinterpret_cast<uint64_t*>(H->red_d)[i]);
+  __syncthreads();
+  return t;
+}
+
+// Exact top-p cut over the list's survivors (x >= theta_s, x finite; x-key in
+// [lo, hi]), given the exact mass strictly above the list (`above`) and the
+// total Z: the smallest x value whose mass of strictly larger values is
+// < top_p * Z.  256-bin narrowing on x-keys with fixed-point masses.
+__device__ float list_mass_cut(const Ctx& cx, LeaderState& L, int count, bool x_keys, float theta_s, Fx4 above,
+                               const Fx4& Z) {
+  const MassBins b = mass_bins(cx.scratch);
+  const double m = static_cast<double>(L.m);
+  const double pz = static_cast<double>(L.top_p) * fx_to_double(Z);
+  // x-key range of the survivors
+  uint32_t mn = 0xFFFFFFFFu, mx = 0;
+  for (int j = threadIdx.x; j < count; j += kThreads) {
+    const float x = entry_x(cx.list[j], x_keys, L.T);
+    if (x >= theta_s && x > -INFINITY) {
+      const uint32_t k = fkey(x);
+      mn = min(mn, k);
+      mx = max(mx, k);
+    }
+  }
+  mn = warp_reduce(mn, [](uint32_t a, uint32_t c) { return a < c ? a : c; });
+  mx = warp_reduce(mx, [](uint32_t a, uint32_t c) { return a > c ? a : c; });
+  SharedHeader* H = cx.H;
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) {
+    H->red_u[(threadIdx.x >> 5) * 2] = mn;
+    H->red_u[(threadIdx.x >> 5) * 2 + 1] = mx;
+  }
+  __syncthreads();
+  uint32_t lo = 0xFFFFFFFFu, hi = 0;
+  for (int i = 0; i < kWarps; ++i) {
+    lo = min(lo, H->red_u[i * 2]);
+    hi = max(hi, H->red_u[i * 2 + 1]);
+  }
+  __syncthreads();
+  if (lo > hi) return key_value(0xFFFFFFFFu);  // no survivor (cannot happen: the max survives)
+  while (lo != hi) {
+    const uint32_t width = hi - lo;
+    const int bits = 32 - __clz(width);
+    const int shift = bits > 8 ? bits - 8 : 0;
+    clear_mass_bins(b);
+    for (int j = threadIdx.x; j < count; j += kThreads) {
+      const float x = entry_x(cx.list[j], x_keys, L.T);
+      const uint32_t k = fkey(x);
+      if (x >= theta_s && x > -INFINITY && k >= lo && k <= hi)
+        add_mass(b, (hi - k) >> shift, exp_neg64(static_cast<double>(x) - m, H->exp_tab));
+    }
+    __syncthreads();
+    const int j = threadIdx.x;
+    Fx4 own = fx_zero();
+#pragma unroll
+    for (int k = 0; k < 4; ++k) own.v[k] = b.limb[k * kSubBins + j];
+    const uint32_t c = b.cnt[j];
+    Fx4 incl = own;
+    block_scan_fx(incl, H);
+    const Fx4 before = fx_add(above, fx_sub(incl, own));
+    const bool cand = c > 0 && fx_to_double(before) < pz;
+    const int jb = max(block_max_i(cand ? j : -1, H), 0);
+    if (j == jb) H->L.found_above = before;
+    __syncthreads();
+    above = H->L.found_above;
+    __syncthreads();
+    const uint32_t nhi = hi - (static_cast<uint32_t>(jb) << shift);
+    const uint32_t span = (static_cast<uint32_t>(jb + 1) << shift) - 1u;
+    lo = (hi - lo) > span ? hi - span : lo;
+    hi = nhi;
+  }
+  return key_value(lo);
+}
+
+// Exact fixed-point total mass of the raw list's survivors (x >= theta_s).
+__device__ Fx4 list_mass_total(const Ctx& cx, const LeaderState& L, int count, float theta_s) {
+  Fx4 t = fx_zero();
+  const double m = static_cast<double>(L.m);
+  for (int j = threadIdx.x; j < count; j += kThreads) {
+    const float x = entry_x(cx.list[j], false, L.T);
+    if (x >= theta_s && x > -INFINITY) t = fx_add(t, fx_of(exp_neg64(static_cast<double>(x) - m, cx.H->exp_tab)));
+  }
+  Fx4 incl = t;
+  block_scan_fx(incl, cx.H);  // the last thread holds the total
+  SharedHeader* H = cx.H;
+  if (threadIdx.x == kThreads - 1) H->L.found_above = incl;
+  __syncthreads();
+  const Fx4 z = H->L.found_above;
+  __syncthreads();
+  return z;
+}
+
+// Best draw candidate (float64 score, id, raw l or 0 for x-lists) over list
+// entries with x >= theta (x finite); every thread gets the result.
+__device__ void list_best(const Ctx& cx, const LeaderState& L, int count, bool x_keys, float theta, double& sd,
+                          int32_t& id, float& l) {
   Best b;
   b.init();
   const uint32_t k0 = static_cast<uint32_t>(cx.a->seed), k1 = static_cast<uint32_t>(cx.a->seed >> 32);
-  for (int j = threadIdx.x; j < nk; j += kThreads) {
-    const uint64_t e = list[j];
-    const float l = key_value(~static_cast<uint32_t>(e >> 32));
-    const int32_t id = static_cast<int32_t>(e & 0xFFFFFFFFu);
+  for (int j = threadIdx.x; j < count; j += kThreads) {
+    const uint64_t e = cx.list[j];
+    const float x = entry_x(e, x_keys, L.T);
+    if (!(x >= theta && x > -INFINITY)) continue;
+    const int32_t id = entry_id(e);
     const uint4 w = philox4x32_10(make_uint4(static_cast<uint32_t>(id) >> 2, cx.pos, cx.req, 0u), k0, k1);
-    b.offer(scale_x(l, L.T), l, word_of(w, id & 3), id);
+    b.offer(x, x_keys ? 0.0f : key_value(entry_key(e)), word_of(w, id & 3), id);
   }
-  double sd = b.valid ? b.exact() : -INFINITY;
-  int32_t id = b.valid ? b.id : 0x7FFFFFFF;
-  float l = b.valid ? b.l : 0.0f;
+  sd = b.valid ? b.exact() : -INFINITY;
+  id = b.valid ? b.id : 0x7FFFFFFF;
+  l = b.valid ? b.l : 0.0f;
   block_best(sd, id, l, cx.H);
+}
+
+// The draw over list entries with x >= theta (x finite), into L.token.
+__device__ void list_gumbel(const Ctx& cx, LeaderState& L, int count, bool x_keys, float theta) {
+  double sd;
+  int32_t id;
+  float l;
+  list_best(cx, L, count, x_keys, theta, sd, id, l);
   if (threadIdx.x == 0) {
     const bool ok = id >= 0 && id < cx.a->V;
     L.token = ok ? id : -1;
     L.token_l = ok ? l : __int_as_float(0x7FC00000);
   }
   __syncthreads();
+}
+
+// List resolution for a sampling row: the raw list holds the top-n and every
+// top-k survivor.  theta_k by rank, exact top-p by mass narrowing, the draw.
+__device__ void list_sample_tail(const Ctx& cx, LeaderState& L, int count) {
+  float theta = -INFINITY;
+  if (L.r_k > 0) theta = scale_x(key_value(list_rank_key(cx, count, static_cast<uint32_t>(L.r_k))), L.T);
+  if (L.top_p < 1.0f) {
+    const Fx4 z = list_mass_total(cx, L, count, theta);
+    const float theta_p = list_mass_cut(cx, L, count, false, theta, fx_zero(), z);
+    theta = fmaxf(theta, theta_p);
+  }
+  list_gumbel(cx, L, count, false, theta);
 }
 
 __device__ Plan narrow_plan(LeaderState& L, uint32_t op) {
@@ -1031,19 +1385,26 @@ __device__ __forceinline__ void narrow_range(LeaderState& L, int j) {
   L.nhi = hi;
 }
 
+// MASS plan: survivors x >= theta_k; bins span [x_low, m], x_low the smallest
+// survivor x (at most 96 below m).
+__device__ __forceinline__ Plan mass_plan(float m, float theta_k, uint32_t kminf, float T) {
+  Plan p{};
+  p.op = OP_MASS;
+  p.theta = theta_k;
+  p.m = m;
+  const float x_low = fmaxf(theta_k, scale_x(key_value(kminf), T));
+  float width = fminf(__fsub_rn(m, x_low), 96.0f);
+  if (!(width > 0.0f)) width = 1.0f;
+  p.step = width / static_cast<float>(kMassBins);
+  return p;
+}
+
 // Survivors known (theta_k): masses for top-p, or the draw directly.
 __device__ Plan plan_after_theta_k(const Ctx& cx, LeaderState& L) {
   Plan p{};
   __syncthreads();
   if (L.top_p < 1.0f) {
-    p.op = OP_MASS;
-    p.theta = L.theta_k;
-    p.m = L.m;
-    // bins span [x_low, m], x_low the smallest survivor x (at most 96 below m)
-    const float x_low = fmaxf(L.theta_k, scale_x(key_value(L.kminf), L.T));
-    float width = fminf(__fsub_rn(L.m, x_low), 96.0f);
-    if (!(width > 0.0f)) width = 1.0f;
-    p.step = width / static_cast<float>(kMassBins);
+    p = mass_plan(L.m, L.theta_k, L.kminf, L.T);
     if (threadIdx.x == 0) {
       L.phase = PH_AFTER_MASS;
       L.part_is_x = 1;
@@ -1081,14 +1442,46 @@ __device__ Plan gumbel_plan(LeaderState& L) {
   return p;
 }
 
-__device__ Plan leader_step(const Ctx& cx, uint32_t& tail) {
-  LeaderState& L = cx.H->L;
+// The top-p cut lies in the x-key range [nlo, nhi] (found_cnt survivors, exact
+// mass L.cum above it): one x value decides it, a range that fits the list is
+// resolved on the leader, a larger one is narrowed further.
+__device__ Plan plan_cut_range(LeaderState& L, SharedHeader* H) {
+  if (L.nlo == L.nhi) {
+    // one x value: every survivor holding it has the same mass above (< pZ)
+    if (threadIdx.x == 0) L.theta_p = key_value(L.nlo);
+    return gumbel_plan(L);
+  }
+  if (L.found_cnt <= static_cast<uint32_t>(kListCap)) {
+    Plan p{};
+    p.op = OP_COLLECT_X;
+    p.lo = L.nlo;
+    p.hi = L.nhi;
+    p.theta = L.theta_k;
+    p.part_is_x = 1;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      L.phase = PH_AFTER_COLLECT_X;
+      H->list_count = 0;
+    }
+    return p;
+  }
+  return narrow_plan(L, OP_NARROW_MASS);
+}
+
+// Resolves theta_p from the x-key list of every survivor in the cut range,
+// with the exact mass above the range (L.cum) and the total (L.z).
+__device__ void list_cut(const Ctx& cx, LeaderState& L, int count) {
+  const float theta_p = list_mass_cut(cx, L, count, true, -INFINITY, L.cum, L.z);
+  if (threadIdx.x == 0) L.theta_p = theta_p;
+  __syncthreads();
+}
+
+// Leader: merges the statistics every CTA pushed, validates data and parameters,
+// and fills the row state.  A flagged row gets its outputs here; returns true
+// for it.  When the first pass's list is complete (`listed`), the top-n is
+// written from it now.
+__device__ bool leader_merge(const Ctx& cx, LeaderState& L) {
   const SampleArgs& a = *cx.a;
-  Plan p{};
-  p.op = OP_END;
-  tail = TAIL_NONE;
-  switch (L.phase) {
-    case PH_START: {
       if (threadIdx.x == 0) {
         uint32_t kmax = 0, kminf = 0xFFFFFFFFu, bad = 0;
         float M = -INFINITY;
@@ -1134,7 +1527,8 @@ __device__ Plan leader_step(const Ctx& cx, uint32_t& tail) {
         L.theta_p = -INFINITY;
         L.part_is_x = 0;
         L.token = -1;
-        L.cum_hi = L.cum_lo = 0;
+        L.cum = fx_zero();
+        L.topn_done = 0;
       }
       __syncthreads();
       if (L.flags) {
@@ -1147,14 +1541,46 @@ __device__ Plan leader_step(const Ctx& cx, uint32_t& tail) {
           a.topn_ids[static_cast<size_t>(cx.row) * a.n_logprobs + j] = -1;
           a.topn_logprob[static_cast<size_t>(cx.row) * a.n_logprobs + j] = __int_as_float(0x7FC00000);
         }
+        return true;
+      }
+  if (cx.H->listed) {
+    // the first pass's union of per-CTA candidates holds the exact top-n
+    const int count = min(static_cast<int>(cx.H->list_count), kListCap);
+    list_topn(cx, L, count);
+    const uint64_t top = list_max_entry(cx, count);
+    if (threadIdx.x == 0) {
+      L.topn_done = 1;
+      L.token = entry_id(top);  // the argmax (greedy rows)
+      L.token_l = key_value(entry_key(top));
+    }
+    __syncthreads();
+  }
+  return false;
+}
+
+__device__ Plan leader_step(const Ctx& cx, uint32_t& tail) {
+  LeaderState& L = cx.H->L;
+  const SampleArgs& a = *cx.a;
+  Plan p{};
+  p.op = OP_END;
+  tail = TAIL_NONE;
+  switch (L.phase) {
+    case PH_START: {
+      if (leader_merge(cx, L)) break;  // flagged row: outputs written
+      if (L.topn_done && L.greedy) {
+        write_outputs(cx, L);
         break;
       }
       // raw-histogram bins from the max key downward
       const uint32_t* hist = reinterpret_cast<const uint32_t*>(cx.scratch);
       const int top = static_cast<int>(L.kmax >> 20);
-      find_rank_bin(cx, hist, top, top + 1, true, static_cast<uint32_t>(L.r_n), L);
-      const int bn = max(L.found_bin, 0);
-      const uint32_t need_n = L.found_cum + L.found_cnt;
+      int bn = 0;
+      uint32_t need_n = 0;
+      if (!L.topn_done) {
+        find_rank_bin(cx, hist, top, top + 1, true, static_cast<uint32_t>(L.r_n), L);
+        bn = max(L.found_bin, 0);
+        need_n = L.found_cum + L.found_cnt;
+      }
       int bk = 0;
       uint32_t need_k = 0, cum_k = 0;
       if (L.r_k > 0) {
@@ -1164,8 +1590,8 @@ __device__ Plan leader_step(const Ctx& cx, uint32_t& tail) {
         need_k = L.found_cum + L.found_cnt;
       }
       if (threadIdx.x == 0) {
-        const uint32_t lo_n = static_cast<uint32_t>(bn) << 20;
-        L.topn_listed = need_n <= static_cast<uint32_t>(kListCap);
+        const uint32_t lo_n = L.topn_done ? 0xFFFFFFFFu : static_cast<uint32_t>(bn) << 20;
+        L.topn_listed = L.topn_done || need_n <= static_cast<uint32_t>(kListCap);
         uint32_t lo = lo_n;
         int mode = 0;  // 0 = stream, 1 = list greedy, 2 = list sample
         if (L.greedy) {
@@ -1188,7 +1614,7 @@ __device__ Plan leader_step(const Ctx& cx, uint32_t& tail) {
         L.mode = mode;
         L.collect_lo = lo;
         cx.H->list_count = 0;
-        if (mode == 0) {
+        if (mode == 0 && !L.topn_done) {
           if (L.topn_listed) {
             L.phase = PH_AFTER_TOPN_COLLECT;
           } else {
@@ -1200,7 +1626,9 @@ __device__ Plan leader_step(const Ctx& cx, uint32_t& tail) {
         }
       }
       __syncthreads();
-      if (L.mode != 0 || L.topn_listed) {
+      if (L.mode == 0 && L.topn_done) {
+        p = plan_stream_sampling(cx, L);
+      } else if (L.mode != 0 || L.topn_listed) {
         p.op = OP_COLLECT_RAW;
         p.lo = L.collect_lo;
         if (L.mode == 1) tail = TAIL_LIST_GREEDY;
@@ -1256,7 +1684,9 @@ __device__ Plan leader_step(const Ctx& cx, uint32_t& tail) {
     }
 
     case PH_AFTER_TOPN_COLLECT: {
-      // the top-n list stays in the leader's memory and is finished in its tail
+      // write the top-n now: the list is reused for the top-p cut later
+      list_topn(cx, L, min(static_cast<int>(cx.H->list_count), kListCap));
+      if (threadIdx.x == 0) L.topn_done = 1;
       p = plan_stream_sampling(cx, L);
       break;
     }
@@ -1280,20 +1710,13 @@ __device__ Plan leader_step(const Ctx& cx, uint32_t& tail) {
     }
 
     case PH_AFTER_MASS: {
-      // exact total mass, then the log bin holding the cut
+      // exact total mass, then the bin holding the cut
       {
         const MassBins b = mass_bins(cx.scratch);
         const int j = threadIdx.x;
-        unsigned long long h = 0, l = 0;
-        if (j < kMassBins) {
-          h = cluster_sum(cx, b.hi + j);
-          l = cluster_sum(cx, b.lo + j);
-        }
-        block_scan_fixed(h, l, cx.H);
-        if (j == kThreads - 1) {
-          L.z_hi = h;
-          L.z_lo = l;
-        }
+        Fx4 f = j < kMassBins ? bin_mass(cx, b, j) : fx_zero();
+        block_scan_fx(f, cx.H);
+        if (j == kThreads - 1) L.z = f;
         __syncthreads();
       }
       find_mass_bin(cx, kMassBins, L);
@@ -1303,17 +1726,11 @@ __device__ Plan leader_step(const Ctx& cx, uint32_t& tail) {
         const uint32_t* edge = mass_bins(cx.scratch).edge;
         L.nhi = edge[bin];
         L.nlo = bin == kMassBins - 1 ? 0u : edge[bin + 1] + 1u;
-        L.cum_hi = L.found_hi;
-        L.cum_lo = L.found_lo;
+        L.cum = L.found_above;
         L.phase = PH_MASS_NARROW;
       }
       __syncthreads();
-      if (L.nlo == L.nhi) {
-        if (threadIdx.x == 0) L.theta_p = key_value(L.nlo);
-        p = gumbel_plan(L);
-        break;
-      }
-      p = narrow_plan(L, OP_NARROW_MASS);
+      p = plan_cut_range(L, cx.H);
       break;
     }
 
@@ -1322,17 +1739,41 @@ __device__ Plan leader_step(const Ctx& cx, uint32_t& tail) {
       find_mass_bin(cx, nb, L);
       if (threadIdx.x == 0) {
         narrow_range(L, max(L.found_bin, 0));
-        L.cum_hi = L.found_hi;
-        L.cum_lo = L.found_lo;
+        L.cum = L.found_above;
       }
       __syncthreads();
-      if (L.nlo != L.nhi) {
-        p = narrow_plan(L, OP_NARROW_MASS);
-        break;
+      p = plan_cut_range(L, cx.H);
+      break;
+    }
+
+    case PH_AFTER_COLLECT_X: {
+      // exact cut inside the range, then the draw: the range's kept entries
+      // here, every survivor above the range in the CTAs' pushed bests
+      const int count = min(static_cast<int>(cx.H->list_count), kListCap);
+      list_cut(cx, L, count);
+      double sd;
+      int32_t id;
+      float l;
+      list_best(cx, L, count, true, L.theta_p, sd, id, l);
+      if (threadIdx.x == 0) {
+        for (uint32_t r = 0; r < cx.C; ++r) {
+          const BestSlot& s = cx.H->best[r];
+          if (s.sd > sd || (s.sd == sd && s.id < id)) {
+            sd = s.sd;
+            id = s.id;
+          }
+        }
+        const bool ok = id >= 0 && id < a.V;
+        L.token = ok ? id : -1;
+        float tl = __int_as_float(0x7FC00000);
+        if (ok) {
+          const int sl = id / a.V_s, jj = id - sl * a.V_s;
+          tl = a.slices[sl][static_cast<size_t>(cx.row) * a.V_s + jj];
+        }
+        L.token_l = tl;
       }
-      // one x value left: every survivor holding it has the same mass above (< pZ)
-      if (threadIdx.x == 0) L.theta_p = key_value(L.nlo);
-      p = gumbel_plan(L);
+      __syncthreads();
+      tail = TAIL_STREAM_DONE;
       break;
     }
 
@@ -1373,19 +1814,15 @@ __device__ void leader_tail(const Ctx& cx, uint32_t tail) {
   if (tail == TAIL_NONE) return;
   const int count = min(static_cast<int>(cx.H->list_count), kListCap);
   if (tail == TAIL_STREAM_DONE) {
-    if (L.topn_listed) {
-      sort_list(cx, count);
-      write_topn_from_list(cx, L);
-    }
     write_outputs(cx, L);
     return;
   }
-  sort_list(cx, count);
-  write_topn_from_list(cx, L);
+  if (!L.topn_done) list_topn(cx, L, count);
   if (tail == TAIL_LIST_GREEDY) {
+    const uint64_t top = list_max_entry(cx, count);
     if (threadIdx.x == 0) {
-      L.token = static_cast<int32_t>(cx.list[0] & 0xFFFFFFFFu);
-      L.token_l = key_value(~static_cast<uint32_t>(cx.list[0] >> 32));
+      L.token = entry_id(top);
+      L.token_l = key_value(entry_key(top));
     }
     __syncthreads();
   } else {
@@ -1449,15 +1886,95 @@ __global__ void __launch_bounds__(kThreads, 3) sample_kernel(const __grid_consta
     }
     const vsl_row_params prm = a.params[cx.row];
     cx.T = prm.temperature;
+    cx.top_k = prm.top_k;
+    cx.top_p = prm.top_p;
     cx.req = prm.request_id;
     cx.pos = prm.position;
   }
   __syncthreads();
 
+  cluster_arrive();  // this CTA's shared memory is initialised
   pass_stats(cx, chunk_q);
+
+  // ---- first-pass candidates from this CTA's own threshold, straight into the leader's list
+  const bool greedy = cx.T == 0.0f;
+  const bool k_on = cx.T > 0.0f && cx.top_k > 0 && cx.top_k < a.V;
+  const bool eligible = greedy || (k_on && cx.top_k <= kLocalTopK);
+  uint32_t rank = a.n_logprobs > 0 ? static_cast<uint32_t>(a.n_logprobs) : 1u;
+  if (eligible && k_on) rank = max(rank, static_cast<uint32_t>(cx.top_k));
+  const LocalPick lp = local_pick(cx, rank, eligible && k_on);
+  cluster_wait();    // every CTA's shared memory is initialised: remote access is safe
+  {
+    Plan pc{};
+    pc.lo = lp.lo;
+    op_collect_raw(cx, pc);
+  }
+  if (threadIdx.x < cx.C) {
+    cluster_ptr(H->need_all, threadIdx.x)[cx.rank] = lp.need;
+    cluster_ptr(H->ok_all, threadIdx.x)[cx.rank] = lp.ok;
+    *cluster_ptr(&H->all[cx.rank], threadIdx.x) = H->stats;  // every CTA sees every CTA's stats
+  }
+  __syncthreads();
   cluster_sync();
+  uint32_t total = 0, all_ok = 1;
+  for (uint32_t r = 0; r < cx.C; ++r) {
+    total += H->need_all[r];
+    all_ok &= H->ok_all[r];
+  }
+  const bool listed = total <= static_cast<uint32_t>(kListCap);
+  if (eligible && listed && all_ok) {
+    // the list holds the top-n and every top-k survivor: the leader finishes alone
+    if (cx.rank == 0) {
+      if (threadIdx.x == 0) H->listed = 0;
+      __syncthreads();
+      LeaderState& L = H->L;
+      if (!leader_merge(cx, L)) leader_tail(cx, greedy ? TAIL_LIST_GREEDY : TAIL_LIST_SAMPLE);
+    }
+    return;
+  }
+  if (threadIdx.x == 0) H->listed = listed ? 1u : 0u;
+  __syncthreads();
 
   uint32_t tail = TAIL_NONE;
+  // ---- streamed rows with top-k off and the top-n listed: every CTA derives the
+  // same first op from the merged statistics and starts it without a plan round
+  {
+    uint32_t kmax = 0, kminf = 0xFFFFFFFFu, bad = 0;
+    float M = -INFINITY;
+    for (uint32_t r = 0; r < cx.C; ++r) {
+      const CtaStats& st = H->all[r];
+      bad |= st.bad;
+      kmax = max(kmax, st.kmax);
+      kminf = min(kminf, st.kminf);
+      M = fmaxf(M, st.m);
+    }
+    const bool valid_row = !bad && kmax != kKeyNegInf && cx.T > 0.0f && cx.T < INFINITY && cx.top_p > 0.0f &&
+                           cx.top_k >= 0 && !isinf(scale_x(key_value(kmax), cx.T)) &&
+                           !isinf(scale_x(key_value(kminf), cx.T));
+    if (valid_row && !k_on && listed) {
+      const float m = scale_x(M, cx.T);
+      Plan p{};
+      if (cx.top_p < 1.0f) {
+        p = mass_plan(m, -INFINITY, kminf, cx.T);
+      } else {
+        p.op = OP_GUMBEL;
+        p.theta = -INFINITY;
+      }
+      if (cx.rank == 0) {
+        LeaderState& L = H->L;
+        leader_merge(cx, L);  // writes the top-n from the first-pass list
+        if (threadIdx.x == 0) {
+          L.phase = p.op == OP_MASS ? PH_AFTER_MASS : PH_AFTER_GUMBEL;
+          L.part_is_x = p.op == OP_MASS ? 1 : 0;
+        }
+        __syncthreads();
+      }
+      if (p.op == OP_MASS) op_mass(cx, p);
+      else op_gumbel(cx, p);
+      __syncthreads();
+      cluster_sync();
+    }
+  }
   for (int iter = 0; iter < 64; ++iter) {
     if (cx.rank == 0) {
       const Plan next = leader_step(cx, tail);
@@ -1473,6 +1990,7 @@ __global__ void __launch_bounds__(kThreads, 3) sample_kernel(const __grid_consta
       case OP_NARROW_COUNT: op_narrow_count(cx, p); break;
       case OP_MASS: op_mass(cx, p); break;
       case OP_NARROW_MASS: op_narrow_mass(cx, p); break;
+      case OP_COLLECT_X: op_collect_x(cx, p); break;
       case OP_GUMBEL: op_gumbel(cx, p); break;
       default: break;
     }
