@@ -54,9 +54,12 @@ constexpr int kSubBins = 256;          // narrowing bins
 constexpr int kListCap = 2048;         // leader candidate list capacity
 constexpr int kMaxCluster = 16;
 constexpr int kMaxPart = 32768;        // floats per CTA (128 KB)
-constexpr int kPreferredPart = 12288;  // floats per CTA (48 KB) when the cluster size allows it
+constexpr int kPreferredPart = 20480;  // floats per CTA (80 KB) when the cluster size allows it
 constexpr int kLoadChunks = 4;
 constexpr int kLocalTopK = 64;         // top-k up to this is resolved from per-CTA candidate lists
+constexpr int kXBins = 2048;           // fine bins of x below m (top-p window search)
+constexpr float kXQuant = 4096.0f;     // in-bin offset quantum: 1 / 4096 of a bin
+constexpr float kXRange = 40.0f;       // x more than 40 below m (mass < 5e-18 each) share the last bin
 
 constexpr uint32_t kKeyNegInf = 0x007FFFFFu;  // key(-inf)
 constexpr uint32_t kKeyPosInf = 0xFF800000u;  // key(+inf)
@@ -74,6 +77,8 @@ enum Op : uint32_t {
   OP_NARROW_MASS,
   OP_COLLECT_X,
   OP_GUMBEL,
+  OP_XHIST,
+  OP_EXACT,
 };
 
 enum Tail : uint32_t { TAIL_NONE = 0, TAIL_LIST_GREEDY, TAIL_LIST_SAMPLE, TAIL_STREAM_DONE };
@@ -128,6 +133,8 @@ enum Phase : uint32_t {
   PH_MASS_NARROW,
   PH_AFTER_COLLECT_X,
   PH_AFTER_GUMBEL,
+  PH_AFTER_XHIST,
+  PH_AFTER_EXACT,
 };
 
 // Exact fixed-point mass: e * 2^60 held as four 16-bit limbs; a sum keeps each
@@ -169,13 +176,15 @@ struct __align__(16) SharedHeader {
   Plan plan;
   LeaderState L;
   BestSlot best[kMaxCluster];
+  double ex_above[kMaxCluster];    // leader only: EXACT sums pushed by every CTA
+  double ex_below[kMaxCluster];
   uint32_t need_all[kMaxCluster];  // every CTA: each CTA's first-pass candidate count
   uint32_t ok_all[kMaxCluster];    // every CTA: each CTA's list is usable for top-k
   uint32_t listed;                 // the first-pass list holds the top-n (and top-k) union
   uint32_t list_aux;               // staging count of a local collection / leader small-buffer counter
   uint32_t list_base;              // reserved offset in the leader's list
   uint32_t list_count;
-  uint32_t pad;
+  uint32_t gbound;                 // CTA-wide draw bound (key of a published float32 score)
   unsigned long long mbar[kLoadChunks];
   double red_d[kWarps];
   uint32_t red_u[kWarps * 4];
@@ -184,7 +193,7 @@ struct __align__(16) SharedHeader {
   double scan_d[kWarps];
   uint32_t scan_u[kWarps];
   unsigned long long scan_fx[kWarps][4];
-  double exp_tab[64];
+  double exp_tab[256];
 };
 
 constexpr size_t kScratchBytes = kHistBins * 4;  // 16 KB: raw histogram, later mass / narrowing bins
@@ -228,31 +237,55 @@ __device__ __forceinline__ int mass_bin(const uint32_t* edge, float m, float inv
   return j;
 }
 
+// Fine bin of a finite x <= m: t = fl(fl(m - x) * inv_w) clamped to the last
+// bin, rounded to the nearest integer j.  Every CTA evaluates the same float32
+// operations, so a value falls in the same bin everywhere, and the bin is
+// non-increasing in x (each rounding step is monotone).  With the two
+// roundings of relative size 2^-24 before the last one, bin j holds x with
+// tau = (m - x) * inv_w in [(j - 0.5)(1 - 2^-22), (j + 0.5)(1 + 2^-22)] (the
+// last bin: open above).  `q` is the offset t - j + 0.5 in [0, 1] rounded to
+// a multiple of 1 / kXQuant (error <= 2^-13 with the float32 steps).
+__device__ __forceinline__ int xbin(float x, float m, float inv_w) {
+  const float t = fminf(__fmul_rn(__fsub_rn(m, x), inv_w), static_cast<float>(kXBins - 1));
+  return __float_as_int(__fadd_rn(t, 0x1p23f)) - 0x4B000000;
+}
+__device__ __forceinline__ int xbin_q(float x, float m, float inv_w, uint32_t& q) {
+  const float t = fminf(__fmul_rn(__fsub_rn(m, x), inv_w), static_cast<float>(kXBins - 1));
+  const float r = __fadd_rn(t, 0x1p23f);
+  const float o = __fadd_rn(__fsub_rn(t, __fsub_rn(r, 0x1p23f)), 0.5f);  // t - j exact (Sterbenz)
+  q = __float_as_uint(__fmaf_rn(o, kXQuant, 0x1p23f)) - 0x4B000000u;
+  return __float_as_int(r) - 0x4B000000;
+}
+// Bins per unit of x: the finite x range [x_min, m], at most kXRange wide, on kXBins bins.
+__device__ __forceinline__ float xbin_scale(float m, float x_min) {
+  float r = fminf(__fsub_rn(m, x_min), kXRange);
+  if (!(r > 0.0f)) r = 1.0f;
+  return __fdiv_rn(static_cast<float>(kXBins - 1), r);
+}
+
 // exp(d) for d <= 0 in float64, table-driven (P. T. P. Tang, "Table-driven
 // implementation of the exponential function in IEEE floating-point
-// arithmetic", ACM TOMS 15(2), 1989): d = (64 m + j) ln2/64 + r with
-// |r| <= ln2/128, exp(d) = 2^m * 2^(j/64) * p(r), p the degree-5 Taylor
-// polynomial of exp (truncation < 4e-17).  tab[j] = 2^(j/64).  ln2/64 is split
-// in a 35-bit high part (so n * hi is exact) and the rest.
+// arithmetic", ACM TOMS 15(2), 1989), with a 256-entry table: d = (256 h + j)
+// ln2/256 + r with |r| <= ln2/512, exp(d) = 2^h * 2^(j/256) * p(r), p the cubic
+// Taylor polynomial of exp (relative truncation < 1.5e-13; the one-constant
+// reduction adds < 3e-14).  n = 256 h + j is rounded by adding 1.5 * 2^52, so
+// no integer <-> float64 conversion is issued.  tab[j] = 2^(j/256).  Below
+// d = -700 the result (< 1e-304) is returned as 0: no sum of < 2^20 masses
+// resolves it.
 __device__ __forceinline__ double exp_neg64(double d, const double* tab) {
-  if (d < -708.0) return 0.0;  // below 1e-307: no mass that a sum of < 2^20 terms resolves
-  constexpr double kInvLn2x64 = 92.33248261689366;           // 64 / ln 2
-  constexpr double kLn2d64Hi = 0.010830424695996044;         // ln2 / 64, 35 significant bits
-  constexpr double kLn2d64Lo = 2.5310172166650877e-13;       // ln2 / 64 - high part
-  const int n = __double2int_rn(d * kInvLn2x64);
-  const double nd = static_cast<double>(n);
-  double r = fma(-nd, kLn2d64Hi, d);
-  r = fma(-nd, kLn2d64Lo, r);
-  double p = 1.0 / 120.0;
-  p = fma(p, r, 1.0 / 24.0);
-  p = fma(p, r, 1.0 / 6.0);
-  p = fma(p, r, 0.5);
+  if (d < -700.0) return 0.0;
+  constexpr double kInvLn2x256 = 369.3299304675746;      // 256 / ln 2
+  constexpr double kLn2d256 = 0.0027076061740622863;     // ln 2 / 256
+  constexpr double kShifter = 6755399441055744.0;        // 1.5 * 2^52
+  const double t = fma(d, kInvLn2x256, kShifter);
+  const int n = __double2loint(t);
+  const double nd = t - kShifter;
+  const double r = fma(-nd, kLn2d256, d);
+  double p = fma(r, 1.0 / 6.0, 0.5);
   p = fma(p, r, 1.0);
   p = fma(p, r, 1.0);
-  const double v = tab[n & 63] * p;
-  const int m = n >> 6;  // floor(n / 64)
-  if (m < -1020) return ldexp(v, m);
-  return __hiloint2double(__double2hiint(v) + (m << 20), __double2loint(v));
+  const double v = tab[n & 255] * p;
+  return __hiloint2double(__double2hiint(v) + ((n >> 8) << 20), __double2loint(v));
 }
 
 // e in (0, 1] as the integer round(e * 2^60) (error <= 2^-61): exact sums of up
@@ -320,22 +353,29 @@ __device__ __forceinline__ double gumbel64(uint32_t w) {
   const double u = (static_cast<double>(w >> 9) + 0.5) * 0x1p-23;
   return -log(-log(u));
 }
-// 1 - u for the word, exact in float32.
+// 1 - u for the word, exact in float32: (0x7FFFFF - (w >> 9) + 0.5) * 2^-23,
+// as (1 + (0x7FFFFF - (w >> 9)) * 2^-23) - (1 - 2^-24) from the bits (no
+// int -> float conversion; the subtraction is exact).
 __device__ __forceinline__ float one_minus_u(uint32_t w) {
-  return (static_cast<float>(0x7FFFFFu - (w >> 9)) + 0.5f) * 0x1p-23f;
+  return __fsub_rn(__uint_as_float(0x3F800000u | (~w >> 9)), 0x1.fffffep-1f);
 }
 // Bound on |float32 score - exact score| for score s (logf / log1pf are within
 // 1 ulp; |g| < 17), with a 3x safety factor.
 __device__ __forceinline__ float score_tol(float s) { return 8e-6f + 3e-7f * fabsf(s); }
 
 // Running best of the draw, exact in float64 whenever float32 cannot decide.
+// `shared_key`, when set, is a CTA-wide word holding the order-preserving key
+// of the best float32 score any thread has published: a candidate that cannot
+// beat it is rejected as early as one that cannot beat the thread's own best,
+// so the slow path stays rare for the warp as a whole, not only per thread.
 struct Best {
   float s, x, l;
   double sd;
   uint32_t w;
   int32_t id;
   bool valid, have_sd;
-  __device__ void init() {
+  uint32_t* shared_key;
+  __device__ void init(uint32_t* shared = nullptr) {
     valid = false;
     have_sd = false;
     s = -INFINITY;
@@ -344,6 +384,13 @@ struct Best {
     x = 0.f;
     l = 0.f;
     w = 0;
+    shared_key = shared;
+  }
+  // The best score known to this thread: its own or the CTA's published one.
+  __device__ __forceinline__ float bound_score() const {
+    float b = valid ? s : -INFINITY;
+    if (shared_key) b = fmaxf(b, key_value(*reinterpret_cast<volatile uint32_t*>(shared_key)));
+    return b;
   }
   __device__ double exact() {
     if (!have_sd) {
@@ -352,28 +399,35 @@ struct Best {
     }
     return sd;
   }
+  __device__ __forceinline__ void take(float cs, float cx, float cl, uint32_t cw, int32_t cid) {
+    s = cs; x = cx; l = cl; w = cw; id = cid; valid = true; have_sd = false;
+    if (shared_key) atomicMax(shared_key, fkey(cs));
+  }
   // Offers candidate (x, raw l, Philox word, id).  A cheap test rejects most
-  // candidates first: beating the best needs -log u < exp(x - bound) with
-  // bound below the best's exact score, and -log u >= 1 - u.
+  // candidates first: beating a score s needs -log u < exp(x - bound) with
+  // bound below s's exact value, and -log u >= 1 - u.
   __device__ __forceinline__ void offer(float cx, float cl, uint32_t cw, int32_t cid) {
-    if (valid) {
-      const float bound = s - score_tol(s) - 3e-5f;
+    const float sb = bound_score();
+    if (sb > -INFINITY) {
+      const float bound = sb - score_tol(sb) - 3e-5f;
       const float q = fast_exp2((cx - bound) * 1.4426950408889634f);
       if (one_minus_u(cw) > q * 1.0001f + 1e-30f) return;
     }
     const float cs = cx + gumbel32(cw);
     if (!valid) {
-      s = cs; x = cx; l = cl; w = cw; id = cid; valid = true; have_sd = false;
+      take(cs, cx, cl, cw, cid);
       return;
     }
     const float tol = score_tol(cs) + score_tol(s);
     if (cs > s + tol) {
-      s = cs; x = cx; l = cl; w = cw; id = cid; have_sd = false;
+      take(cs, cx, cl, cw, cid);
     } else if (cs >= s - tol) {
       const double csd = static_cast<double>(cx) + gumbel64(cw);
       const double bsd = exact();
       if (csd > bsd || (csd == bsd && cid < id)) {
-        s = cs; x = cx; l = cl; w = cw; id = cid; sd = csd; have_sd = true;
+        take(cs, cx, cl, cw, cid);
+        sd = csd;
+        have_sd = true;
       }
     }
   }
@@ -493,19 +547,31 @@ __device__ void block_best(double& sd, int32_t& id, float& l, SharedHeader* H) {
   }
 }
 
-// Ascending bitonic sort of n (power of two) u64 keys in shared memory.
+// Ascending bitonic sort of n (power of two, <= 2 * 4 * kThreads) u64 keys in
+// shared memory.  A step compares disjoint pairs, so each thread loads all of
+// its pairs before it stores any: the loads of a step overlap instead of
+// waiting for one another.
 __device__ void bitonic_sort(uint64_t* a, int n) {
+  const int half = n >> 1;
   for (int k = 2; k <= n; k <<= 1) {
     for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = threadIdx.x; i < n; i += kThreads) {
-        const int p = i ^ j;
-        if (p > i) {
-          const uint64_t x = a[i], y = a[p];
-          const bool up = (i & k) == 0;
-          if ((x > y) == up) {
-            a[i] = y;
-            a[p] = x;
-          }
+      uint64_t x[4], y[4];
+      int lo[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int q = static_cast<int>(threadIdx.x) + r * kThreads;
+        lo[r] = ((q & ~(j - 1)) << 1) | (q & (j - 1));  // pair (lo, lo + j)
+        if (q < half) {
+          x[r] = a[lo[r]];
+          y[r] = a[lo[r] + j];
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int q = static_cast<int>(threadIdx.x) + r * kThreads;
+        if (q < half && (x[r] > y[r]) == ((lo[r] & k) == 0)) {
+          a[lo[r]] = y[r];
+          a[lo[r] + j] = x[r];
         }
       }
       __syncthreads();
@@ -826,7 +892,7 @@ __device__ __forceinline__ Fx4 bin_mass(const Ctx& cx, const MassBins& b, int j)
   return f;
 }
 
-// ---- MASS: x = fl(l / T) written in place; survivors' masses on bins of
+// ---- MASS: x = fl(l / T) written in place (unless the part holds x already); survivors' masses on bins of
 // equal width in x below m (exact key edges), exact fixed point.
 __device__ void op_mass(const Ctx& cx, const Plan& p) {
   const MassBins b = mass_bins(cx.scratch);
@@ -840,12 +906,12 @@ __device__ void op_mass(const Ctx& cx, const Plan& p) {
     float v[4] = {v4.x, v4.y, v4.z, v4.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const float x = key_finite(fkey(v[i])) ? scale_x(v[i], cx.T) : -INFINITY;
+      const float x = p.part_is_x ? v[i] : key_finite(fkey(v[i])) ? scale_x(v[i], cx.T) : -INFINITY;
       v[i] = x;
       if (x >= p.theta && x > -INFINITY)
         add_mass(b, mass_bin(b.edge, p.m, inv_step, x, fkey(x)), exp_neg64(static_cast<double>(x) - m, tab));
     }
-    cx.part4[q] = make_float4(v[0], v[1], v[2], v[3]);
+    if (!p.part_is_x) cx.part4[q] = make_float4(v[0], v[1], v[2], v[3]);
   }
 }
 
@@ -891,8 +957,10 @@ __device__ void op_collect_x(const Ctx& cx, const Plan& p) {
     if (threadIdx.x == 0) cx.H->list_aux = 0;
     __syncthreads();
   }
+  if (threadIdx.x == 0) cx.H->gbound = kKeyNegInf;
+  __syncthreads();
   Best b;
-  b.init();
+  b.init(&cx.H->gbound);
   const uint32_t k0 = static_cast<uint32_t>(cx.a->seed), k1 = static_cast<uint32_t>(cx.a->seed >> 32);
   constexpr float kGMax = 16.7f;  // > the largest noise value, -log(-log(1 - 2^-24)) = 16.63
   const int nq = (cx.n4 + kThreads - 1) / kThreads * kThreads;
@@ -920,7 +988,11 @@ __device__ void op_collect_x(const Ctx& cx, const Plan& p) {
         local_append(counter, cx.list, pred[i],
                      (static_cast<uint64_t>(~k[i]) << 32) | static_cast<uint32_t>(cx.g0 + 4 * q + i));
     }
-    if (!any_above || (b.valid && xmax + kGMax < b.s - score_tol(b.s))) continue;
+    if (!any_above) continue;
+    {
+      const float sb = b.bound_score();
+      if (sb > -INFINITY && xmax + kGMax < sb - score_tol(sb)) continue;
+    }
     const long long gid0 = cx.g0 + 4LL * q;
     const uint4 w = philox4x32_10(make_uint4(static_cast<uint32_t>(gid0 >> 2), cx.pos, cx.req, 0u), k0, k1);
 #pragma unroll
@@ -931,42 +1003,184 @@ __device__ void op_collect_x(const Ctx& cx, const Plan& p) {
   push_best(cx, b);
 }
 
+// Cheap test that a candidate with x <= xu cannot beat a score s: that
+// needs -log u < exp(x - bound) for any bound below the best's exact score, and
+// -log u >= 1 - u.
+__device__ __forceinline__ bool gumbel_rejects(float s, float xu, uint32_t w) {
+  const float bound = s - score_tol(s) - 3e-5f;
+  const float q = fast_exp2((xu - bound) * 1.4426950408889634f);
+  return one_minus_u(w) > q * 1.0001f + 1e-30f;
+}
+
 // ---- GUMBEL: argmax of x + g over kept elements (x >= theta), float64-exact;
-// the CTA's best is pushed into the leader's slot [rank].
+// the CTA's best is pushed into the leader's slot [rank].  On raw logits the
+// tests run first on xa = l * (1 / T), within |xa| * 2^-21 of x = fl(l / T), and
+// the division is done only for the rare element that passes them.
 __device__ void op_gumbel(const Ctx& cx, const Plan& p) {
+  if (threadIdx.x == 0) cx.H->gbound = kKeyNegInf;
+  __syncthreads();
   Best b;
-  b.init();
+  b.init(&cx.H->gbound);
   const uint32_t k0 = static_cast<uint32_t>(cx.a->seed), k1 = static_cast<uint32_t>(cx.a->seed >> 32);
   constexpr float kGMax = 16.7f;  // > -log(-log(1 - 2^-24)) = 16.63: the largest noise value
-  const uint32_t raw_lo = p.part_is_x ? 0u : raw_prefilter(p.theta, cx.T);
+  const float invT = __frcp_rn(cx.T);
+  const bool approx = !p.part_is_x && invT < INFINITY;
   for (int q = threadIdx.x; q < cx.n4; q += kThreads) {
     const float4 v4 = cx.part4[q];
     const float v[4] = {v4.x, v4.y, v4.z, v4.w};
-    float x[4];
-    bool kept[4];
+    float xu[4];  // upper bound of x (exact on an x part)
+    bool maybe[4];
     bool any = false;
     float xmax = -INFINITY;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      x[i] = -INFINITY;
       if (p.part_is_x) {
-        x[i] = v[i];
+        xu[i] = v[i];
+      } else if (approx) {
+        const float xa = key_finite(fkey(v[i])) ? v[i] * invT : -INFINITY;
+        xu[i] = xa + fabsf(xa) * 5e-7f + 1e-37f;
       } else {
-        const uint32_t k = fkey(v[i]);
-        if (key_finite(k) && k >= raw_lo) x[i] = scale_x(v[i], cx.T);
+        xu[i] = key_finite(fkey(v[i])) ? scale_x(v[i], cx.T) : -INFINITY;
       }
-      kept[i] = x[i] >= p.theta && x[i] > -INFINITY;
-      if (kept[i]) xmax = fmaxf(xmax, x[i]);
-      any |= kept[i];
+      maybe[i] = xu[i] >= p.theta && xu[i] > -INFINITY;
+      if (maybe[i]) xmax = fmaxf(xmax, xu[i]);
+      any |= maybe[i];
     }
     // no kept element of this group can beat the current best, whatever its noise
-    if (!any || (b.valid && xmax + kGMax < b.s - score_tol(b.s))) continue;
+    if (!any) continue;
+    const float sb = b.bound_score();
+    if (sb > -INFINITY && xmax + kGMax < sb - score_tol(sb)) continue;
+    const long long gid0 = cx.g0 + 4LL * q;
+    const uint4 w = philox4x32_10(make_uint4(static_cast<uint32_t>(gid0 >> 2), cx.pos, cx.req, 0u), k0, k1);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (!maybe[i]) continue;
+      const uint32_t wi = word_of(w, i);
+      if (sb > -INFINITY && gumbel_rejects(sb, xu[i], wi)) continue;
+      const float x = p.part_is_x ? v[i] : scale_x(v[i], cx.T);
+      if (x >= p.theta) b.offer(x, p.part_is_x ? 0.0f : v[i], wi, static_cast<int32_t>(gid0 + i));
+    }
+  }
+  push_best(cx, b);
+}
+
+// ---- XHIST: x = fl(l / T) written in place, and per fine bin below m (p.m,
+// bins per unit p.step) the count of the finite x and the sum of their
+// quantised in-bin offsets; then CTA r sums bins [r, r + 1) * kXBins / C over
+// the cluster into the leader's list area (counts, then offset sums).
+__device__ void op_xhist(const Ctx& cx, const Plan& p) {
+  uint32_t* cnt = reinterpret_cast<uint32_t*>(cx.scratch);
+  uint32_t* qs = cnt + kXBins;
+  for (int i = threadIdx.x; i < 2 * kXBins; i += kThreads) cnt[i] = 0;
+  __syncthreads();
+  for (int q = threadIdx.x; q < cx.n4; q += kThreads) {
+    const float4 v4 = cx.part4[q];
+    float v[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const bool fin = key_finite(fkey(v[i]));
+      const float x = fin ? scale_x(v[i], cx.T) : -INFINITY;
+      v[i] = x;
+      if (fin) {
+        uint32_t qo;
+        const int j = xbin_q(x, p.m, p.step, qo);
+        atomicAdd(&cnt[j], 1u);
+        atomicAdd(&qs[j], qo);
+      }
+    }
+    cx.part4[q] = make_float4(v[0], v[1], v[2], v[3]);
+  }
+  __syncthreads();
+  cluster_sync();  // every CTA's counts are complete
+  uint32_t* tot = reinterpret_cast<uint32_t*>(cluster_ptr(cx.list, 0));
+  const int per = kXBins / static_cast<int>(cx.C);
+  const int j0 = static_cast<int>(cx.rank) * per;
+  for (int j = j0 + threadIdx.x; j < j0 + per; j += kThreads) {
+    tot[j] = cluster_sum(cx, cnt + j);
+    tot[kXBins + j] = cluster_sum(cx, qs + j);
+  }
+}
+
+// Deterministic block sum of a double (fixed shuffle tree, warps in order);
+// thread 0 gets the total.
+__device__ __forceinline__ double block_sum_d0(double v, SharedHeader* H) {
+  v = warp_reduce(v, [](double a, double b) { return a + b; });
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) H->red_d[threadIdx.x >> 5] = v;
+  __syncthreads();
+  double t = 0.0;
+  if (threadIdx.x == 0)
+    for (int i = 0; i < kWarps; ++i) t += H->red_d[i];
+  return t;
+}
+
+// ---- EXACT: with the window of fine bins [lo, hi] that may hold the top-p
+// cut, every finite x above the window is kept for certain (its float64 mass
+// summed, the draw run over it here), every x below it is dropped (mass
+// summed), and the window's members go to the leader's list (sort key ~xkey, id).
+__device__ void op_exact(const Ctx& cx, const Plan& p) {
+  uint32_t* counter = collect_counter(cx);
+  if (cx.rank != 0) {
+    if (threadIdx.x == 0) cx.H->list_aux = 0;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) cx.H->gbound = kKeyNegInf;
+  __syncthreads();
+  Best b;
+  b.init(&cx.H->gbound);
+  const uint32_t k0 = static_cast<uint32_t>(cx.a->seed), k1 = static_cast<uint32_t>(cx.a->seed >> 32);
+  constexpr float kGMax = 16.7f;
+  const double m = p.m;
+  const double* tab = cx.H->exp_tab;
+  const int jlo = static_cast<int>(p.lo), jhi = static_cast<int>(p.hi);
+  double above = 0.0, below = 0.0;
+  const int nq = (cx.n4 + kThreads - 1) / kThreads * kThreads;
+  for (int q = threadIdx.x; q < nq; q += kThreads) {
+    const bool valid = q < cx.n4;
+    const float4 v4 = valid ? cx.part4[q] : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+    const float v[4] = {v4.x, v4.y, v4.z, v4.w};
+    bool win[4], ab[4];
+    bool any_win = false, any_ab = false;
+    float xmax = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const bool fin = v[i] > -INFINITY;
+      const int j = fin ? xbin(v[i], p.m, p.step) : kXBins;
+      win[i] = fin && j >= jlo && j <= jhi;
+      ab[i] = fin && j < jlo;
+      if (fin && !win[i]) {
+        const double e = exp_neg64(static_cast<double>(v[i]) - m, tab);
+        above += ab[i] ? e : 0.0;
+        below += ab[i] ? 0.0 : e;
+      }
+      any_win |= win[i];
+      any_ab |= ab[i];
+      if (ab[i]) xmax = fmaxf(xmax, v[i]);
+    }
+    if (__any_sync(0xFFFFFFFFu, any_win)) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        local_append(counter, cx.list, win[i],
+                     (static_cast<uint64_t>(~fkey(v[i])) << 32) | static_cast<uint32_t>(cx.g0 + 4 * q + i));
+    }
+    if (!any_ab) continue;
+    {
+      const float sb = b.bound_score();
+      if (sb > -INFINITY && xmax + kGMax < sb - score_tol(sb)) continue;
+    }
     const long long gid0 = cx.g0 + 4LL * q;
     const uint4 w = philox4x32_10(make_uint4(static_cast<uint32_t>(gid0 >> 2), cx.pos, cx.req, 0u), k0, k1);
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-      if (kept[i]) b.offer(x[i], p.part_is_x ? 0.0f : v[i], word_of(w, i), static_cast<int32_t>(gid0 + i));
+      if (ab[i]) b.offer(v[i], 0.0f, word_of(w, i), static_cast<int32_t>(gid0 + i));
   }
+  const double ta = block_sum_d0(above, cx.H);
+  const double tb = block_sum_d0(below, cx.H);
+  if (threadIdx.x == 0) {
+    *cluster_ptr(&cx.H->ex_above[cx.rank], 0) = ta;
+    *cluster_ptr(&cx.H->ex_below[cx.rank], 0) = tb;
+  }
+  publish_local_list(cx);
   push_best(cx, b);
 }
 
@@ -1315,8 +1529,10 @@ __device__ Fx4 list_mass_total(const Ctx& cx, const LeaderState& L, int count, f
 // entries with x >= theta (x finite); every thread gets the result.
 __device__ void list_best(const Ctx& cx, const LeaderState& L, int count, bool x_keys, float theta, double& sd,
                           int32_t& id, float& l) {
+  if (threadIdx.x == 0) cx.H->gbound = kKeyNegInf;
+  __syncthreads();
   Best b;
-  b.init();
+  b.init(&cx.H->gbound);
   const uint32_t k0 = static_cast<uint32_t>(cx.a->seed), k1 = static_cast<uint32_t>(cx.a->seed >> 32);
   for (int j = threadIdx.x; j < count; j += kThreads) {
     const uint64_t e = cx.list[j];
@@ -1413,6 +1629,7 @@ __device__ Plan plan_after_theta_k(const Ctx& cx, LeaderState& L) {
     p.op = OP_GUMBEL;
     p.theta = L.theta_k;
     p.part_is_x = L.part_is_x;
+    p.last = 1;
     if (threadIdx.x == 0) L.phase = PH_AFTER_GUMBEL;
   }
   __syncthreads();
@@ -1436,6 +1653,7 @@ __device__ Plan gumbel_plan(LeaderState& L) {
   p.op = OP_GUMBEL;
   p.theta = fmaxf(L.theta_k, L.theta_p);
   p.part_is_x = 1;
+  p.last = 1;
   __syncthreads();
   if (threadIdx.x == 0) L.phase = PH_AFTER_GUMBEL;
   __syncthreads();
@@ -1458,6 +1676,7 @@ __device__ Plan plan_cut_range(LeaderState& L, SharedHeader* H) {
     p.hi = L.nhi;
     p.theta = L.theta_k;
     p.part_is_x = 1;
+    p.last = 1;
     __syncthreads();
     if (threadIdx.x == 0) {
       L.phase = PH_AFTER_COLLECT_X;
@@ -1474,6 +1693,178 @@ __device__ void list_cut(const Ctx& cx, LeaderState& L, int count) {
   const float theta_p = list_mass_cut(cx, L, count, true, -INFINITY, L.cum, L.z);
   if (threadIdx.x == 0) L.theta_p = theta_p;
   __syncthreads();
+}
+
+// Mass bounds of fine bin j from its count n and offset sum qsum: with g(tau)
+// = exp(-tau w), w = 1 / inv_w, and every tau of the bin in [ta, tb], the
+// bin's mass lies between n g(mean tau) (Jensen: g is convex) and the chord of
+// g over [ta, tb] at the mean (above g on the interval).  The mean of t is
+// j - 0.5 + qsum / (n kXQuant) within 2^-12, tau within a factor 1 +- 2^-22
+// of t.  The last bin, open above, is bounded by [0, n g(ta)].
+__device__ __forceinline__ void bin_bounds(int j, uint32_t n, uint32_t qsum, double w, const double* tab,
+                                           double& lo, double& hi) {
+  lo = hi = 0.0;
+  if (n == 0) return;
+  constexpr double eps = 0x1p-22;
+  const double ta = fmax(0.0, (j - 0.5) * (1.0 - eps));
+  const double ga = exp_neg64(-ta * w, tab);
+  if (j == kXBins - 1) {
+    hi = n * ga;
+    return;
+  }
+  const double tb = (j + 0.5) * (1.0 + eps);
+  const double gb = exp_neg64(-tb * w, tab);
+  const double mo = static_cast<double>(qsum) / (static_cast<double>(n) * kXQuant);
+  const double mt_hi = fmin(tb, (j - 0.5 + fmin(1.0, mo + 0x1p-12)) * (1.0 + eps));
+  const double mt_lo = fmax(ta, (j - 0.5 + fmax(0.0, mo - 0x1p-12)) * (1.0 - eps));
+  lo = n * exp_neg64(-mt_hi * w, tab);
+  hi = n * (ga + (gb - ga) * ((mt_lo - ta) / (tb - ta)));
+}
+
+// Window of the top-p cut from the fine bins (cluster totals in the list area:
+// counts, then offset sums).  With P_lo(j), P_hi(j) bounds of the mass above
+// bin j and Z_lo, Z_hi of the total, a non-empty bin is kept for certain when
+// P_hi(j + 1) < top_p Z_lo and dropped for certain when P_lo(j) >= top_p Z_hi
+// (each side with a relative slack of 1e-11 for float64 rounding); the window
+// is the non-empty bins between.  A window that fits the list is resolved by
+// EXACT, a larger one by the fixed-point mass bins.
+__device__ Plan window_plan(const Ctx& cx, LeaderState& L) {
+  constexpr int per = kXBins / kThreads;
+  const uint32_t* cnt = reinterpret_cast<const uint32_t*>(cx.list);
+  const uint32_t* qs = cnt + kXBins;
+  SharedHeader* H = cx.H;
+  const float inv_w = xbin_scale(L.m, scale_x(key_value(L.kminf), L.T));
+  const double w = 1.0 / static_cast<double>(inv_w);
+  const int j0 = static_cast<int>(threadIdx.x) * per;
+  uint32_t c[per];
+  double blo[per], bhi[per];
+  double slo = 0.0, shi = 0.0;
+#pragma unroll
+  for (int k = 0; k < per; ++k) {
+    c[k] = cnt[j0 + k];
+    bin_bounds(j0 + k, c[k], qs[j0 + k], w, H->exp_tab, blo[k], bhi[k]);
+    slo += blo[k];
+    shi += bhi[k];
+  }
+  double zlo, zhi;
+  const double plo0 = block_scan_d(slo, &zlo, H) - slo;
+  const double phi0 = block_scan_d(shi, &zhi, H) - shi;
+  const double tp = static_cast<double>(L.top_p);
+  const double keep_lim = tp * zlo * (1.0 - 1e-11);
+  const double drop_lim = tp * zhi * (1.0 + 1e-11);
+  int jlo = kXBins, jhi = -1;
+  {
+    double plo = plo0, phi = phi0;
+#pragma unroll
+    for (int k = 0; k < per; ++k) {
+      const int j = j0 + k;
+      const double nphi = phi + bhi[k];
+      if (c[k] > 0) {
+        if (!(nphi * (1.0 + 1e-11) < keep_lim)) jlo = min(jlo, j);
+        if (!(plo * (1.0 - 1e-11) >= drop_lim)) jhi = max(jhi, j);
+      }
+      plo += blo[k];
+      phi = nphi;
+    }
+  }
+  jlo = block_min_i(jlo, H);
+  jhi = block_max_i(jhi, H);
+  uint32_t in_win = 0;
+#pragma unroll
+  for (int k = 0; k < per; ++k) in_win += (j0 + k >= jlo && j0 + k <= jhi) ? c[k] : 0u;
+  uint32_t total;
+  block_scan_u(in_win, &total, H);
+  Plan p{};
+  if (total <= static_cast<uint32_t>(kListCap)) {
+    p.op = OP_EXACT;
+    p.lo = static_cast<uint32_t>(jlo);
+    p.hi = static_cast<uint32_t>(jhi);
+    p.m = L.m;
+    p.step = inv_w;
+    p.theta = -INFINITY;
+    p.part_is_x = 1;
+    p.last = 1;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      L.phase = PH_AFTER_EXACT;
+      H->list_count = 0;
+    }
+  } else {
+    p = mass_plan(L.m, -INFINITY, L.kminf, L.T);
+    p.part_is_x = 1;
+    __syncthreads();
+    if (threadIdx.x == 0) L.phase = PH_AFTER_MASS;
+  }
+  __syncthreads();
+  return p;
+}
+
+// The row's token from the leader's best (sd, id) and every CTA's pushed best;
+// its raw logit is read back from the slices.
+__device__ void finish_draw(const Ctx& cx, LeaderState& L, double sd, int32_t id) {
+  const SampleArgs& a = *cx.a;
+  if (threadIdx.x == 0) {
+    for (uint32_t r = 0; r < cx.C; ++r) {
+      const BestSlot& s = cx.H->best[r];
+      if (s.sd > sd || (s.sd == sd && s.id < id)) {
+        sd = s.sd;
+        id = s.id;
+      }
+    }
+    const bool ok = id >= 0 && id < a.V;
+    L.token = ok ? id : -1;
+    float tl = __int_as_float(0x7FC00000);
+    if (ok) {
+      const int sl = id / a.V_s, jj = id - sl * a.V_s;
+      tl = a.slices[sl][static_cast<size_t>(cx.row) * a.V_s + jj];
+    }
+    L.token_l = tl;
+  }
+  __syncthreads();
+}
+
+// After EXACT: Z = A + W + B from the pushed sums and the window's exact
+// masses; the window sorted by (x desc, id asc) gives the cut as the smallest
+// x whose mass of strictly larger values is < top_p Z; the draw adds the
+// window's kept entries to the CTAs' bests.
+__device__ void exact_tail(const Ctx& cx, LeaderState& L) {
+  SharedHeader* H = cx.H;
+  const int count = min(static_cast<int>(H->list_count), kListCap);
+  double A = 0.0, B = 0.0;
+  for (uint32_t r = 0; r < cx.C; ++r) {
+    A += H->ex_above[r];
+    B += H->ex_below[r];
+  }
+  float theta_p = INFINITY;  // no window entry is kept unless the cut is found in it
+  if (count > 0) {
+    const int np2 = pow2_ceil(count);
+    for (int j = count + threadIdx.x; j < np2; j += kThreads) cx.list[j] = ~0ull;
+    __syncthreads();
+    bitonic_sort(cx.list, np2);
+    const double m = static_cast<double>(L.m);
+    const int cs = (np2 + kThreads - 1) / kThreads;
+    const int i0 = min(static_cast<int>(threadIdx.x) * cs, count), i1 = min(i0 + cs, count);
+    double sum = 0.0;
+    for (int i = i0; i < i1; ++i) sum += exp_neg64(static_cast<double>(key_value(entry_key(cx.list[i]))) - m, H->exp_tab);
+    double W;
+    const double incl = block_scan_d(sum, &W, H);
+    const double pz = static_cast<double>(L.top_p) * (A + W + B);
+    double run = A + (incl - sum);
+    int cand = -1;
+    for (int i = i0; i < i1; ++i) {
+      const uint32_t k = entry_key(cx.list[i]);
+      const bool start = i == 0 || entry_key(cx.list[i - 1]) != k;
+      if (start && run < pz) cand = i;
+      run += exp_neg64(static_cast<double>(key_value(k)) - m, H->exp_tab);
+    }
+    const int best = block_max_i(cand, H);
+    if (best >= 0) theta_p = key_value(entry_key(cx.list[best]));
+  }
+  double sd;
+  int32_t id;
+  float l;
+  list_best(cx, L, count, true, theta_p, sd, id, l);
+  finish_draw(cx, L, sd, id);
 }
 
 // Leader: merges the statistics every CTA pushed, validates data and parameters,
@@ -1777,6 +2168,17 @@ __device__ Plan leader_step(const Ctx& cx, uint32_t& tail) {
       break;
     }
 
+    case PH_AFTER_XHIST: {
+      p = window_plan(cx, L);
+      break;
+    }
+
+    case PH_AFTER_EXACT: {
+      exact_tail(cx, L);
+      tail = TAIL_STREAM_DONE;
+      break;
+    }
+
     case PH_AFTER_GUMBEL: {
       if (threadIdx.x == 0) {
         double bsd = -INFINITY;
@@ -1831,7 +2233,7 @@ __device__ void leader_tail(const Ctx& cx, uint32_t tail) {
   write_outputs(cx, L);
 }
 
-__global__ void __launch_bounds__(kThreads, 3) sample_kernel(const __grid_constant__ SampleArgs a) {
+__global__ void __launch_bounds__(kThreads, 2) sample_kernel(const __grid_constant__ SampleArgs a) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   SharedHeader* H = reinterpret_cast<SharedHeader*>(smem_raw);
   uint8_t* scratch = smem_raw + ((sizeof(SharedHeader) + 127) & ~size_t(127));
@@ -1879,7 +2281,7 @@ __global__ void __launch_bounds__(kThreads, 3) sample_kernel(const __grid_consta
   {
     uint32_t* hist = reinterpret_cast<uint32_t*>(scratch);
     for (int i = threadIdx.x; i < kHistBins; i += kThreads) hist[i] = 0;
-    for (int j = threadIdx.x; j < 64; j += kThreads) H->exp_tab[j] = exp2(static_cast<double>(j) / 64.0);
+    for (int j = threadIdx.x; j < 256; j += kThreads) H->exp_tab[j] = exp2(static_cast<double>(j) / 256.0);
     if (threadIdx.x == 0) {
       H->L.phase = PH_START;
       H->list_count = 0;
@@ -1955,7 +2357,9 @@ __global__ void __launch_bounds__(kThreads, 3) sample_kernel(const __grid_consta
       const float m = scale_x(M, cx.T);
       Plan p{};
       if (cx.top_p < 1.0f) {
-        p = mass_plan(m, -INFINITY, kminf, cx.T);
+        p.op = OP_XHIST;
+        p.m = m;
+        p.step = xbin_scale(m, scale_x(key_value(kminf), cx.T));
       } else {
         p.op = OP_GUMBEL;
         p.theta = -INFINITY;
@@ -1964,15 +2368,23 @@ __global__ void __launch_bounds__(kThreads, 3) sample_kernel(const __grid_consta
         LeaderState& L = H->L;
         leader_merge(cx, L);  // writes the top-n from the first-pass list
         if (threadIdx.x == 0) {
-          L.phase = p.op == OP_MASS ? PH_AFTER_MASS : PH_AFTER_GUMBEL;
-          L.part_is_x = p.op == OP_MASS ? 1 : 0;
+          L.phase = p.op == OP_XHIST ? PH_AFTER_XHIST : PH_AFTER_GUMBEL;
+          L.part_is_x = p.op == OP_XHIST ? 1 : 0;
         }
         __syncthreads();
       }
-      if (p.op == OP_MASS) op_mass(cx, p);
+      if (p.op == OP_XHIST) op_xhist(cx, p);
       else op_gumbel(cx, p);
       __syncthreads();
       cluster_sync();
+      if (p.op == OP_GUMBEL) {
+        // what remains is the leader's alone: the CTAs' bests are in its slots
+        if (cx.rank == 0) {
+          leader_step(cx, tail);
+          leader_tail(cx, tail);
+        }
+        return;
+      }
     }
   }
   for (int iter = 0; iter < 64; ++iter) {
@@ -1992,13 +2404,20 @@ __global__ void __launch_bounds__(kThreads, 3) sample_kernel(const __grid_consta
       case OP_NARROW_MASS: op_narrow_mass(cx, p); break;
       case OP_COLLECT_X: op_collect_x(cx, p); break;
       case OP_GUMBEL: op_gumbel(cx, p); break;
+      case OP_EXACT: op_exact(cx, p); break;
       default: break;
     }
     __syncthreads();
     cluster_sync();
     if (p.last) break;  // what remains of the row is the leader's alone
   }
-  if (cx.rank == 0) leader_tail(cx, tail);
+  if (cx.rank == 0) {
+    // a last op after which only the leader's own memory is read: its step runs here
+    const uint32_t ph = H->L.phase;
+    if (tail == TAIL_NONE && (ph == PH_AFTER_EXACT || ph == PH_AFTER_GUMBEL || ph == PH_AFTER_COLLECT_X))
+      leader_step(cx, tail);
+    leader_tail(cx, tail);
+  }
 }
 
 // ------------------------------------------------------------------ host side
