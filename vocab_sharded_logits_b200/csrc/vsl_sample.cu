@@ -57,6 +57,9 @@ constexpr int kMaxPart = 32768;        // floats per CTA (128 KB)
 constexpr int kPreferredPart = 20480;  // floats per CTA (80 KB) when the cluster size allows it
 constexpr int kLoadChunks = 4;
 constexpr int kLocalTopK = 64;         // top-k up to this is resolved from per-CTA candidate lists
+constexpr int32_t kDeferred = -2;      // token id of a row the streaming kernel leaves to the cluster kernel
+constexpr int kStreamChunk = 2048;     // streaming kernel: floats per ring stage (8 KB)
+constexpr int kStreamStages = 6;       // streaming kernel: ring depth (40 KB in flight per CTA)
 constexpr int kXBins = 2048;           // fine bins of x below m (top-p window search)
 constexpr float kXQuant = 4096.0f;     // in-bin offset quantum: 1 / 4096 of a bin
 constexpr float kXRange = 40.0f;       // x more than 40 below m (mass < 5e-18 each) share the last bin
@@ -186,6 +189,7 @@ struct __align__(16) SharedHeader {
   uint32_t list_count;
   uint32_t gbound;                 // CTA-wide draw bound (key of a published float32 score)
   unsigned long long mbar[kLoadChunks];
+  unsigned long long ring_bar[kStreamStages];  // streaming kernel: one per ring stage
   double red_d[kWarps];
   uint32_t red_u[kWarps * 4];
   float red_f[kWarps * 2];
@@ -1352,13 +1356,14 @@ __device__ void list_key_range(const Ctx& cx, int count, uint32_t& lo, uint32_t&
 }
 
 // The r-th largest key among the list entries (1 <= r <= count), by 256-bin
-// rank narrowing on the key.
-__device__ uint32_t list_rank_key(const Ctx& cx, int count, uint32_t r) {
+// rank narrowing on the key.  With a limit on the narrowing rounds, the lower
+// end of the key range still holding the r-th key (a key <= the r-th).
+__device__ uint32_t list_rank_key(const Ctx& cx, int count, uint32_t r, int max_rounds = 64) {
   uint32_t lo, hi;
   list_key_range(cx, count, lo, hi);
   uint32_t* cnt = reinterpret_cast<uint32_t*>(cx.scratch);
   SharedHeader* H = cx.H;
-  while (lo != hi) {
+  for (int round = 0; lo != hi && round < max_rounds; ++round) {
     const uint32_t width = hi - lo;
     const int bits = 32 - __clz(width);
     const int shift = bits > 8 ? bits - 8 : 0;
@@ -2248,6 +2253,8 @@ __global__ void __launch_bounds__(kThreads, 2) sample_kernel(const __grid_consta
   cx.C = static_cast<uint32_t>(a.C);
   cx.rank = cluster_ctarank();
   cx.row = static_cast<int>(blockIdx.x / a.C);
+  // rows the streaming kernel resolved (it runs first on the same stream) are done
+  if (a.token_ids[cx.row] != kDeferred) return;
   cx.g0 = static_cast<long long>(cx.rank) * a.part;
   const long long g1 = min(cx.g0 + a.part, static_cast<long long>(a.V));
   const int n = g1 > cx.g0 ? static_cast<int>(g1 - cx.g0) : 0;
@@ -2420,6 +2427,12 @@ __global__ void __launch_bounds__(kThreads, 2) sample_kernel(const __grid_consta
   }
 }
 
+}  // namespace vsl
+
+#include "vsl_stream.cuh"
+
+namespace vsl {
+
 // ------------------------------------------------------------------ host side
 size_t sample_smem_bytes(int part) {
   return ((sizeof(SharedHeader) + 127) & ~size_t(127)) + kScratchBytes + kListBytes +
@@ -2471,8 +2484,40 @@ static cudaError_t prepare_sample_kernel() {
     }
     cudaGetLastError();
   }
+  e = cudaFuncSetAttribute(stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(stream_smem_bytes()));
+  if (e != cudaSuccess) return e;
   done = true;
   return cudaSuccess;
+}
+
+// Streaming kernel geometry: CTAs per row so that R * C covers two CTAs per
+// SM where the batch is small (at most 8, a portable cluster), and the part
+// of each (a multiple of 4 floats: every part starts 16-byte aligned).
+static void stream_geometry(int R, long long V, int sms, int* cluster, int* part) {
+  int c = 1;
+  while (c < 8 && static_cast<long long>(R) * c < 2LL * sms) c <<= 1;
+  long long p = (V + c - 1) / c;
+  p = (p + 3) / 4 * 4;
+  *cluster = c;
+  *part = static_cast<int>(p);
+}
+
+static cudaError_t launch_with_cluster(const void* fn, const SampleArgs& a, int grid, size_t smem, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(a.C);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  void* args[] = {const_cast<SampleArgs*>(&a)};
+  return cudaLaunchKernelExC(&cfg, fn, args);
 }
 
 cudaError_t launch_sample(const float* const* logits, int R, int S, int V_s, const vsl_row_params* params,
@@ -2498,21 +2543,21 @@ cudaError_t launch_sample(const float* const* logits, int R, int S, int V_s, con
   a.n_logprobs = n_logprobs;
   int c = 0, part = 0;
   if (!sample_geometry(a.V, &c, &part)) return cudaErrorInvalidValue;
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  }
+  // 1) rows resolved from streamed candidates; the rest are marked kDeferred
+  SampleArgs sa = a;
+  stream_geometry(R, a.V, sms, &sa.C, &sa.part);
+  e = launch_with_cluster(reinterpret_cast<const void*>(stream_kernel), sa, R * sa.C, stream_smem_bytes(), stream);
+  if (e != cudaSuccess) return e;
+  // 2) the deferred rows, with the row held in the cluster's shared memory
   a.C = c;
   a.part = part;
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(static_cast<unsigned>(R) * c, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = sample_smem_bytes(part);
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = c;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, sample_kernel, a);
+  return launch_with_cluster(reinterpret_cast<const void*>(sample_kernel), a, R * c, sample_smem_bytes(part), stream);
 }
 
 }  // namespace vsl

@@ -1,0 +1,380 @@
+// vsl_stream.cuh - streaming sampler for rows resolved from a candidate list
+// (greedy rows, and sampling rows with 0 < top_k <= kStreamMaxK), included by
+// vsl_sample.cu after the cluster kernel it shares the list toolkit with.
+//
+// Such a row needs one pass over its logits: the statistics of the softmax
+// (max, sum of exp, NaN / +inf, smallest finite value) and every logit that
+// can be among the top max(n, k), ties included.  Its part of the row streams
+// from HBM through a ring of shared-memory stages fed by 1-D bulk copies, so
+// the row is never held on chip: while a stage is scanned the next ones are
+// in flight.  Candidates above a running threshold go to a list; when the
+// list fills up it is compacted and the threshold raised.  The cluster's
+// leader then resolves the row from the merged list with the same toolkit as
+// the cluster kernel.  A row this kernel does not take (or whose candidates
+// do not fit) gets the token id kDeferred, and the cluster kernel, launched
+// next on the same stream, samples exactly those rows.
+#pragma once
+
+namespace vsl {
+
+constexpr int kStreamCap = 4096;      // candidate list capacity while streaming
+constexpr int kStreamMaxK = 1024;     // largest top-k resolved from streamed candidates
+
+constexpr size_t kStreamListBytes = static_cast<size_t>(kStreamCap) * 8;
+constexpr size_t kStreamRingBytes = static_cast<size_t>(kStreamStages) * kStreamChunk * 4;
+
+__host__ __device__ __forceinline__ size_t stream_smem_bytes() {
+  return ((sizeof(SharedHeader) + 127) & ~size_t(127)) + kScratchBytes + kStreamListBytes + kStreamRingBytes;
+}
+
+// Rows this kernel resolves: valid parameters, and greedy or a top-k the list holds.
+__device__ __forceinline__ bool stream_row(const vsl_row_params& p, int V) {
+  if (!(p.top_p > 0.0f) || p.top_k < 0) return false;
+  if (p.temperature == 0.0f) return true;
+  return p.temperature > 0.0f && p.temperature < INFINITY && p.top_k > 0 && p.top_k < V &&
+         p.top_k <= kStreamMaxK;
+}
+
+// Lowest raw key a compaction may keep when the rank-`r` value found is `v`:
+// for a sampling row every l that can scale to the same x as v (the
+// temperature maps up to a few adjacent floats to one x) stays listed.
+__device__ __forceinline__ uint32_t stream_floor(uint32_t key, float T) {
+  if (!(T > 0.0f) || !key_finite(key)) return key;
+  return min(key, raw_prefilter(scale_x(key_value(key), T), T));
+}
+
+// Keeps the list entries whose key is >= a new threshold at or below the
+// list's r-th largest key (after `rounds` 256-bin narrowings, or exact when
+// that leaves less than a chunk of room; lowered by stream_floor), when that
+// raises `thr`.  In place: every thread holds its entries in registers before
+// any is written back.  Every thread returns the threshold in force and sets
+// `left` to the list's count after it (no thread re-reads the shared counter,
+// which the next chunk's appends may already be moving).  Called by the whole
+// block at a point no thread appends.
+__device__ uint32_t stream_compact(const Ctx& cx, uint32_t r, uint32_t thr, int rounds, uint32_t& left) {
+  SharedHeader* H = cx.H;
+  left = H->list_count;
+  const int count = min(static_cast<int>(left), kStreamCap);
+  if (count <= static_cast<int>(r)) return thr;
+  constexpr int per = kStreamCap / kThreads;
+  uint64_t e[per];
+#pragma unroll
+  for (int i = 0; i < per; ++i) {
+    const int idx = static_cast<int>(threadIdx.x) + i * kThreads;
+    e[i] = idx < count ? cx.list[idx] : 0ull;
+  }
+  uint32_t cut = stream_floor(list_rank_key(cx, count, r, rounds), cx.T);
+  uint32_t kept = 0, total = 0;
+  for (int pass = 0; pass < 2; ++pass) {
+    kept = 0;
+#pragma unroll
+    for (int i = 0; i < per; ++i) {
+      const int idx = static_cast<int>(threadIdx.x) + i * kThreads;
+      kept += (idx < count && entry_key(e[i]) >= cut) ? 1u : 0u;
+    }
+    block_scan_u(kept, &total, H);
+    if (pass == 1 || rounds >= 64 || total <= static_cast<uint32_t>(kStreamCap - kStreamChunk)) break;
+    cut = stream_floor(list_rank_key(cx, count, r), cx.T);
+  }
+  if (cut <= thr) return thr;
+  left = total;
+  uint32_t off = block_scan_u(kept, &total, H) - kept;
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < per; ++i) {
+    const int idx = static_cast<int>(threadIdx.x) + i * kThreads;
+    if (idx < count && entry_key(e[i]) >= cut) cx.list[off++] = e[i];
+  }
+  if (threadIdx.x == 0) H->list_count = total;
+  __syncthreads();
+  return cut;
+}
+
+// Issues the bulk copies of chunk `c` of this CTA's part [g0, g0 + n) into
+// ring stage c % kStreamStages (thread 0; chunks in increasing order, so the
+// slice `s` holding the chunk's start only moves forward).  A chunk may span
+// two slices.
+__device__ __forceinline__ void stream_issue(const SampleArgs& a, int row, int g0, int n, int c, int& s,
+                                             float* ring, unsigned long long* bars, uint64_t pol) {
+  const int stage = c % kStreamStages;
+  const int e0 = g0 + c * kStreamChunk;
+  const int e1 = g0 + min((c + 1) * kStreamChunk, n);
+  const uint32_t bar = smem_u32(&bars[stage]);
+  mbar_arrive_expect_tx(bar, static_cast<uint32_t>(e1 - e0) * 4u);
+  float* dst = ring + static_cast<size_t>(stage) * kStreamChunk;
+  int g = e0;
+  while (g < e1) {
+    while (g >= (s + 1) * a.V_s) ++s;
+    const int s_end = min((s + 1) * a.V_s, e1);
+    const float* src = a.slices[s] + static_cast<size_t>(row) * a.V_s + (g - s * a.V_s);
+    bulk_load(smem_u32(dst + (g - e0)), src, static_cast<uint32_t>(s_end - g) * 4u, bar, pol);
+    g = s_end;
+  }
+}
+
+// Statistics a thread keeps over the logits it scans.  The sum of exp runs
+// against the thread's largest finite value m (prescaled: mL = m log2 e); m
+// starts at -1e30 so that a thread that never sees a finite value adds only
+// exp(-inf) = 0.  NaN of either sign makes the sum NaN; +inf shows in kmax.
+struct ScanStats {
+  uint32_t kmax;   // largest key
+  uint32_t kmf;    // smallest (key - key(-inf) - 1) mod 2^32: the smallest key above key(-inf)
+  float m, mL, s;
+};
+constexpr float kScanNoMax = -1e30f;
+
+// Scans one ring stage (nq float4 of it) with first id `gid`: statistics and
+// candidates (key >= thr) appended to the list (`seen`: this warp's list end).
+// A thread takes kPer float4; a warp with any candidate reserves the slots of
+// all of them with one atomic.
+template <bool kFull>
+__device__ __forceinline__ void stream_scan(const float4* st4, int nq, uint32_t thr, uint32_t gid, ScanStats& st,
+                                            uint32_t& seen, uint32_t* counter, uint64_t* list) {
+  constexpr float kLog2e = 1.4426950408889634f;
+  constexpr int kPer = kStreamChunk / 4 / kThreads;
+  const int lane = threadIdx.x & 31;
+  uint32_t k[kPer][4];
+  bool any = false;
+#pragma unroll
+  for (int it = 0; it < kPer; ++it) {
+    const int q = static_cast<int>(threadIdx.x) + it * kThreads;
+    const bool valid = kFull || q < nq;
+    const float4 v4 = valid ? st4[q] : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+    const float v[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      // order-preserving key of v + 0 (-0 becomes +0); padding keys are 0 (never listed)
+      const uint32_t b = __float_as_uint(__fadd_rn(v[i], 0.0f));
+      k[it][i] = valid ? b ^ (static_cast<uint32_t>(static_cast<int32_t>(b) >> 31) | 0x80000000u) : 0u;
+      st.kmf = min(st.kmf, valid ? k[it][i] - (kKeyNegInf + 1u) : 0xFFFFFFFFu);
+    }
+    const uint32_t kq = max(max(k[it][0], k[it][1]), max(k[it][2], k[it][3]));
+    if (kq > st.kmax) {
+      st.kmax = kq;
+      if (kq > kKeyNegInf) {  // a new largest value: rescale the sum to it
+        const float mn = key_value(kq);
+        const float mnL = mn * kLog2e;
+        st.s *= fast_exp2(st.mL - mnL);
+        st.m = mn;
+        st.mL = mnL;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) st.s += fast_exp2(fmaf(v[i], kLog2e, -st.mL));
+    any |= kq >= thr && valid;
+  }
+  if (!__any_sync(0xFFFFFFFFu, any)) return;
+  uint32_t mask[kPer][4];
+  uint32_t total = 0;
+#pragma unroll
+  for (int it = 0; it < kPer; ++it)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      mask[it][i] = __ballot_sync(0xFFFFFFFFu, k[it][i] >= thr && k[it][i] != 0u);
+      total += __popc(mask[it][i]);
+    }
+  uint32_t base = 0;
+  if (lane == 0) base = atomicAdd(counter, total);
+  base = __shfl_sync(0xFFFFFFFFu, base, 0);
+  seen = max(seen, base + total);
+  const uint32_t below = (1u << lane) - 1u;
+#pragma unroll
+  for (int it = 0; it < kPer; ++it)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t idx = base + __popc(mask[it][i] & below);
+      if (((mask[it][i] >> lane) & 1u) && idx < static_cast<uint32_t>(kStreamCap)) {
+        const int q = static_cast<int>(threadIdx.x) + it * kThreads;
+        list[idx] = (static_cast<uint64_t>(~k[it][i]) << 32) | (gid + 4u * static_cast<uint32_t>(q) + i);
+      }
+      base += __popc(mask[it][i]);
+    }
+}
+
+// One CTA per (row, part) of a cluster of C CTAs per row; grid R * C.
+__global__ void __launch_bounds__(kThreads, 2) stream_kernel(const __grid_constant__ SampleArgs a) {
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  SharedHeader* H = reinterpret_cast<SharedHeader*>(smem_raw);
+  uint8_t* scratch = smem_raw + ((sizeof(SharedHeader) + 127) & ~size_t(127));
+  uint64_t* list = reinterpret_cast<uint64_t*>(scratch + kScratchBytes);
+  float* ring = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(list) + kStreamListBytes);
+
+  Ctx cx;
+  cx.a = &a;
+  cx.H = H;
+  cx.scratch = scratch;
+  cx.list = list;
+  cx.C = static_cast<uint32_t>(a.C);
+  cx.rank = cluster_ctarank();
+  cx.row = static_cast<int>(blockIdx.x / a.C);
+  const vsl_row_params prm = a.params[cx.row];
+  if (!stream_row(prm, a.V)) {
+    if (cx.rank == 0 && threadIdx.x == 0) a.token_ids[cx.row] = kDeferred;
+    return;  // the whole cluster leaves: the row is the cluster kernel's
+  }
+  cx.T = prm.temperature;
+  cx.top_k = prm.top_k;
+  cx.top_p = prm.top_p;
+  cx.req = prm.request_id;
+  cx.pos = prm.position;
+  cx.g0 = static_cast<long long>(cx.rank) * a.part;
+  const long long g1 = min(cx.g0 + a.part, static_cast<long long>(a.V));
+  const int n = g1 > cx.g0 ? static_cast<int>(g1 - cx.g0) : 0;
+  cx.n4 = n >> 2;
+  cx.part4 = nullptr;
+  const int nch = (n + kStreamChunk - 1) / kStreamChunk;
+  const bool greedy = prm.temperature == 0.0f;
+  uint32_t R = a.n_logprobs > 0 ? static_cast<uint32_t>(a.n_logprobs) : 1u;
+  if (!greedy) R = max(R, static_cast<uint32_t>(prm.top_k));
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStreamStages; ++s) mbar_init(smem_u32(&H->ring_bar[s]), 1);
+    fence_mbar_init();
+    H->list_count = 0;
+  }
+  for (int j = threadIdx.x; j < 256; j += kThreads) H->exp_tab[j] = exp2(static_cast<double>(j) / 256.0);
+  __syncthreads();
+  // thread 0 keeps kStreamStages - 1 chunks in flight ahead of the one scanned
+  const uint64_t pol = policy_evict_first();
+  const int g0 = static_cast<int>(cx.g0);
+  int s_issue = 0;
+  if (threadIdx.x == 0)
+    for (int c = 0; c < min(nch, kStreamStages - 1); ++c) stream_issue(a, cx.row, g0, n, c, s_issue, ring, H->ring_bar, pol);
+
+  constexpr float kLog2e = 1.4426950408889634f;
+  uint32_t thr = 0;  // every key (-inf included) is a candidate until the first compaction
+  ScanStats st{0u, 0xFFFFFFFFu, kScanNoMax, kScanNoMax * kLog2e, 0.0f};
+  bool load_ok = true;
+  bool dropped = false;  // some candidate was not listed: the row goes to the cluster kernel
+  uint32_t seen = 0;     // this warp's list end after its appends of the current chunk
+  const int lane = threadIdx.x & 31;
+  for (int c = 0; c < nch; ++c) {
+    const int stage = c % kStreamStages;
+    // refill the stage scanned in the previous iteration (its barrier has passed)
+    if (threadIdx.x == 0 && c + kStreamStages - 1 < nch)
+      stream_issue(a, cx.row, g0, n, c + kStreamStages - 1, s_issue, ring, H->ring_bar, pol);
+    if (load_ok && !mbar_wait_bounded(smem_u32(&H->ring_bar[stage]), static_cast<uint32_t>(c / kStreamStages) & 1u)) {
+      if (threadIdx.x == 0) atomicOr(a.err, kErrSampleLoad);
+      load_ok = false;
+    }
+    const float4* st4 = reinterpret_cast<const float4*>(ring + static_cast<size_t>(stage) * kStreamChunk);
+    const int nq = min(kStreamChunk, n - c * kStreamChunk) >> 2;
+    const uint32_t gid = static_cast<uint32_t>(g0 + c * kStreamChunk);
+    if (nq == kStreamChunk / 4) stream_scan<true>(st4, nq, thr, gid, st, seen, &H->list_count, list);
+    else stream_scan<false>(st4, nq, thr, gid, st, seen, &H->list_count, list);
+    // the stage is consumed and the appends are visible; the barrier also
+    // tells every thread whether the list has less than a chunk of room left
+    const bool full = __syncthreads_or(seen > static_cast<uint32_t>(kStreamCap - kStreamChunk)) != 0;
+    seen = 0;
+    if (full && !dropped) {
+      uint32_t left;
+      dropped = H->list_count > static_cast<uint32_t>(kStreamCap);
+      thr = stream_compact(cx, R, thr, 2, left);
+      // no room for another chunk (ties at the threshold): the row is deferred, stop listing
+      if (left > static_cast<uint32_t>(kStreamCap - kStreamChunk)) dropped = true;
+      if (dropped) thr = 0xFFFFFFFFu;
+    }
+  }
+
+  // ---- CTA statistics (the cluster kernel's CtaStats layout)
+  // (m, s) pairs merge by rescaling to the larger m; kScanNoMax pairs add 0
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    st.kmax = max(st.kmax, __shfl_xor_sync(0xFFFFFFFFu, st.kmax, o));
+    st.kmf = min(st.kmf, __shfl_xor_sync(0xFFFFFFFFu, st.kmf, o));
+    const float om = __shfl_xor_sync(0xFFFFFFFFu, st.m, o);
+    const float os = __shfl_xor_sync(0xFFFFFFFFu, st.s, o);
+    const float nm = fmaxf(st.m, om);
+    st.s = st.s * fast_exp2((st.m - nm) * kLog2e) + os * fast_exp2((om - nm) * kLog2e);
+    st.m = nm;
+  }
+  const int warp = threadIdx.x >> 5;
+  if (lane == 0) {
+    H->red_u[warp * 4 + 0] = st.kmax;
+    H->red_u[warp * 4 + 2] = st.kmf;
+    H->red_u[warp * 4 + 3] = load_ok ? 0u : 1u;
+    H->red_f[warp * 2 + 0] = st.m;
+    H->red_f[warp * 2 + 1] = st.s;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t ka = 0, kf = 0xFFFFFFFFu, bad = 0;
+    float M = kScanNoMax;
+    for (int i = 0; i < kWarps; ++i) {
+      ka = max(ka, H->red_u[i * 4 + 0]);
+      kf = min(kf, H->red_u[i * 4 + 2]);
+      bad |= H->red_u[i * 4 + 3];
+      M = fmaxf(M, H->red_f[i * 2]);
+    }
+    float S = 0.0f;
+    for (int i = 0; i < kWarps; ++i) S += H->red_f[i * 2 + 1] * fast_exp2((H->red_f[i * 2] - M) * kLog2e);
+    // NaN of either sign turns the sum NaN; +inf (and a NaN's key) lies at or above key(+inf)
+    bad |= (ka >= kKeyPosInf || isnan(S)) ? 1u : 0u;
+    H->stats.kmax = ka;
+    H->stats.kminf = kf == 0xFFFFFFFFu ? kf : kf + (kKeyNegInf + 1u);  // smallest finite key
+    H->stats.bad = bad;
+    const bool none = !(M > kScanNoMax);
+    H->stats.m = none ? -INFINITY : M;
+    H->stats.s = none ? 0.0f : S;
+  }
+  // exact local top R: the union of the parts' lists then holds the row's top R
+  dropped |= H->list_count > static_cast<uint32_t>(kStreamCap);
+  uint32_t own = 0;
+  if (!dropped) thr = stream_compact(cx, R, thr, 64, own);
+  own = dropped ? 0u : min(own, static_cast<uint32_t>(kStreamCap));
+  const uint32_t overflow = dropped ? 1u : 0u;
+
+  // ---- merge into the leader: statistics, thresholds, candidates
+  if (cx.C > 1) cluster_sync();
+  if (cx.rank != 0) {
+    if (threadIdx.x == 0) {
+      H->list_base = atom_add_dsmem_u32(mapa(smem_u32(&H->list_count), 0), own);
+      *cluster_ptr(&H->all[cx.rank], 0) = H->stats;
+      cluster_ptr(H->need_all, 0)[cx.rank] = thr;
+      cluster_ptr(H->ok_all, 0)[cx.rank] = overflow;
+    }
+    __syncthreads();
+    const uint32_t base = H->list_base;
+    uint64_t* dst = cluster_ptr(list, 0);
+    for (uint32_t i = threadIdx.x; i < own; i += kThreads)
+      if (base + i < static_cast<uint32_t>(kStreamCap)) dst[base + i] = list[i];
+    __syncthreads();
+    cluster_sync();
+    return;
+  }
+  if (threadIdx.x == 0) {
+    H->all[0] = H->stats;
+    H->need_all[0] = thr;
+    H->ok_all[0] = overflow;
+  }
+  __syncthreads();
+  if (cx.C > 1) cluster_sync();
+
+  // ---- leader: the row from the merged list
+  uint32_t defer = H->list_count > static_cast<uint32_t>(kListCap) ? 1u : 0u;
+  for (uint32_t r = 0; r < cx.C; ++r) defer |= H->ok_all[r];
+  if (defer) {
+    if (threadIdx.x == 0) a.token_ids[cx.row] = kDeferred;
+    return;
+  }
+  const int count = static_cast<int>(H->list_count);
+  if (threadIdx.x == 0) H->listed = 1;
+  __syncthreads();
+  LeaderState& L = H->L;
+  if (leader_merge(cx, L)) return;  // flagged row: outputs written
+  if (!greedy) {
+    // every value that can scale to theta_k must have been a candidate in every part
+    const float theta_k = scale_x(key_value(list_rank_key(cx, count, static_cast<uint32_t>(L.r_k))), L.T);
+    const uint32_t lo = raw_prefilter(theta_k, L.T);
+    uint32_t miss = 0;
+    for (uint32_t r = 0; r < cx.C; ++r) miss |= H->need_all[r] > lo ? 1u : 0u;
+    if (miss) {
+      if (threadIdx.x == 0) a.token_ids[cx.row] = kDeferred;
+      return;
+    }
+    list_sample_tail(cx, L, count);
+  }
+  write_outputs(cx, L);
+}
+
+}  // namespace vsl
