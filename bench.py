@@ -44,24 +44,33 @@ def _peaks():
         return 6650.0, 1590.0, 1400.0, "fallback"
 
 
-_KERNEL_SOURCES = {"logits_local_kernel": "vsl_gemm.cu", "sample_kernel": "vsl_sample.cu"}
+# The timed units of a step and the sources each is built from.  "sample" is
+# one call of the sampler: the streaming kernel (greedy and top-k <= 1024 rows)
+# followed by the cluster kernel (the other rows).
+_KERNEL_SOURCES = {"logits_local_kernel": ["vsl_gemm.cu"], "sample": ["vsl_sample.cu", "vsl_stream.cuh"]}
+
+
+def _source_sha(kernel):
+    import hashlib
+    h = hashlib.sha256()
+    for name in _KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "vocab_sharded_logits_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
 
 
 def _recorded_traffic(kernel, workload):
-    """DRAM bytes per launch recorded from an ncu capture in profiles/<kernel>_<workload>.md,
-    or None when there is none or the kernel source changed since (sha256 differs)."""
-    import hashlib
+    """DRAM bytes per call recorded from an ncu capture in profiles/<kernel>_<workload>.md,
+    or None when there is none or the sources changed since (sha256 over them differs)."""
     prof = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
-    src = os.path.join(ROOT, "vocab_sharded_logits_b200", "csrc", _KERNEL_SOURCES[kernel])
-    if not (os.path.exists(prof) and os.path.exists(src)):
+    if not os.path.exists(prof):
         return None
     fields = {}
     for line in open(prof):
         if ":" in line and line.split(":", 1)[0] in ("traffic_bytes_per_launch", "source_sha256"):
             k, v = line.split(":", 1)
             fields[k] = v.strip()
-    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
-    if fields.get("source_sha256") != sha:
+    if fields.get("source_sha256") != _source_sha(kernel):
         return None
     try:
         return int(fields["traffic_bytes_per_launch"])
@@ -351,7 +360,7 @@ def run_gpu(args, w):
             roof = {"kernel": "logits_local_kernel", "bound": "tensor", "achieved": gemm_flops / (gemm_ms / 1e3) / 1e12,
                     "peak": tf_sus, "unit": "TFLOP/s"}
     else:
-        roof = {"kernel": "sample_kernel", "bound": "hbm", "achieved": samp_bytes / (samp_ms / 1e3) / 1e9,
+        roof = {"kernel": "sample", "bound": "hbm", "achieved": samp_bytes / (samp_ms / 1e3) / 1e9,
                 "peak": hbm_peak, "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["peak_source"] = peak_kind
@@ -371,7 +380,7 @@ def run_gpu(args, w):
             "sampler_hbm_gbs_in_step": samp_bytes / (samp_ms / 1e3) / 1e9,
         },
         "e2e": {"value": e2e_value, "unit": "rows/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": 3 * args.steps,  # logits_local_kernel, stream_kernel, sample_kernel
         "clocks": clk,
         "cpu_baseline": None,
     }
