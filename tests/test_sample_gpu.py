@@ -168,3 +168,35 @@ def test_draw_frequencies_chi_square(cuda_device):
     if exp_m[-1] == 0:
         obs_m, exp_m = obs_m[:-1], exp_m[:-1]
     assert stats.chisquare(obs_m, exp_m).pvalue > 1e-3
+
+
+@pytest.mark.parametrize("R", [8, 80, 150, 300])
+def test_streaming_geometries(cuda_device, R):
+    """The streaming kernel's CTAs per row (8, 4, 2, 1 for these batch sizes on a
+    148-SM part) and the cluster kernel's rows in one batch: greedy, small and
+    large top-k (several compactions) and top-k off, sampled rows vs the oracle."""
+    V, S = 151936, 4
+    rng = np.random.default_rng(R)
+    logits = torch.from_numpy((rng.standard_normal((R, V)) * 1.3).astype(np.float32))
+    kinds = np.arange(R) % 4
+    T = np.where(kinds == 0, 0.0, rng.uniform(0.5, 1.5, R)).astype(np.float32)
+    k = np.choose(kinds, [0, 20, 900, 0]).astype(np.int32)
+    p = np.where(kinds == 3, 0.9, rng.uniform(0.8, 1.0, R)).astype(np.float32)
+    params = (T, k, p, np.arange(R), np.arange(R) * 7 + 3)
+    gpu = run_sampler(logits, params, 99, 20, S, cuda_device)
+    rows = sorted(set(np.random.default_rng(1).choice(R, min(R, 12), replace=False).tolist()) | {0, 1, 2, 3})
+    compare(gpu, logits.numpy(), params, 99, 20, rows)
+
+
+def test_streaming_tie_flood_defers(cuda_device):
+    """Rows whose top-k ties overflow the streaming kernel's candidate list (a few
+    distinct values over the whole vocabulary) are resolved by the cluster kernel."""
+    V, S, R = 151936, 4, 6
+    rng = np.random.default_rng(3)
+    logits = np.round(rng.standard_normal((R, V)) * 2).astype(np.float32) / 2  # ~16 distinct values
+    T = np.full(R, 1.0, np.float32)
+    k = np.array([5, 50, 1000, 300, 1, 20], np.int32)
+    p = np.array([0.9, 1.0, 0.99, 0.5, 1.0, 0.8], np.float32)
+    params = (T, k, p, np.arange(R), np.arange(R))
+    gpu = run_sampler(torch.from_numpy(logits), params, 5, 20, S, cuda_device)
+    compare(gpu, logits, params, 5, 20, range(R))

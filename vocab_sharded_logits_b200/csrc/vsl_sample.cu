@@ -551,36 +551,76 @@ __device__ void block_best(double& sd, int32_t& id, float& l, SharedHeader* H) {
   }
 }
 
-// Ascending bitonic sort of n (power of two, <= 2 * 4 * kThreads) u64 keys in
-// shared memory.  A step compares disjoint pairs, so each thread loads all of
-// its pairs before it stores any: the loads of a step overlap instead of
-// waiting for one another.
-__device__ void bitonic_sort(uint64_t* a, int n) {
-  const int half = n >> 1;
-  for (int k = 2; k <= n; k <<= 1) {
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      uint64_t x[4], y[4];
-      int lo[4];
+// Ascending bitonic sort of n u64 keys in shared memory, n a power of two,
+// 2 <= n <= 8 * kThreads.  Thread t holds elements [t E, t E + E) in registers
+// (E = max(1, n / kThreads); threads past n hold ~0 and only swap among
+// themselves): a step of stride j < E swaps registers of one thread, j < 32 E
+// goes through warp shuffles, and only the larger strides go through shared
+// memory, so 2048 keys take 6 barrier-separated steps instead of 66.
+template <int E>
+__device__ __forceinline__ void sort_step_regs(uint64_t (&v)[E], int base, int k, int j) {
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int q = static_cast<int>(threadIdx.x) + r * kThreads;
-        lo[r] = ((q & ~(j - 1)) << 1) | (q & (j - 1));  // pair (lo, lo + j)
-        if (q < half) {
-          x[r] = a[lo[r]];
-          y[r] = a[lo[r] + j];
-        }
-      }
+  for (int i = 0; i < E; ++i) {
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int q = static_cast<int>(threadIdx.x) + r * kThreads;
-        if (q < half && (x[r] > y[r]) == ((lo[r] & k) == 0)) {
-          a[lo[r]] = y[r];
-          a[lo[r] + j] = x[r];
-        }
+    for (int jj = 1; jj < E; jj <<= 1) {
+      if (jj == j && (i & jj) == 0) {
+        const bool up = ((base + i) & k) == 0;
+        const uint64_t x = v[i], y = v[i + jj];
+        const bool sw = (x > y) == up;
+        v[i] = sw ? y : x;
+        v[i + jj] = sw ? x : y;
       }
-      __syncthreads();
     }
   }
+}
+template <int E>
+__device__ void bitonic_sort_e(uint64_t* a, int n) {
+  uint64_t v[E];
+  const int base = static_cast<int>(threadIdx.x) * E;
+#pragma unroll
+  for (int i = 0; i < E; ++i) v[i] = base + i < n ? a[base + i] : ~0ull;
+  for (int k = 2; k <= n; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      if (j < E) {
+        sort_step_regs<E>(v, base, k, j);
+      } else if (j < 32 * E) {
+        const int lj = j / E;  // the partner is lane ^ lj, same register
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+          const uint64_t y = __shfl_xor_sync(0xFFFFFFFFu, v[i], lj);
+          const int e = base + i;
+          const bool keep_min = ((e & j) == 0) == ((e & k) == 0);
+          v[i] = keep_min ? min(v[i], y) : max(v[i], y);
+        }
+      } else {
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < E; ++i)
+          if (base + i < n) a[base + i] = v[i];
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+          const int e = base + i;
+          if (e < n) {
+            const uint64_t y = a[e ^ j];
+            const bool keep_min = ((e & j) == 0) == ((e & k) == 0);
+            v[i] = keep_min ? min(v[i], y) : max(v[i], y);
+          }
+        }
+      }
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < E; ++i)
+    if (base + i < n) a[base + i] = v[i];
+  __syncthreads();
+}
+__device__ void bitonic_sort(uint64_t* a, int n) {
+  if (n <= kThreads) bitonic_sort_e<1>(a, n);
+  else if (n <= 2 * kThreads) bitonic_sort_e<2>(a, n);
+  else if (n <= 4 * kThreads) bitonic_sort_e<4>(a, n);
+  else bitonic_sort_e<8>(a, n);
 }
 
 // ------------------------------------------------------------------ per-CTA context
@@ -1580,6 +1620,100 @@ __device__ void list_sample_tail(const Ctx& cx, LeaderState& L, int count) {
   list_gumbel(cx, L, count, false, theta);
 }
 
+// Sorts `count` distinct sort keys (~key << 32 | id) ascending from `in` into
+// `out` (count <= kListCap; `out` distinct from `in`).  Up to 2 * kThreads
+// entries every thread ranks its entries against all of them in one pass of
+// broadcast reads and stores each at its rank; a longer list is copied and
+// sorted by the bitonic network.
+__device__ void sort_entries(const uint64_t* in, int count, uint64_t* out) {
+  if (count <= 2 * kThreads) {
+    const int t = static_cast<int>(threadIdx.x);
+    const uint64_t e0 = t < count ? in[t] : ~0ull;
+    const uint64_t e1 = t + kThreads < count ? in[t + kThreads] : ~0ull;
+    int r0 = 0, r1 = 0;
+    for (int j = 0; j < count; ++j) {
+      const uint64_t y = in[j];
+      r0 += y < e0 ? 1 : 0;
+      r1 += y < e1 ? 1 : 0;
+    }
+    if (t < count) out[r0] = e0;
+    if (t + kThreads < count) out[r1] = e1;
+    __syncthreads();
+    return;
+  }
+  const int np2 = pow2_ceil(count);
+  for (int j = threadIdx.x; j < np2; j += kThreads) out[j] = j < count ? in[j] : ~0ull;
+  __syncthreads();
+  bitonic_sort(out, np2);
+}
+
+// Resolves a list row from its list sorted by (raw key desc, id asc) in `buf`
+// (every top-n entry and every top-k survivor present): the top-n is the
+// prefix; greedy takes the first entry; a sampling row keeps x >= theta_k (a
+// prefix: x = fl(l / T) is monotone in l), cuts top-p on float64 masses summed
+// in that order, and draws over the kept prefix.  Fills L.token / L.token_l.
+__device__ void list_resolve_sorted(const Ctx& cx, LeaderState& L, const uint64_t* buf, int count, bool sample) {
+  const SampleArgs& a = *cx.a;
+  SharedHeader* H = cx.H;
+  const int n = a.n_logprobs;
+  for (int j = threadIdx.x; j < n; j += kThreads) {
+    const uint64_t e = buf[min(j, count - 1)];
+    a.topn_ids[static_cast<size_t>(cx.row) * n + j] = entry_id(e);
+    a.topn_logprob[static_cast<size_t>(cx.row) * n + j] = key_value(entry_key(e)) - L.lse;
+  }
+  if (!sample) {
+    if (threadIdx.x == 0) {
+      L.token = entry_id(buf[0]);
+      L.token_l = key_value(entry_key(buf[0]));
+    }
+    __syncthreads();
+    return;
+  }
+  const float T = L.T;
+  const float theta_k = L.r_k > 0 ? scale_x(key_value(entry_key(buf[min(L.r_k, count) - 1])), T) : -INFINITY;
+  // survivors: the prefix of entries with x >= theta_k (and x finite)
+  int s_own = 0;
+  for (int j = threadIdx.x; j < count; j += kThreads) {
+    const float x = scale_x(key_value(entry_key(buf[j])), T);
+    if (x >= theta_k && x > -INFINITY) s_own = max(s_own, j + 1);
+  }
+  const int s = block_max_i(s_own, H);
+  float theta = theta_k;
+  if (L.top_p < 1.0f && s > 0) {
+    const double m = static_cast<double>(scale_x(key_value(entry_key(buf[0])), T));
+    const int cs = (s + kThreads - 1) / kThreads;
+    const int i0 = min(static_cast<int>(threadIdx.x) * cs, s), i1 = min(i0 + cs, s);
+    double sum = 0.0;
+    for (int i = i0; i < i1; ++i)
+      sum += exp_neg64(static_cast<double>(scale_x(key_value(entry_key(buf[i])), T)) - m, H->exp_tab);
+    double Z;
+    const double incl = block_scan_d(sum, &Z, H);
+    const double pz = static_cast<double>(L.top_p) * Z;
+    double run = incl - sum;  // mass of the entries before i0
+    int cand = -1;
+    float prev = i0 > 0 ? scale_x(key_value(entry_key(buf[i0 - 1])), T) : INFINITY;
+    for (int i = i0; i < i1; ++i) {
+      const float x = scale_x(key_value(entry_key(buf[i])), T);
+      if (x != prev && run < pz) cand = i;  // first of its x value, mass of larger x below top_p * Z
+      run += exp_neg64(static_cast<double>(x) - m, H->exp_tab);
+      prev = x;
+    }
+    const int cut = block_max_i(cand, H);
+    if (cut >= 0) theta = fmaxf(theta, scale_x(key_value(entry_key(buf[cut])), T));
+  }
+  // the draw over the kept prefix
+  Ctx sub = cx;
+  sub.list = const_cast<uint64_t*>(buf);
+  list_gumbel(sub, L, s, false, theta);
+}
+
+// Sorts the leader's list into the scratch area and resolves the row (list tails).
+__device__ void list_resolve(const Ctx& cx, LeaderState& L, int count, bool sample) {
+  uint64_t* buf = reinterpret_cast<uint64_t*>(cx.scratch);
+  sort_entries(cx.list, count, buf);
+  list_resolve_sorted(cx, L, buf, count, sample);
+}
+
 __device__ Plan narrow_plan(LeaderState& L, uint32_t op) {
   Plan p{};
   p.op = op;
@@ -2224,17 +2358,8 @@ __device__ void leader_tail(const Ctx& cx, uint32_t tail) {
     write_outputs(cx, L);
     return;
   }
-  if (!L.topn_done) list_topn(cx, L, count);
-  if (tail == TAIL_LIST_GREEDY) {
-    const uint64_t top = list_max_entry(cx, count);
-    if (threadIdx.x == 0) {
-      L.token = entry_id(top);
-      L.token_l = key_value(entry_key(top));
-    }
-    __syncthreads();
-  } else {
-    list_sample_tail(cx, L, count);
-  }
+  // the list holds the top-n and every top-k survivor: resolve from it sorted
+  list_resolve(cx, L, count, tail == TAIL_LIST_SAMPLE);
   write_outputs(cx, L);
 }
 

@@ -358,13 +358,15 @@ __global__ void __launch_bounds__(kThreads, 2) stream_kernel(const __grid_consta
     return;
   }
   const int count = static_cast<int>(H->list_count);
-  if (threadIdx.x == 0) H->listed = 1;
+  if (threadIdx.x == 0) H->listed = 0;  // leader_merge only merges statistics and flags
   __syncthreads();
   LeaderState& L = H->L;
   if (leader_merge(cx, L)) return;  // flagged row: outputs written
+  uint64_t* buf = reinterpret_cast<uint64_t*>(cx.scratch);
+  sort_entries(list, count, buf);
   if (!greedy) {
     // every value that can scale to theta_k must have been a candidate in every part
-    const float theta_k = scale_x(key_value(list_rank_key(cx, count, static_cast<uint32_t>(L.r_k))), L.T);
+    const float theta_k = scale_x(key_value(entry_key(buf[min(L.r_k, count) - 1])), L.T);
     const uint32_t lo = raw_prefilter(theta_k, L.T);
     uint32_t miss = 0;
     for (uint32_t r = 0; r < cx.C; ++r) miss |= H->need_all[r] > lo ? 1u : 0u;
@@ -372,8 +374,8 @@ __global__ void __launch_bounds__(kThreads, 2) stream_kernel(const __grid_consta
       if (threadIdx.x == 0) a.token_ids[cx.row] = kDeferred;
       return;
     }
-    list_sample_tail(cx, L, count);
   }
+  list_resolve_sorted(cx, L, buf, count, !greedy);
   write_outputs(cx, L);
 }
 
