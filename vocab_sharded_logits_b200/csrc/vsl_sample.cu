@@ -40,6 +40,7 @@
 #include <cfloat>
 #include <cmath>
 #include <cstdint>
+#include <mutex>
 
 #include "vsl_internal.h"
 #include "vsl_ptx.cuh"
@@ -58,6 +59,11 @@ constexpr int kPreferredPart = 20480;  // floats per CTA (80 KB) when the cluste
 constexpr int kLoadChunks = 4;
 constexpr int kLocalTopK = 64;         // top-k up to this is resolved from per-CTA candidate lists
 constexpr int32_t kDeferred = -2;      // token id of a row the streaming kernel leaves to the cluster kernel
+constexpr int kStreamMaxK = 1024;      // largest top-k resolved from streamed candidates
+// sample_kernel row selection: rows whose token id reads kDeferred (after the
+// streaming kernel), or every row the streaming kernel does not take (run
+// alongside it).  stream_kernel: kStreamMarks makes it mark those rows kDeferred.
+constexpr int kSelectDeferred = 0, kSelectOthers = 1, kStreamMarks = 1;
 constexpr int kStreamChunk = 2048;     // streaming kernel: floats per ring stage (8 KB)
 constexpr int kStreamStages = 6;       // streaming kernel: ring depth (40 KB in flight per CTA)
 constexpr int kXBins = 2048;           // fine bins of x below m (top-p window search)
@@ -97,6 +103,7 @@ struct SampleArgs {
   uint32_t* err;
   unsigned long long seed;
   int R, S, V_s, V, C, part, n_logprobs;
+  int select;  // rows a kernel takes: see kSelectDeferred, kSelectOthers, kStreamMarks
 };
 
 // Per-CTA results the leader reads through distributed shared memory.
@@ -204,6 +211,15 @@ constexpr size_t kScratchBytes = kHistBins * 4;  // 16 KB: raw histogram, later 
 constexpr size_t kListBytes = kListCap * 8;
 
 // ------------------------------------------------------------------ small helpers
+// Rows the streaming kernel resolves: valid parameters, and greedy or a top-k
+// its candidate list holds.
+__device__ __forceinline__ bool stream_row(const vsl_row_params& p, int V) {
+  if (!(p.top_p > 0.0f) || p.top_k < 0) return false;
+  if (p.temperature == 0.0f) return true;
+  return p.temperature > 0.0f && p.temperature < INFINITY && p.top_k > 0 && p.top_k < V &&
+         p.top_k <= kStreamMaxK;
+}
+
 // Order-preserving key of a float, computed on its bits with integer operations
 // only (no float arithmetic, so NaN payloads cannot change the result): -0 and
 // +0 share one key, larger keys are larger values, -inf < finite < +inf.
@@ -273,11 +289,11 @@ __device__ __forceinline__ float xbin_scale(float m, float x_min) {
 // ln2/256 + r with |r| <= ln2/512, exp(d) = 2^h * 2^(j/256) * p(r), p the cubic
 // Taylor polynomial of exp (relative truncation < 1.5e-13; the one-constant
 // reduction adds < 3e-14).  n = 256 h + j is rounded by adding 1.5 * 2^52, so
-// no integer <-> float64 conversion is issued.  tab[j] = 2^(j/256).  Below
-// d = -700 the result (< 1e-304) is returned as 0: no sum of < 2^20 masses
-// resolves it.
+// no integer <-> float64 conversion is issued.  tab[j] = 2^(j/256).  d is
+// clamped at -700 (the result there, < 1e-304, is below what any sum of < 2^20
+// masses resolves), so no branch is taken.
 __device__ __forceinline__ double exp_neg64(double d, const double* tab) {
-  if (d < -700.0) return 0.0;
+  d = fmax(d, -700.0);  // exp(-700) < 1e-304: no sum of < 2^20 masses resolves it
   constexpr double kInvLn2x256 = 369.3299304675746;      // 256 / ln 2
   constexpr double kLn2d256 = 0.0027076061740622863;     // ln 2 / 256
   constexpr double kShifter = 6755399441055744.0;        // 1.5 * 2^52
@@ -407,16 +423,27 @@ struct Best {
     s = cs; x = cx; l = cl; w = cw; id = cid; valid = true; have_sd = false;
     if (shared_key) atomicMax(shared_key, fkey(cs));
   }
-  // Offers candidate (x, raw l, Philox word, id).  A cheap test rejects most
-  // candidates first: beating a score s needs -log u < exp(x - bound) with
-  // bound below s's exact value, and -log u >= 1 - u.
-  __device__ __forceinline__ void offer(float cx, float cl, uint32_t cw, int32_t cid) {
+  // log2(e) times a value below the exact score of the best known score s
+  // (kNoBound when there is none): the rejection test's reference.
+  static constexpr float kNoBound = -3.0e38f;
+  __device__ __forceinline__ float bound_l2e() const {
     const float sb = bound_score();
-    if (sb > -INFINITY) {
-      const float bound = sb - score_tol(sb) - 3e-5f;
-      const float q = fast_exp2((cx - bound) * 1.4426950408889634f);
-      if (one_minus_u(cw) > q * 1.0001f + 1e-30f) return;
-    }
+    return sb > -INFINITY ? (sb - score_tol(sb) - 3e-5f) * 1.4426950408889634f : kNoBound;
+  }
+  // Cheap test that candidate (x, word) cannot beat the bound: beating a score
+  // needs -log u < exp(x - bound), and -log u >= 1 - u.
+  static __device__ __forceinline__ bool rejects(float bl2e, float cx, uint32_t cw) {
+    const float q = fast_exp2(fmaf(cx, 1.4426950408889634f, -bl2e));
+    return one_minus_u(cw) > q * 1.0001f + 1e-30f;
+  }
+  // Offers candidate (x, raw l, Philox word, id).
+  __device__ __forceinline__ void offer(float cx, float cl, uint32_t cw, int32_t cid) {
+    const float bl = bound_l2e();
+    if (bl != kNoBound && rejects(bl, cx, cw)) return;
+    offer_passed(cx, cl, cw, cid);
+  }
+  // The exact comparison for a candidate that passed the cheap test.
+  __device__ __forceinline__ void offer_passed(float cx, float cl, uint32_t cw, int32_t cid) {
     const float cs = cx + gumbel32(cw);
     if (!valid) {
       take(cs, cx, cl, cw, cid);
@@ -1039,9 +1066,11 @@ __device__ void op_collect_x(const Ctx& cx, const Plan& p) {
     }
     const long long gid0 = cx.g0 + 4LL * q;
     const uint4 w = philox4x32_10(make_uint4(static_cast<uint32_t>(gid0 >> 2), cx.pos, cx.req, 0u), k0, k1);
+    const float bl = b.bound_l2e();
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-      if (above[i]) b.offer(v[i], 0.0f, word_of(w, i), static_cast<int32_t>(gid0 + i));
+      if (above[i] && (bl == Best::kNoBound || !Best::rejects(bl, v[i], word_of(w, i))))
+        b.offer_passed(v[i], 0.0f, word_of(w, i), static_cast<int32_t>(gid0 + i));
   }
   publish_local_list(cx);
   push_best(cx, b);
@@ -1096,13 +1125,14 @@ __device__ void op_gumbel(const Ctx& cx, const Plan& p) {
     if (sb > -INFINITY && xmax + kGMax < sb - score_tol(sb)) continue;
     const long long gid0 = cx.g0 + 4LL * q;
     const uint4 w = philox4x32_10(make_uint4(static_cast<uint32_t>(gid0 >> 2), cx.pos, cx.req, 0u), k0, k1);
+    const float bl = b.bound_l2e();
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       if (!maybe[i]) continue;
       const uint32_t wi = word_of(w, i);
-      if (sb > -INFINITY && gumbel_rejects(sb, xu[i], wi)) continue;
+      if (bl != Best::kNoBound && Best::rejects(bl, xu[i], wi)) continue;
       const float x = p.part_is_x ? v[i] : scale_x(v[i], cx.T);
-      if (x >= p.theta) b.offer(x, p.part_is_x ? 0.0f : v[i], wi, static_cast<int32_t>(gid0 + i));
+      if (x >= p.theta) b.offer_passed(x, p.part_is_x ? 0.0f : v[i], wi, static_cast<int32_t>(gid0 + i));
     }
   }
   push_best(cx, b);
@@ -1110,8 +1140,9 @@ __device__ void op_gumbel(const Ctx& cx, const Plan& p) {
 
 // ---- XHIST: x = fl(l / T) written in place, and per fine bin below m (p.m,
 // bins per unit p.step) the count of the finite x and the sum of their
-// quantised in-bin offsets; then CTA r sums bins [r, r + 1) * kXBins / C over
-// the cluster into the leader's list area (counts, then offset sums).
+// quantised in-bin offsets; then CTA r replaces its own bins [r, r + 1) *
+// kXBins / C with their sums over the cluster (only CTA r reads that slice of
+// any CTA, so the slice can be overwritten in place).
 __device__ void op_xhist(const Ctx& cx, const Plan& p) {
   uint32_t* cnt = reinterpret_cast<uint32_t*>(cx.scratch);
   uint32_t* qs = cnt + kXBins;
@@ -1136,12 +1167,13 @@ __device__ void op_xhist(const Ctx& cx, const Plan& p) {
   }
   __syncthreads();
   cluster_sync();  // every CTA's counts are complete
-  uint32_t* tot = reinterpret_cast<uint32_t*>(cluster_ptr(cx.list, 0));
   const int per = kXBins / static_cast<int>(cx.C);
   const int j0 = static_cast<int>(cx.rank) * per;
   for (int j = j0 + threadIdx.x; j < j0 + per; j += kThreads) {
-    tot[j] = cluster_sum(cx, cnt + j);
-    tot[kXBins + j] = cluster_sum(cx, qs + j);
+    const uint32_t tc = cluster_sum(cx, cnt + j);
+    const uint32_t tq = cluster_sum(cx, qs + j);
+    cnt[j] = tc;
+    qs[j] = tq;
   }
 }
 
@@ -1214,9 +1246,11 @@ __device__ void op_exact(const Ctx& cx, const Plan& p) {
     }
     const long long gid0 = cx.g0 + 4LL * q;
     const uint4 w = philox4x32_10(make_uint4(static_cast<uint32_t>(gid0 >> 2), cx.pos, cx.req, 0u), k0, k1);
+    const float bl = b.bound_l2e();
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-      if (ab[i]) b.offer(v[i], 0.0f, word_of(w, i), static_cast<int32_t>(gid0 + i));
+      if (ab[i] && (bl == Best::kNoBound || !Best::rejects(bl, v[i], word_of(w, i))))
+        b.offer_passed(v[i], 0.0f, word_of(w, i), static_cast<int32_t>(gid0 + i));
   }
   const double ta = block_sum_d0(above, cx.H);
   const double tb = block_sum_d0(below, cx.H);
@@ -1441,6 +1475,30 @@ __device__ void list_topn(const Ctx& cx, const LeaderState& L, int count) {
   const SampleArgs& a = *cx.a;
   const int n = a.n_logprobs;
   if (n <= 0) return;
+  if (count <= 2 * kThreads) {
+    // sort keys are distinct: an entry of rank r < n (entries smaller than it) is the (r+1)-th
+    const int t = static_cast<int>(threadIdx.x);
+    const uint64_t e0 = t < count ? cx.list[t] : ~0ull;
+    const uint64_t e1 = t + kThreads < count ? cx.list[t + kThreads] : ~0ull;
+    int r0 = 0, r1 = 0;
+#pragma unroll 8
+    for (int j = 0; j < count; ++j) {
+      const uint64_t y = cx.list[j];
+      r0 += y < e0 ? 1 : 0;
+      r1 += y < e1 ? 1 : 0;
+    }
+    const size_t o = static_cast<size_t>(cx.row) * n;
+    if (t < count && r0 < n) {
+      a.topn_ids[o + r0] = entry_id(e0);
+      a.topn_logprob[o + r0] = key_value(entry_key(e0)) - L.lse;
+    }
+    if (t + kThreads < count && r1 < n) {
+      a.topn_ids[o + r1] = entry_id(e1);
+      a.topn_logprob[o + r1] = key_value(entry_key(e1)) - L.lse;
+    }
+    __syncthreads();
+    return;
+  }
   const uint32_t kn = list_rank_key(cx, count, static_cast<uint32_t>(n));
   // gather every entry with key >= the n-th key into a small buffer, sort it
   uint64_t* buf = reinterpret_cast<uint64_t*>(cx.scratch);
@@ -1631,6 +1689,7 @@ __device__ void sort_entries(const uint64_t* in, int count, uint64_t* out) {
     const uint64_t e0 = t < count ? in[t] : ~0ull;
     const uint64_t e1 = t + kThreads < count ? in[t + kThreads] : ~0ull;
     int r0 = 0, r1 = 0;
+#pragma unroll 8
     for (int j = 0; j < count; ++j) {
       const uint64_t y = in[j];
       r0 += y < e0 ? 1 : 0;
@@ -1838,24 +1897,23 @@ __device__ void list_cut(const Ctx& cx, LeaderState& L, int count) {
 // = exp(-tau w), w = 1 / inv_w, and every tau of the bin in [ta, tb], the
 // bin's mass lies between n g(mean tau) (Jensen: g is convex) and the chord of
 // g over [ta, tb] at the mean (above g on the interval).  The mean of t is
-// j - 0.5 + qsum / (n kXQuant) within 2^-12, tau within a factor 1 +- 2^-22
-// of t.  The last bin, open above, is bounded by [0, n g(ta)].
-__device__ __forceinline__ void bin_bounds(int j, uint32_t n, uint32_t qsum, double w, const double* tab,
-                                           double& lo, double& hi) {
+// j - 0.5 + qsum / (n kXQuant) within 2^-12 (float32 here: its error is far
+// below that slack), tau within a factor 1 +- 2^-22 of t.  The last bin, open
+// above, is bounded by [0, n g(ta)].  ga = g(ta), gb = g(tb) are passed in.
+__device__ __forceinline__ void bin_bounds(int j, uint32_t n, uint32_t qsum, double w, double ga, double gb,
+                                           const double* tab, double& lo, double& hi) {
   lo = hi = 0.0;
   if (n == 0) return;
   constexpr double eps = 0x1p-22;
-  const double ta = fmax(0.0, (j - 0.5) * (1.0 - eps));
-  const double ga = exp_neg64(-ta * w, tab);
   if (j == kXBins - 1) {
     hi = n * ga;
     return;
   }
+  const double ta = fmax(0.0, (j - 0.5) * (1.0 - eps));
   const double tb = (j + 0.5) * (1.0 + eps);
-  const double gb = exp_neg64(-tb * w, tab);
-  const double mo = static_cast<double>(qsum) / (static_cast<double>(n) * kXQuant);
-  const double mt_hi = fmin(tb, (j - 0.5 + fmin(1.0, mo + 0x1p-12)) * (1.0 + eps));
-  const double mt_lo = fmax(ta, (j - 0.5 + fmax(0.0, mo - 0x1p-12)) * (1.0 - eps));
+  const float mo = __fdiv_rn(static_cast<float>(qsum), static_cast<float>(n) * kXQuant);
+  const double mt_hi = fmin(tb, (j - 0.5 + fmin(1.0, static_cast<double>(mo) + 0x1p-12)) * (1.0 + eps));
+  const double mt_lo = fmax(ta, (j - 0.5 + fmax(0.0, static_cast<double>(mo) - 0x1p-12)) * (1.0 - eps));
   lo = n * exp_neg64(-mt_hi * w, tab);
   hi = n * (ga + (gb - ga) * ((mt_lo - ta) / (tb - ta)));
 }
@@ -1869,21 +1927,34 @@ __device__ __forceinline__ void bin_bounds(int j, uint32_t n, uint32_t qsum, dou
 // EXACT, a larger one by the fixed-point mass bins.
 __device__ Plan window_plan(const Ctx& cx, LeaderState& L) {
   constexpr int per = kXBins / kThreads;
-  const uint32_t* cnt = reinterpret_cast<const uint32_t*>(cx.list);
-  const uint32_t* qs = cnt + kXBins;
   SharedHeader* H = cx.H;
+  // this thread's bins [j0, j0 + per) lie in one CTA's slice: read the totals there
+  const uint32_t owner = (static_cast<uint32_t>(threadIdx.x) * per) / (kXBins / cx.C);
+  const uint32_t* cnt = cluster_ptr(reinterpret_cast<const uint32_t*>(cx.scratch), owner);
+  const uint32_t* qs = cnt + kXBins;
   const float inv_w = xbin_scale(L.m, scale_x(key_value(L.kminf), L.T));
   const double w = 1.0 / static_cast<double>(inv_w);
   const int j0 = static_cast<int>(threadIdx.x) * per;
   uint32_t c[per];
   double blo[per], bhi[per];
   double slo = 0.0, shi = 0.0;
+  {
+    // g at the bin ends: geometric in j (ratios qa, qb), started exactly for this thread's run
+    constexpr double eps = 0x1p-22;
+    const double wa = (1.0 - eps) * w, wb = (1.0 + eps) * w;
+    const double qa = exp_neg64(-wa, H->exp_tab), qb = exp_neg64(-wb, H->exp_tab);
+    double ga = exp_neg64(-fmax(0.0, (j0 - 0.5) * (1.0 - eps)) * w, H->exp_tab);
+    double gb = exp_neg64(-(j0 + 0.5) * (1.0 + eps) * w, H->exp_tab);
 #pragma unroll
-  for (int k = 0; k < per; ++k) {
-    c[k] = cnt[j0 + k];
-    bin_bounds(j0 + k, c[k], qs[j0 + k], w, H->exp_tab, blo[k], bhi[k]);
-    slo += blo[k];
-    shi += bhi[k];
+    for (int k = 0; k < per; ++k) {
+      c[k] = cnt[j0 + k];
+      bin_bounds(j0 + k, c[k], qs[j0 + k], w, ga, gb, H->exp_tab, blo[k], bhi[k]);
+      slo += blo[k];
+      shi += bhi[k];
+      ga = j0 + k == 0 ? exp_neg64(-0.5 * wa, H->exp_tab) : ga * qa;
+      gb *= qb;
+    }
+    // the recurrences' rounding (< 1e-15 relative) is covered by the 1e-11 slack below
   }
   double zlo, zhi;
   const double plo0 = block_scan_d(slo, &zlo, H) - slo;
@@ -1913,8 +1984,10 @@ __device__ Plan window_plan(const Ctx& cx, LeaderState& L) {
   for (int k = 0; k < per; ++k) in_win += (j0 + k >= jlo && j0 + k <= jhi) ? c[k] : 0u;
   uint32_t total;
   block_scan_u(in_win, &total, H);
+  // the window's entries go after the first-pass list, which still holds the top-n
+  const uint32_t first = min(H->list_count, static_cast<uint32_t>(kListCap));
   Plan p{};
-  if (total <= static_cast<uint32_t>(kListCap)) {
+  if (total <= static_cast<uint32_t>(kListCap) - first) {
     p.op = OP_EXACT;
     p.lo = static_cast<uint32_t>(jlo);
     p.hi = static_cast<uint32_t>(jhi);
@@ -1926,9 +1999,10 @@ __device__ Plan window_plan(const Ctx& cx, LeaderState& L) {
     __syncthreads();
     if (threadIdx.x == 0) {
       L.phase = PH_AFTER_EXACT;
-      H->list_count = 0;
+      L.topn_count = static_cast<int>(first);
     }
   } else {
+    list_topn(cx, L, static_cast<int>(first));  // before the list area is reused
     p = mass_plan(L.m, -INFINITY, L.kminf, L.T);
     p.part_is_x = 1;
     __syncthreads();
@@ -1968,7 +2042,10 @@ __device__ void finish_draw(const Ctx& cx, LeaderState& L, double sd, int32_t id
 // window's kept entries to the CTAs' bests.
 __device__ void exact_tail(const Ctx& cx, LeaderState& L) {
   SharedHeader* H = cx.H;
-  const int count = min(static_cast<int>(H->list_count), kListCap);
+  const int first = L.topn_count;  // the first-pass list [0, first), then the window
+  const int count = min(static_cast<int>(H->list_count), kListCap) - first;
+  Ctx win = cx;
+  win.list = cx.list + first;
   double A = 0.0, B = 0.0;
   for (uint32_t r = 0; r < cx.C; ++r) {
     A += H->ex_above[r];
@@ -1976,41 +2053,40 @@ __device__ void exact_tail(const Ctx& cx, LeaderState& L) {
   }
   float theta_p = INFINITY;  // no window entry is kept unless the cut is found in it
   if (count > 0) {
-    const int np2 = pow2_ceil(count);
-    for (int j = count + threadIdx.x; j < np2; j += kThreads) cx.list[j] = ~0ull;
-    __syncthreads();
-    bitonic_sort(cx.list, np2);
+    uint64_t* buf = reinterpret_cast<uint64_t*>(cx.scratch);  // the window sorted by (x desc, id asc)
+    sort_entries(win.list, count, buf);
     const double m = static_cast<double>(L.m);
-    const int cs = (np2 + kThreads - 1) / kThreads;
+    const int cs = (count + kThreads - 1) / kThreads;
     const int i0 = min(static_cast<int>(threadIdx.x) * cs, count), i1 = min(i0 + cs, count);
     double sum = 0.0;
-    for (int i = i0; i < i1; ++i) sum += exp_neg64(static_cast<double>(key_value(entry_key(cx.list[i]))) - m, H->exp_tab);
+    for (int i = i0; i < i1; ++i) sum += exp_neg64(static_cast<double>(key_value(entry_key(buf[i]))) - m, H->exp_tab);
     double W;
     const double incl = block_scan_d(sum, &W, H);
     const double pz = static_cast<double>(L.top_p) * (A + W + B);
     double run = A + (incl - sum);
     int cand = -1;
     for (int i = i0; i < i1; ++i) {
-      const uint32_t k = entry_key(cx.list[i]);
-      const bool start = i == 0 || entry_key(cx.list[i - 1]) != k;
+      const uint32_t k = entry_key(buf[i]);
+      const bool start = i == 0 || entry_key(buf[i - 1]) != k;
       if (start && run < pz) cand = i;
       run += exp_neg64(static_cast<double>(key_value(k)) - m, H->exp_tab);
     }
     const int best = block_max_i(cand, H);
-    if (best >= 0) theta_p = key_value(entry_key(cx.list[best]));
+    if (best >= 0) theta_p = key_value(entry_key(buf[best]));
   }
   double sd;
   int32_t id;
   float l;
-  list_best(cx, L, count, true, theta_p, sd, id, l);
+  list_best(win, L, count, true, theta_p, sd, id, l);
   finish_draw(cx, L, sd, id);
+  list_topn(cx, L, first);
 }
 
 // Leader: merges the statistics every CTA pushed, validates data and parameters,
 // and fills the row state.  A flagged row gets its outputs here; returns true
 // for it.  When the first pass's list is complete (`listed`), the top-n is
 // written from it now.
-__device__ bool leader_merge(const Ctx& cx, LeaderState& L) {
+__device__ bool leader_merge(const Ctx& cx, LeaderState& L, bool topn_now = true) {
   const SampleArgs& a = *cx.a;
       if (threadIdx.x == 0) {
         uint32_t kmax = 0, kminf = 0xFFFFFFFFu, bad = 0;
@@ -2073,7 +2149,7 @@ __device__ bool leader_merge(const Ctx& cx, LeaderState& L) {
         }
         return true;
       }
-  if (cx.H->listed) {
+  if (cx.H->listed && topn_now) {
     // the first pass's union of per-CTA candidates holds the exact top-n
     const int count = min(static_cast<int>(cx.H->list_count), kListCap);
     list_topn(cx, L, count);
@@ -2378,8 +2454,8 @@ __global__ void __launch_bounds__(kThreads, 2) sample_kernel(const __grid_consta
   cx.C = static_cast<uint32_t>(a.C);
   cx.rank = cluster_ctarank();
   cx.row = static_cast<int>(blockIdx.x / a.C);
-  // rows the streaming kernel resolved (it runs first on the same stream) are done
-  if (a.token_ids[cx.row] != kDeferred) return;
+  // rows the streaming kernel takes (alongside), or resolved (before), are not this kernel's
+  if (a.select == kSelectOthers ? stream_row(a.params[cx.row], a.V) : a.token_ids[cx.row] != kDeferred) return;
   cx.g0 = static_cast<long long>(cx.rank) * a.part;
   const long long g1 = min(cx.g0 + a.part, static_cast<long long>(a.V));
   const int n = g1 > cx.g0 ? static_cast<int>(g1 - cx.g0) : 0;
@@ -2498,7 +2574,8 @@ __global__ void __launch_bounds__(kThreads, 2) sample_kernel(const __grid_consta
       }
       if (cx.rank == 0) {
         LeaderState& L = H->L;
-        leader_merge(cx, L);  // writes the top-n from the first-pass list
+        // the top-n from the first-pass list: now, or (XHIST path) at the end, off the critical path
+        leader_merge(cx, L, p.op != OP_XHIST);
         if (threadIdx.x == 0) {
           L.phase = p.op == OP_XHIST ? PH_AFTER_XHIST : PH_AFTER_GUMBEL;
           L.part_is_x = p.op == OP_XHIST ? 1 : 0;
@@ -2674,15 +2751,50 @@ cudaError_t launch_sample(const float* const* logits, int R, int S, int V_s, con
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   }
-  // 1) rows resolved from streamed candidates; the rest are marked kDeferred
   SampleArgs sa = a;
   stream_geometry(R, a.V, sms, &sa.C, &sa.part);
-  e = launch_with_cluster(reinterpret_cast<const void*>(stream_kernel), sa, R * sa.C, stream_smem_bytes(), stream);
-  if (e != cudaSuccess) return e;
-  // 2) the deferred rows, with the row held in the cluster's shared memory
   a.C = c;
   a.part = part;
-  return launch_with_cluster(reinterpret_cast<const void*>(sample_kernel), a, R * c, sample_smem_bytes(part), stream);
+  const void* fs = reinterpret_cast<const void*>(stream_kernel);
+  const void* fc = reinterpret_cast<const void*>(sample_kernel);
+  if (static_cast<long long>(R) * c > 4LL * sms) {
+    // a large batch: the streaming kernel first (it marks the rows it leaves),
+    // then the cluster kernel on the marked rows
+    sa.select = kStreamMarks;
+    a.select = kSelectDeferred;
+    if ((e = launch_with_cluster(fs, sa, R * sa.C, stream_smem_bytes(), stream)) != cudaSuccess) return e;
+    return launch_with_cluster(fc, a, R * c, sample_smem_bytes(part), stream);
+  }
+  // a small batch is latency-bound: the two kernels take disjoint rows (decided
+  // by the parameters alone) and run side by side, the cluster kernel on a side
+  // stream forked from and joined back to the caller's; then the cluster kernel
+  // samples the rows the streaming kernel could not hold (marked kDeferred)
+  struct Side {
+    cudaStream_t s = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+  };
+  static std::mutex mu;
+  static Side sides[64];
+  int dev = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  Side& sd = sides[dev];
+  if (sd.s == nullptr) {
+    if ((e = cudaStreamCreateWithFlags(&sd.s, cudaStreamNonBlocking)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&sd.fork, cudaEventDisableTiming)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&sd.join, cudaEventDisableTiming)) != cudaSuccess) return e;
+  }
+  sa.select = 0;  // the streaming kernel leaves the other rows untouched
+  a.select = kSelectOthers;
+  if ((e = cudaEventRecord(sd.fork, stream)) != cudaSuccess) return e;
+  if ((e = cudaStreamWaitEvent(sd.s, sd.fork, 0)) != cudaSuccess) return e;
+  if ((e = launch_with_cluster(fc, a, R * c, sample_smem_bytes(part), sd.s)) != cudaSuccess) return e;
+  if ((e = launch_with_cluster(fs, sa, R * sa.C, stream_smem_bytes(), stream)) != cudaSuccess) return e;
+  if ((e = cudaEventRecord(sd.join, sd.s)) != cudaSuccess) return e;
+  if ((e = cudaStreamWaitEvent(stream, sd.join, 0)) != cudaSuccess) return e;
+  a.select = kSelectDeferred;
+  return launch_with_cluster(fc, a, R * c, sample_smem_bytes(part), stream);
 }
 
 }  // namespace vsl

@@ -18,21 +18,12 @@
 namespace vsl {
 
 constexpr int kStreamCap = 4096;      // candidate list capacity while streaming
-constexpr int kStreamMaxK = 1024;     // largest top-k resolved from streamed candidates
 
 constexpr size_t kStreamListBytes = static_cast<size_t>(kStreamCap) * 8;
 constexpr size_t kStreamRingBytes = static_cast<size_t>(kStreamStages) * kStreamChunk * 4;
 
 __host__ __device__ __forceinline__ size_t stream_smem_bytes() {
   return ((sizeof(SharedHeader) + 127) & ~size_t(127)) + kScratchBytes + kStreamListBytes + kStreamRingBytes;
-}
-
-// Rows this kernel resolves: valid parameters, and greedy or a top-k the list holds.
-__device__ __forceinline__ bool stream_row(const vsl_row_params& p, int V) {
-  if (!(p.top_p > 0.0f) || p.top_k < 0) return false;
-  if (p.temperature == 0.0f) return true;
-  return p.temperature > 0.0f && p.temperature < INFINITY && p.top_k > 0 && p.top_k < V &&
-         p.top_k <= kStreamMaxK;
 }
 
 // Lowest raw key a compaction may keep when the rank-`r` value found is `v`:
@@ -209,7 +200,7 @@ __global__ void __launch_bounds__(kThreads, 2) stream_kernel(const __grid_consta
   cx.row = static_cast<int>(blockIdx.x / a.C);
   const vsl_row_params prm = a.params[cx.row];
   if (!stream_row(prm, a.V)) {
-    if (cx.rank == 0 && threadIdx.x == 0) a.token_ids[cx.row] = kDeferred;
+    if (a.select == kStreamMarks && cx.rank == 0 && threadIdx.x == 0) a.token_ids[cx.row] = kDeferred;
     return;  // the whole cluster leaves: the row is the cluster kernel's
   }
   cx.T = prm.temperature;
