@@ -188,6 +188,11 @@ struct __align__(16) SharedHeader {
   BestSlot best[kMaxCluster];
   double ex_above[kMaxCluster];    // leader only: EXACT sums pushed by every CTA
   double ex_below[kMaxCluster];
+  double win_lo[kMaxCluster];      // every CTA: each slice's lower / upper mass bound
+  double win_hi[kMaxCluster];
+  int32_t win_jlo[kMaxCluster];    // every CTA: each slice's window edges and count
+  int32_t win_jhi[kMaxCluster];
+  uint32_t win_cnt[kMaxCluster];
   uint32_t need_all[kMaxCluster];  // every CTA: each CTA's first-pass candidate count
   uint32_t ok_all[kMaxCluster];    // every CTA: each CTA's list is usable for top-k
   uint32_t listed;                 // the first-pass list holds the top-n (and top-k) union
@@ -2012,6 +2017,111 @@ __device__ Plan window_plan(const Ctx& cx, LeaderState& L) {
   return p;
 }
 
+// The top-p window computed by the whole cluster right after XHIST (each CTA
+// holds the cluster totals of its slice of the fine bins): every CTA bounds
+// its own bins, the slices' mass bounds are exchanged (prefix offsets and Z in
+// rank order, the same in every CTA), then each slice's window edges and
+// count.  Returns false when the window does not fit the list (the leader
+// then plans the fixed-point fallback); else `e` is the EXACT plan.
+__device__ bool window_distributed(const Ctx& cx, const Plan& px, Plan& e) {
+  SharedHeader* H = cx.H;
+  const uint32_t* cnt = reinterpret_cast<const uint32_t*>(cx.scratch);
+  const uint32_t* qs = cnt + kXBins;
+  const int S = kXBins / static_cast<int>(cx.C);
+  const int q = max(1, S / kThreads);
+  const int t = static_cast<int>(threadIdx.x);
+  const bool act = t * q < S;
+  const int b0 = static_cast<int>(cx.rank) * S + t * q;
+  const double w = 1.0 / static_cast<double>(px.step);
+  constexpr double eps = 0x1p-22;
+  constexpr int kMaxQ = kXBins / kThreads;
+  uint32_t c[kMaxQ];
+  double blo[kMaxQ], bhi[kMaxQ];
+  double slo = 0.0, shi = 0.0;
+#pragma unroll
+  for (int k = 0; k < kMaxQ; ++k) {
+    c[k] = 0;
+    blo[k] = bhi[k] = 0.0;
+    if (k < q && act) {
+      const int j = b0 + k;
+      c[k] = cnt[j];
+      const double ga = exp_neg64(-fmax(0.0, (j - 0.5) * (1.0 - eps)) * w, H->exp_tab);
+      const double gb = exp_neg64(-(j + 0.5) * (1.0 + eps) * w, H->exp_tab);
+      bin_bounds(j, c[k], qs[j], w, ga, gb, H->exp_tab, blo[k], bhi[k]);
+      slo += blo[k];
+      shi += bhi[k];
+    }
+  }
+  double tlo, thi;
+  const double ilo = block_scan_d(slo, &tlo, H) - slo;
+  const double ihi = block_scan_d(shi, &thi, H) - shi;
+  if (threadIdx.x < cx.C) {
+    cluster_ptr(H->win_lo, threadIdx.x)[cx.rank] = tlo;
+    cluster_ptr(H->win_hi, threadIdx.x)[cx.rank] = thi;
+  }
+  __syncthreads();
+  cluster_sync();
+  double zlo = 0.0, zhi = 0.0, olo = 0.0, ohi = 0.0;
+  for (uint32_t r = 0; r < cx.C; ++r) {
+    if (r < cx.rank) {
+      olo += H->win_lo[r];
+      ohi += H->win_hi[r];
+    }
+    zlo += H->win_lo[r];
+    zhi += H->win_hi[r];
+  }
+  const double tp = static_cast<double>(cx.top_p);
+  const double keep_lim = tp * zlo * (1.0 - 1e-11);
+  const double drop_lim = tp * zhi * (1.0 + 1e-11);
+  int jlo = kXBins, jhi = -1;
+  uint32_t nwin = 0;
+  double plo = olo + ilo, phi = ohi + ihi;
+#pragma unroll
+  for (int k = 0; k < kMaxQ; ++k) {
+    if (k < q && act && c[k] > 0) {
+      const int j = b0 + k;
+      const double nphi = phi + bhi[k];
+      const bool keep = nphi * (1.0 + 1e-11) < keep_lim;  // kept for certain
+      const bool drop = plo * (1.0 - 1e-11) >= drop_lim;  // dropped for certain
+      if (!keep) jlo = min(jlo, j);
+      if (!drop) jhi = max(jhi, j);
+      if (!keep && !drop) nwin += c[k];
+    }
+    plo += blo[k];
+    phi += bhi[k];
+  }
+  jlo = block_min_i(jlo, H);
+  jhi = block_max_i(jhi, H);
+  uint32_t nt;
+  block_scan_u(nwin, &nt, H);
+  if (threadIdx.x < cx.C) {
+    cluster_ptr(H->win_jlo, threadIdx.x)[cx.rank] = jlo;
+    cluster_ptr(H->win_jhi, threadIdx.x)[cx.rank] = jhi;
+    cluster_ptr(H->win_cnt, threadIdx.x)[cx.rank] = nt;
+  }
+  __syncthreads();
+  cluster_sync();
+  int glo = kXBins, ghi = -1;
+  uint32_t gn = 0;
+  for (uint32_t r = 0; r < cx.C; ++r) {
+    glo = min(glo, H->win_jlo[r]);
+    ghi = max(ghi, H->win_jhi[r]);
+    gn += H->win_cnt[r];
+  }
+  const uint32_t first = min(*cluster_ptr(&H->list_count, 0), static_cast<uint32_t>(kListCap));
+  if (gn > static_cast<uint32_t>(kListCap) - first) return false;
+  e = Plan{};
+  e.op = OP_EXACT;
+  e.lo = static_cast<uint32_t>(glo);
+  e.hi = static_cast<uint32_t>(ghi);
+  e.m = px.m;
+  e.step = px.step;
+  e.theta = -INFINITY;
+  e.part_is_x = 1;
+  e.last = 1;
+  return true;
+}
+
 // The row's token from the leader's best (sd, id) and every CTA's pushed best;
 // its raw logit is read back from the slices.
 __device__ void finish_draw(const Ctx& cx, LeaderState& L, double sd, int32_t id) {
@@ -2586,6 +2696,22 @@ __global__ void __launch_bounds__(kThreads, 2) sample_kernel(const __grid_consta
       else op_gumbel(cx, p);
       __syncthreads();
       cluster_sync();
+      Plan ex;
+      if (p.op == OP_XHIST && window_distributed(cx, p, ex)) {
+        // every CTA knows the window: EXACT without a plan round
+        if (cx.rank == 0 && threadIdx.x == 0) {
+          H->L.phase = PH_AFTER_EXACT;
+          H->L.topn_count = static_cast<int>(min(H->list_count, static_cast<uint32_t>(kListCap)));
+        }
+        op_exact(cx, ex);
+        __syncthreads();
+        cluster_sync();
+        if (cx.rank == 0) {
+          leader_step(cx, tail);
+          leader_tail(cx, tail);
+        }
+        return;
+      }
       if (p.op == OP_GUMBEL) {
         // what remains is the leader's alone: the CTAs' bests are in its slots
         if (cx.rank == 0) {
