@@ -380,7 +380,7 @@ def run_gpu(args, w):
             "sampler_hbm_gbs_in_step": samp_bytes / (samp_ms / 1e3) / 1e9,
         },
         "e2e": {"value": e2e_value, "unit": "rows/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 3 * args.steps,  # logits_local_kernel, stream_kernel, sample_kernel
+        "gpu_launches": (1 + vsl.sample_launches(w.R, w.S, w.V_s)) * args.steps,  # projection + sampler kernels
         "clocks": clk,
         "cpu_baseline": None,
     }

@@ -83,3 +83,12 @@ def test_binding_has_no_cpu_fallback(monkeypatch, tmp_path):
     mod = importlib.util.module_from_spec(spec)
     with pytest.raises(ImportError):
         spec.loader.exec_module(mod)
+
+
+def test_sample_launches_rejects_bad_sizes_on_the_host():
+    import vocab_sharded_logits_b200 as v
+    lib = v.lib
+    assert lib.vsl_sample_launches(0, 4, 37984) == -1
+    assert lib.vsl_sample_launches(64, 0, 37984) == -1
+    assert lib.vsl_sample_launches(64, 17, 37984) == -1
+    assert lib.vsl_sample_launches(64, 4, 37983) == -1

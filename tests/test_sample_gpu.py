@@ -200,3 +200,11 @@ def test_streaming_tie_flood_defers(cuda_device):
     params = (T, k, p, np.arange(R), np.arange(R))
     gpu = run_sampler(torch.from_numpy(logits), params, 5, 20, S, cuda_device)
     compare(gpu, logits, params, 5, 20, range(R))
+
+
+def test_sample_launch_count(cuda_device):
+    """Small batches run the sampler's kernels side by side (3 launches), large ones in
+    order (2): the decode and speculative-verify sizes on a 148-SM part."""
+    sms = torch.cuda.get_device_properties(cuda_device).multi_processor_count
+    assert vsl.sample_launches(64, 4, 37984) == (3 if 64 * 8 <= 4 * sms else 2)
+    assert vsl.sample_launches(512, 4, 37984) == 2

@@ -11,7 +11,7 @@ import os
 import torch
 
 __all__ = [
-    "logits_local", "sample", "make_row_params", "SampleResult", "lib", "status_string",
+    "logits_local", "sample", "sample_launches", "make_row_params", "SampleResult", "lib", "status_string",
     "device_error", "VslError", "ROW_NONFINITE", "ROW_ALL_NEG_INF", "ROW_BAD_TEMPERATURE",
     "ROW_BAD_TOP_P", "ROW_BAD_TOP_K", "ROW_SCALE_OVERFLOW", "MAX_SLICES", "MAX_LOGPROBS",
 ]
@@ -47,6 +47,8 @@ def _load():
     l.vsl_logits_local.argtypes = [vp, ctypes.POINTER(vp), ctypes.POINTER(vp), i32, i32, i32, i32, vp]
     l.vsl_sample_workspace_bytes.restype = sz
     l.vsl_sample_workspace_bytes.argtypes = [i32, i32, i32, i32]
+    l.vsl_sample_launches.restype = i32
+    l.vsl_sample_launches.argtypes = [i32, i32, i32]
     l.vsl_sample.restype = ctypes.c_int
     l.vsl_sample.argtypes = [ctypes.POINTER(vp), i32, i32, i32, vp, u64, i32, vp, vp, vp, vp, vp, vp, sz, vp]
     l.vsl_device_error.restype = ctypes.c_int
@@ -171,6 +173,14 @@ def sample(logits_slices, params, seed, n_logprobs, out=None, stream=None):
                             _ptr(topn_lp), _ptr(out.row_flags), _ptr(ws), ws_bytes, _stream_handle(stream, dev))
     _check(status, "vsl_sample")
     return out
+
+
+def sample_launches(R, S, V_s):
+    """Kernels one ``sample`` call with these sizes launches on the current device."""
+    n = lib.vsl_sample_launches(int(R), int(S), int(V_s))
+    if n < 0:
+        raise VslError(f"vsl_sample_launches: sizes rejected (R={R}, S={S}, V_s={V_s})")
+    return n
 
 
 def device_error():

@@ -64,6 +64,11 @@ size_t vsl_sample_workspace_bytes(int32_t R, int32_t S, int32_t V_s, int32_t n_l
   return 0;  // every intermediate lives in shared memory
 }
 
+int32_t vsl_sample_launches(int32_t R, int32_t S, int32_t V_s) {
+  if (R <= 0 || S <= 0 || S > VSL_MAX_SLICES || V_s <= 0 || V_s % 4 != 0) return -1;
+  return vsl::sample_launches(R, static_cast<long long>(S) * V_s);
+}
+
 vsl_status vsl_sample(const float* const* logits_slices, int32_t R, int32_t S, int32_t V_s,
                       const vsl_row_params* params_dev, uint64_t seed, int32_t n_logprobs, int32_t* token_ids,
                       float* token_logprob, int32_t* topn_ids, float* topn_logprob, uint32_t* row_flags,

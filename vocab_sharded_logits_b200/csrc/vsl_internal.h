@@ -26,5 +26,6 @@ cudaError_t launch_sample(const float* const* logits, int R, int S, int V_s,
 // Sampler launch geometry for a vocabulary of V tokens: CTAs per row (cluster
 // size) and elements per CTA.  Returns false if V cannot be handled.
 bool sample_geometry(long long V, int* cluster, int* part);
+int sample_launches(int R, long long V);
 
 }  // namespace vsl

@@ -65,7 +65,7 @@ constexpr int kStreamMaxK = 1024;      // largest top-k resolved from streamed c
 // alongside it).  stream_kernel: kStreamMarks makes it mark those rows kDeferred.
 constexpr int kSelectDeferred = 0, kSelectOthers = 1, kStreamMarks = 1;
 constexpr int kStreamChunk = 2048;     // streaming kernel: floats per ring stage (8 KB)
-constexpr int kStreamStages = 6;       // streaming kernel: ring depth (40 KB in flight per CTA)
+constexpr int kStreamStages = 8;       // streaming kernel: ring depth (56 KB in flight per CTA)
 constexpr int kXBins = 2048;           // fine bins of x below m (top-p window search)
 constexpr float kXQuant = 4096.0f;     // in-bin offset quantum: 1 / 4096 of a bin
 constexpr float kXRange = 40.0f;       // x more than 40 below m (mass < 5e-18 each) share the last bin
@@ -2848,6 +2848,30 @@ static cudaError_t launch_with_cluster(const void* fn, const SampleArgs& a, int 
   return cudaLaunchKernelExC(&cfg, fn, args);
 }
 
+// A batch whose cluster kernel grid covers at most 4 CTAs per SM is latency
+// bound: the sampler's kernels then run side by side (three launches).
+static bool small_batch(int R, int cluster, int sms) {
+  return static_cast<long long>(R) * cluster <= 4LL * sms;
+}
+
+static int device_sms() {
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  }
+  return sms;
+}
+
+int sample_launches(int R, long long V) {
+  int c = 0, part = 0;
+  if (prepare_sample_kernel() != cudaSuccess || !sample_geometry(V, &c, &part)) return -1;
+  const int sms = device_sms();
+  if (sms <= 0) return -1;
+  return small_batch(R, c, sms) ? 3 : 2;
+}
+
 cudaError_t launch_sample(const float* const* logits, int R, int S, int V_s, const vsl_row_params* params,
                           uint64_t seed, int n_logprobs, int32_t* token_ids, float* token_logprob,
                           int32_t* topn_ids, float* topn_logprob, uint32_t* row_flags, cudaStream_t stream) {
@@ -2871,19 +2895,15 @@ cudaError_t launch_sample(const float* const* logits, int R, int S, int V_s, con
   a.n_logprobs = n_logprobs;
   int c = 0, part = 0;
   if (!sample_geometry(a.V, &c, &part)) return cudaErrorInvalidValue;
-  static int sms = 0;
-  if (sms == 0) {
-    int dev = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-  }
+  const int sms = device_sms();
+  if (sms <= 0) return cudaErrorInvalidDevice;
   SampleArgs sa = a;
   stream_geometry(R, a.V, sms, &sa.C, &sa.part);
   a.C = c;
   a.part = part;
   const void* fs = reinterpret_cast<const void*>(stream_kernel);
   const void* fc = reinterpret_cast<const void*>(sample_kernel);
-  if (static_cast<long long>(R) * c > 4LL * sms) {
+  if (!small_batch(R, c, sms)) {
     // a large batch: the streaming kernel first (it marks the rows it leaves),
     // then the cluster kernel on the marked rows
     sa.select = kStreamMarks;

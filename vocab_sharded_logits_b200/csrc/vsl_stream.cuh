@@ -22,8 +22,13 @@ constexpr int kStreamCap = 4096;      // candidate list capacity while streaming
 constexpr size_t kStreamListBytes = static_cast<size_t>(kStreamCap) * 8;
 constexpr size_t kStreamRingBytes = static_cast<size_t>(kStreamStages) * kStreamChunk * 4;
 
+// Layout: header | 1 KB of narrowing bins | list | ring.  After the stream the
+// ring's first kScratchBytes serve as the leader's scratch (every copy into
+// the ring has landed by then).
+constexpr size_t kStreamBinsBytes = 1024;
+static_assert(kStreamRingBytes >= kScratchBytes, "the ring doubles as the leader's scratch");
 __host__ __device__ __forceinline__ size_t stream_smem_bytes() {
-  return ((sizeof(SharedHeader) + 127) & ~size_t(127)) + kScratchBytes + kStreamListBytes + kStreamRingBytes;
+  return ((sizeof(SharedHeader) + 127) & ~size_t(127)) + kStreamBinsBytes + kStreamListBytes + kStreamRingBytes;
 }
 
 // Lowest raw key a compaction may keep when the rank-`r` value found is `v`:
@@ -186,14 +191,14 @@ __device__ __forceinline__ void stream_scan(const float4* st4, int nq, uint32_t 
 __global__ void __launch_bounds__(kThreads, 2) stream_kernel(const __grid_constant__ SampleArgs a) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   SharedHeader* H = reinterpret_cast<SharedHeader*>(smem_raw);
-  uint8_t* scratch = smem_raw + ((sizeof(SharedHeader) + 127) & ~size_t(127));
-  uint64_t* list = reinterpret_cast<uint64_t*>(scratch + kScratchBytes);
+  uint8_t* bins = smem_raw + ((sizeof(SharedHeader) + 127) & ~size_t(127));
+  uint64_t* list = reinterpret_cast<uint64_t*>(bins + kStreamBinsBytes);
   float* ring = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(list) + kStreamListBytes);
 
   Ctx cx;
   cx.a = &a;
   cx.H = H;
-  cx.scratch = scratch;
+  cx.scratch = bins;  // the compactions' 256 narrowing bins while streaming
   cx.list = list;
   cx.C = static_cast<uint32_t>(a.C);
   cx.rank = cluster_ctarank();
@@ -315,6 +320,7 @@ __global__ void __launch_bounds__(kThreads, 2) stream_kernel(const __grid_consta
   own = dropped ? 0u : min(own, static_cast<uint32_t>(kStreamCap));
   const uint32_t overflow = dropped ? 1u : 0u;
 
+  cx.scratch = reinterpret_cast<uint8_t*>(ring);  // the stream is over: the ring is scratch
   // ---- merge into the leader: statistics, thresholds, candidates
   if (cx.C > 1) cluster_sync();
   if (cx.rank != 0) {
