@@ -174,17 +174,19 @@ def test_draw_frequencies_chi_square(cuda_device):
 def test_streaming_geometries(cuda_device, R):
     """The streaming kernel's CTAs per row (8, 4, 2, 1 for these batch sizes on a
     148-SM part) and the cluster kernel's rows in one batch: greedy, small and
-    large top-k (several compactions) and top-k off, sampled rows vs the oracle."""
+    large top-k (several compactions), top-k off with and without top-p (taken
+    by the streaming kernel's three-pass path at one CTA per row, R = 300),
+    sampled rows vs the oracle."""
     V, S = 151936, 4
     rng = np.random.default_rng(R)
     logits = torch.from_numpy((rng.standard_normal((R, V)) * 1.3).astype(np.float32))
-    kinds = np.arange(R) % 4
-    T = np.where(kinds == 0, 0.0, rng.uniform(0.5, 1.5, R)).astype(np.float32)
-    k = np.choose(kinds, [0, 20, 900, 0]).astype(np.int32)
-    p = np.where(kinds == 3, 0.9, rng.uniform(0.8, 1.0, R)).astype(np.float32)
+    kinds = np.arange(R) % 5
+    T = np.where(kinds == 0, 0.0, rng.uniform(0.3, 1.5, R)).astype(np.float32)
+    k = np.choose(kinds, [0, 20, 900, 0, 0]).astype(np.int32)
+    p = np.choose(kinds, [1.0, 0.9, 0.95, 0.7, 1.0]).astype(np.float32)
     params = (T, k, p, np.arange(R), np.arange(R) * 7 + 3)
     gpu = run_sampler(logits, params, 99, 20, S, cuda_device)
-    rows = sorted(set(np.random.default_rng(1).choice(R, min(R, 12), replace=False).tolist()) | {0, 1, 2, 3})
+    rows = sorted(set(np.random.default_rng(1).choice(R, min(R, 12), replace=False).tolist()) | {0, 1, 2, 3, 4})
     compare(gpu, logits.numpy(), params, 99, 20, rows)
 
 

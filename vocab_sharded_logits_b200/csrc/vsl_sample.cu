@@ -62,8 +62,9 @@ constexpr int32_t kDeferred = -2;      // token id of a row the streaming kernel
 constexpr int kStreamMaxK = 1024;      // largest top-k resolved from streamed candidates
 // sample_kernel row selection: rows whose token id reads kDeferred (after the
 // streaming kernel), or every row the streaming kernel does not take (run
-// alongside it).  stream_kernel: kStreamMarks makes it mark those rows kDeferred.
-constexpr int kSelectDeferred = 0, kSelectOthers = 1, kStreamMarks = 1;
+// alongside it).  stream_kernel: kStreamMarks makes it mark those rows
+// kDeferred; kStreamKoff makes it also take top-k-off rows (one CTA per row).
+constexpr int kSelectDeferred = 0, kSelectOthers = 1, kStreamMarks = 1, kStreamKoff = 2;
 constexpr int kStreamChunk = 2048;     // streaming kernel: floats per ring stage (8 KB)
 constexpr int kStreamStages = 8;       // streaming kernel: ring depth (56 KB in flight per CTA)
 constexpr int kXBins = 2048;           // fine bins of x below m (top-p window search)
@@ -217,12 +218,13 @@ constexpr size_t kListBytes = kListCap * 8;
 
 // ------------------------------------------------------------------ small helpers
 // Rows the streaming kernel resolves: valid parameters, and greedy or a top-k
-// its candidate list holds.
-__device__ __forceinline__ bool stream_row(const vsl_row_params& p, int V) {
+// its candidate list holds, or (koff) top-k off.
+__device__ __forceinline__ bool stream_row(const vsl_row_params& p, int V, bool koff = false) {
   if (!(p.top_p > 0.0f) || p.top_k < 0) return false;
   if (p.temperature == 0.0f) return true;
-  return p.temperature > 0.0f && p.temperature < INFINITY && p.top_k > 0 && p.top_k < V &&
-         p.top_k <= kStreamMaxK;
+  if (!(p.temperature > 0.0f && p.temperature < INFINITY)) return false;
+  if (p.top_k > 0 && p.top_k < V) return p.top_k <= kStreamMaxK;
+  return koff;
 }
 
 // Order-preserving key of a float, computed on its bits with integer operations
@@ -2906,7 +2908,7 @@ cudaError_t launch_sample(const float* const* logits, int R, int S, int V_s, con
   if (!small_batch(R, c, sms)) {
     // a large batch: the streaming kernel first (it marks the rows it leaves),
     // then the cluster kernel on the marked rows
-    sa.select = kStreamMarks;
+    sa.select = kStreamMarks | (sa.C == 1 ? kStreamKoff : 0);
     a.select = kSelectDeferred;
     if ((e = launch_with_cluster(fs, sa, R * sa.C, stream_smem_bytes(), stream)) != cudaSuccess) return e;
     return launch_with_cluster(fc, a, R * c, sample_smem_bytes(part), stream);

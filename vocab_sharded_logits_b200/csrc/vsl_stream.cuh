@@ -91,8 +91,9 @@ __device__ uint32_t stream_compact(const Ctx& cx, uint32_t r, uint32_t thr, int 
 // slice `s` holding the chunk's start only moves forward).  A chunk may span
 // two slices.
 __device__ __forceinline__ void stream_issue(const SampleArgs& a, int row, int g0, int n, int c, int& s,
-                                             float* ring, unsigned long long* bars, uint64_t pol) {
-  const int stage = c % kStreamStages;
+                                             float* ring, unsigned long long* bars, uint64_t pol,
+                                             int stage_base = 0) {
+  const int stage = (stage_base + c) % kStreamStages;
   const int e0 = g0 + c * kStreamChunk;
   const int e1 = g0 + min((c + 1) * kStreamChunk, n);
   const uint32_t bar = smem_u32(&bars[stage]);
@@ -187,6 +188,199 @@ __device__ __forceinline__ void stream_scan(const float4* st4, int nq, uint32_t 
     }
 }
 
+// One more streaming pass over this CTA's part [g0, g0 + n), continuing the
+// ring where the previous pass left it (`cg`: chunks streamed so far, which
+// fixes each stage's mbarrier phase).  `body(st4, nq, gid)` scans one stage
+// (nq float4 from global id gid); every thread calls it for every chunk, so
+// it may use warp- and block-collective operations.  Returns false if a load
+// did not land within the bounded wait.
+template <typename F>
+__device__ bool stream_pass(const SampleArgs& a, int row, int g0, int n, float* ring, unsigned long long* bars,
+                            int& cg, F&& body) {
+  const int nch = (n + kStreamChunk - 1) / kStreamChunk;
+  const uint64_t pol = policy_evict_first();
+  int s_issue = 0;
+  bool ok = true;
+  __syncthreads();  // every stage of the previous pass is consumed
+  if (threadIdx.x == 0)
+    for (int c = 0; c < min(nch, kStreamStages - 1); ++c)
+      stream_issue(a, row, g0, n, c, s_issue, ring, bars, pol, cg % kStreamStages);
+  for (int c = 0; c < nch; ++c) {
+    const int g = cg + c;
+    const int stage = g % kStreamStages;
+    if (threadIdx.x == 0 && c + kStreamStages - 1 < nch)
+      stream_issue(a, row, g0, n, c + kStreamStages - 1, s_issue, ring, bars, pol, cg % kStreamStages);
+    if (ok && !mbar_wait_bounded(smem_u32(&bars[stage]), static_cast<uint32_t>(g / kStreamStages) & 1u)) {
+      if (threadIdx.x == 0) atomicOr(a.err, kErrSampleLoad);
+      ok = false;
+    }
+    body(reinterpret_cast<const float4*>(ring + static_cast<size_t>(stage) * kStreamChunk),
+         min(kStreamChunk, n - c * kStreamChunk) >> 2, static_cast<uint32_t>(g0 + c * kStreamChunk));
+    __syncthreads();  // the stage is consumed
+  }
+  cg += nch;
+  return ok;
+}
+
+// A top-k-off row on one CTA (the whole row, top-n already written from
+// pass 1).  top_p < 1: pass 2 bins x = fl(l / T) on the fine bins (count and
+// offset sums in the list area's first half), the CTA finds the window, pass 3
+// sums the float64 masses above and below it, lists its members (the list
+// area's second half) and draws over the certainly kept tokens, then the
+// exact cut and the draw over the window's kept members.  top_p >= 1: one
+// draw pass over every finite token.  Fills L.token / L.token_l; returns false
+// when the window does not fit the list (the cluster kernel takes the row).
+__device__ bool stream_koff(const Ctx& cx, LeaderState& L, const SampleArgs& a, float* ring, int n, int& cg) {
+  SharedHeader* H = cx.H;
+  const int g0 = static_cast<int>(cx.g0);
+  const float T = L.T;
+  const int t = static_cast<int>(threadIdx.x);
+  const uint32_t k0 = static_cast<uint32_t>(a.seed), k1 = static_cast<uint32_t>(a.seed >> 32);
+  constexpr float kGMax = 16.7f;  // > -log(-log(1 - 2^-24)) = 16.63: the largest noise value
+  if (t == 0) H->gbound = kKeyNegInf;
+  if (!(L.top_p < 1.0f)) {
+    // pure sampling: argmax of x + g over every finite token
+    __syncthreads();
+    Best b;
+    b.init(&H->gbound);
+    const float invT = __frcp_rn(T);
+    const bool approx = invT < INFINITY;
+    stream_pass(a, cx.row, g0, n, ring, H->ring_bar, cg, [&](const float4* st4, int nq, uint32_t gid) {
+#pragma unroll
+      for (int it = 0; it < kStreamChunk / 4 / kThreads; ++it) {
+        const int q = t + it * kThreads;
+        if (q >= nq) continue;
+        const float4 v4 = st4[q];
+        const float v[4] = {v4.x, v4.y, v4.z, v4.w};
+        float xu[4];
+        bool any = false;
+        float xmax = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const bool fin = key_finite(fkey(v[i]));
+          const float xa = approx ? v[i] * invT : scale_x(v[i], T);
+          xu[i] = fin ? (approx ? xa + fabsf(xa) * 5e-7f + 1e-37f : xa) : -INFINITY;
+          any |= fin;
+          xmax = fmaxf(xmax, xu[i]);
+        }
+        if (!any) continue;
+        const float sb = b.bound_score();
+        if (sb > -INFINITY && xmax + kGMax < sb - score_tol(sb)) continue;
+        const uint32_t gq = gid + 4u * static_cast<uint32_t>(q);
+        const uint4 w = philox4x32_10(make_uint4(gq >> 2, cx.pos, cx.req, 0u), k0, k1);
+        const float bl = b.bound_l2e();
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          if (!(xu[i] > -INFINITY)) continue;
+          const uint32_t wi = word_of(w, i);
+          if (bl != Best::kNoBound && Best::rejects(bl, xu[i], wi)) continue;
+          b.offer_passed(scale_x(v[i], T), v[i], wi, static_cast<int32_t>(gq + i));
+        }
+      }
+    });
+    push_best(cx, b);
+    __syncthreads();
+    finish_draw(cx, L, -INFINITY, 0x7FFFFFFF);
+    return true;
+  }
+  // ---- pass 2: fine bins of x below m (the list area's first 16 KB)
+  uint32_t* cnt = reinterpret_cast<uint32_t*>(cx.list);
+  uint32_t* qs = cnt + kXBins;
+  for (int i = t; i < 2 * kXBins; i += kThreads) cnt[i] = 0;
+  const float m = L.m;
+  const float inv_w = xbin_scale(m, scale_x(key_value(L.kminf), T));
+  stream_pass(a, cx.row, g0, n, ring, H->ring_bar, cg, [&](const float4* st4, int nq, uint32_t) {
+#pragma unroll
+    for (int it = 0; it < kStreamChunk / 4 / kThreads; ++it) {
+      const int q = t + it * kThreads;
+      if (q >= nq) continue;
+      const float4 v4 = st4[q];
+      const float v[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (!key_finite(fkey(v[i]))) continue;
+        uint32_t qo;
+        const int j = xbin_q(scale_x(v[i], T), m, inv_w, qo);
+        atomicAdd(&cnt[j], 1u);
+        atomicAdd(&qs[j], qo);
+      }
+    }
+  });
+  // ---- the window (a cluster of one CTA)
+  Ctx wc = cx;
+  wc.scratch = reinterpret_cast<uint8_t*>(cnt);
+  wc.list = cx.list + kListCap;
+  if (t == 0) H->list_count = 0;
+  __syncthreads();
+  Plan px{};
+  px.m = m;
+  px.step = inv_w;
+  Plan e;
+  if (!window_distributed(wc, px, e)) return false;
+  // ---- pass 3: float64 masses above / below the window, its members, the draw above it
+  if (t == 0) H->gbound = kKeyNegInf;
+  __syncthreads();
+  Best b;
+  b.init(&H->gbound);
+  const double md = static_cast<double>(m);
+  const double* tab = H->exp_tab;
+  const int jlo = static_cast<int>(e.lo), jhi = static_cast<int>(e.hi);
+  double above = 0.0, below = 0.0;
+  stream_pass(a, cx.row, g0, n, ring, H->ring_bar, cg, [&](const float4* st4, int nq, uint32_t gid) {
+#pragma unroll
+    for (int it = 0; it < kStreamChunk / 4 / kThreads; ++it) {
+      const int q = t + it * kThreads;
+      const bool valid = q < nq;
+      const float4 v4 = valid ? st4[q] : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      const float l[4] = {v4.x, v4.y, v4.z, v4.w};
+      float v[4];
+      bool win[4], ab[4];
+      bool any_win = false, any_ab = false;
+      float xmax = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const bool fin = key_finite(fkey(l[i]));
+        v[i] = fin ? scale_x(l[i], T) : -INFINITY;
+        const int j = fin ? xbin(v[i], m, inv_w) : kXBins;
+        win[i] = fin && j >= jlo && j <= jhi;
+        ab[i] = fin && j < jlo;
+        const double ev = exp_neg64(static_cast<double>(v[i]) - md, tab);
+        above += ab[i] ? ev : 0.0;
+        below += (fin && !ab[i] && !win[i]) ? ev : 0.0;
+        any_win |= win[i];
+        any_ab |= ab[i];
+        if (ab[i]) xmax = fmaxf(xmax, v[i]);
+      }
+      const uint32_t gq = gid + 4u * static_cast<uint32_t>(q);
+      if (__any_sync(0xFFFFFFFFu, any_win)) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          local_append(&H->list_count, wc.list, win[i], (static_cast<uint64_t>(~fkey(v[i])) << 32) | (gq + i));
+      }
+      if (!any_ab) continue;
+      const float sb = b.bound_score();
+      if (sb > -INFINITY && xmax + kGMax < sb - score_tol(sb)) continue;
+      const uint4 w = philox4x32_10(make_uint4(gq >> 2, cx.pos, cx.req, 0u), k0, k1);
+      const float bl = b.bound_l2e();
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (ab[i] && (bl == Best::kNoBound || !Best::rejects(bl, v[i], word_of(w, i))))
+          b.offer_passed(v[i], 0.0f, word_of(w, i), static_cast<int32_t>(gq + i));
+    }
+  });
+  const double ta = block_sum_d0(above, H);
+  const double tb = block_sum_d0(below, H);
+  if (t == 0) {
+    H->ex_above[0] = ta;
+    H->ex_below[0] = tb;
+    L.topn_count = 0;  // the window list starts at wc.list[0]
+  }
+  push_best(wc, b);
+  __syncthreads();
+  exact_tail(wc, L);
+  return true;
+}
+
 // One CTA per (row, part) of a cluster of C CTAs per row; grid R * C.
 __global__ void __launch_bounds__(kThreads, 2) stream_kernel(const __grid_constant__ SampleArgs a) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -204,7 +398,8 @@ __global__ void __launch_bounds__(kThreads, 2) stream_kernel(const __grid_consta
   cx.rank = cluster_ctarank();
   cx.row = static_cast<int>(blockIdx.x / a.C);
   const vsl_row_params prm = a.params[cx.row];
-  if (!stream_row(prm, a.V)) {
+  const bool take_koff = (a.select & kStreamKoff) != 0 && a.C == 1;
+  if (!stream_row(prm, a.V, take_koff)) {
     if (a.select == kStreamMarks && cx.rank == 0 && threadIdx.x == 0) a.token_ids[cx.row] = kDeferred;
     return;  // the whole cluster leaves: the row is the cluster kernel's
   }
@@ -220,8 +415,9 @@ __global__ void __launch_bounds__(kThreads, 2) stream_kernel(const __grid_consta
   cx.part4 = nullptr;
   const int nch = (n + kStreamChunk - 1) / kStreamChunk;
   const bool greedy = prm.temperature == 0.0f;
+  const bool k_on = !greedy && prm.top_k > 0 && prm.top_k < a.V;
   uint32_t R = a.n_logprobs > 0 ? static_cast<uint32_t>(a.n_logprobs) : 1u;
-  if (!greedy) R = max(R, static_cast<uint32_t>(prm.top_k));
+  if (k_on) R = max(R, static_cast<uint32_t>(prm.top_k));
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStreamStages; ++s) mbar_init(smem_u32(&H->ring_bar[s]), 1);
@@ -272,6 +468,7 @@ __global__ void __launch_bounds__(kThreads, 2) stream_kernel(const __grid_consta
     }
   }
 
+  int cg = nch;  // chunks streamed so far (the ring's position)
   // ---- CTA statistics (the cluster kernel's CtaStats layout)
   // (m, s) pairs merge by rescaling to the larger m; kScanNoMax pairs add 0
 #pragma unroll
@@ -361,7 +558,17 @@ __global__ void __launch_bounds__(kThreads, 2) stream_kernel(const __grid_consta
   if (leader_merge(cx, L)) return;  // flagged row: outputs written
   uint64_t* buf = reinterpret_cast<uint64_t*>(cx.scratch);
   sort_entries(list, count, buf);
-  if (!greedy) {
+  if (!greedy && !k_on) {
+    // top-k off (one CTA holds the row): the top-n now, then the passes of stream_koff
+    list_resolve_sorted(cx, L, buf, count, false);
+    if (!stream_koff(cx, L, a, ring, n, cg)) {
+      if (threadIdx.x == 0) a.token_ids[cx.row] = kDeferred;
+      return;
+    }
+    write_outputs(cx, L);
+    return;
+  }
+  if (k_on) {
     // every value that can scale to theta_k must have been a candidate in every part
     const float theta_k = scale_x(key_value(entry_key(buf[min(L.r_k, count) - 1])), L.T);
     const uint32_t lo = raw_prefilter(theta_k, L.T);
