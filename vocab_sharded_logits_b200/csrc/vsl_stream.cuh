@@ -59,7 +59,26 @@ __device__ uint32_t stream_compact(const Ctx& cx, uint32_t r, uint32_t thr, int 
     const int idx = static_cast<int>(threadIdx.x) + i * kThreads;
     e[i] = idx < count ? cx.list[idx] : 0ull;
   }
-  uint32_t cut = stream_floor(list_rank_key(cx, count, r, rounds), cx.T);
+  uint32_t cut;
+  if (count <= 2 * kThreads) {
+    // a short list: the r-th largest key directly, every entry ranked against all (sort keys are distinct)
+    const int t = static_cast<int>(threadIdx.x);
+    const uint64_t e0 = t < count ? cx.list[t] : ~0ull, e1 = t + kThreads < count ? cx.list[t + kThreads] : ~0ull;
+    int r0 = 0, r1 = 0;
+#pragma unroll 8
+    for (int j = 0; j < count; ++j) {
+      const uint64_t y = cx.list[j];
+      r0 += y < e0 ? 1 : 0;
+      r1 += y < e1 ? 1 : 0;
+    }
+    if (t < count && r0 == static_cast<int>(r) - 1) H->L.found_cum = entry_key(e0);
+    if (t + kThreads < count && r1 == static_cast<int>(r) - 1) H->L.found_cum = entry_key(e1);
+    __syncthreads();
+    cut = stream_floor(H->L.found_cum, cx.T);
+    rounds = 64;  // exact
+  } else {
+    cut = stream_floor(list_rank_key(cx, count, r, rounds), cx.T);
+  }
   uint32_t kept = 0, total = 0;
   for (int pass = 0; pass < 2; ++pass) {
     kept = 0;
@@ -439,6 +458,11 @@ __global__ void __launch_bounds__(kThreads, 2) stream_kernel(const __grid_consta
   bool load_ok = true;
   bool dropped = false;  // some candidate was not listed: the row goes to the cluster kernel
   uint32_t seen = 0;     // this warp's list end after its appends of the current chunk
+  // compact when less than a chunk of room is left, and, once the threshold
+  // is set, whenever the list has grown past 4R + 64: the threshold then
+  // follows the R-th largest key seen so far and far fewer logits are listed
+  uint32_t grow_limit = static_cast<uint32_t>(kStreamCap - kStreamChunk);
+  const uint32_t small_limit = min(grow_limit, 4u * R + 64u);
   const int lane = threadIdx.x & 31;
   for (int c = 0; c < nch; ++c) {
     const int stage = c % kStreamStages;
@@ -456,7 +480,7 @@ __global__ void __launch_bounds__(kThreads, 2) stream_kernel(const __grid_consta
     else stream_scan<false>(st4, nq, thr, gid, st, seen, &H->list_count, list);
     // the stage is consumed and the appends are visible; the barrier also
     // tells every thread whether the list has less than a chunk of room left
-    const bool full = __syncthreads_or(seen > static_cast<uint32_t>(kStreamCap - kStreamChunk)) != 0;
+    const bool full = __syncthreads_or(seen > grow_limit) != 0;
     seen = 0;
     if (full && !dropped) {
       uint32_t left;
@@ -465,6 +489,7 @@ __global__ void __launch_bounds__(kThreads, 2) stream_kernel(const __grid_consta
       // no room for another chunk (ties at the threshold): the row is deferred, stop listing
       if (left > static_cast<uint32_t>(kStreamCap - kStreamChunk)) dropped = true;
       if (dropped) thr = 0xFFFFFFFFu;
+      grow_limit = min(static_cast<uint32_t>(kStreamCap - kStreamChunk), max(small_limit, left + 64u));
     }
   }
 
