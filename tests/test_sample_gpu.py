@@ -204,6 +204,30 @@ def test_streaming_tie_flood_defers(cuda_device):
     compare(gpu, logits, params, 5, 20, range(R))
 
 
+def test_deferred_rows_of_a_large_batch(cuda_device):
+    """A large batch whose every row floods the streaming kernel's list with ties:
+    the cluster kernel's deferred-row pass (a fixed number of clusters, each
+    taking every G-th row and, past 256 rows per cluster, a second block of
+    marks) samples them all."""
+    R, V, S = 9600, 90112, 4
+    g = torch.Generator(device=cuda_device)
+    g.manual_seed(17)
+    # integer logits: the top 1000 of a row reach into a tie of ~5,500 values at 2.0
+    logits = torch.round(torch.randn(R, V, generator=g, device=cuda_device))
+    T = np.full(R, 1.0, np.float32)
+    k = np.full(R, 1000, np.int32)
+    p = np.full(R, 0.99, np.float32)
+    params = (T, k, p, np.arange(R), np.arange(R))
+    gpu = run_sampler(logits, params, 9, 20, S, cuda_device)
+    assert np.all(gpu["flags"] == 0)
+    assert np.all((gpu["token"] >= 0) & (gpu["token"] < V))
+    sel = np.array([0, 1, 36, 37, 500, 4095, 9471, 9472, 9500, R - 1])
+    sub = {key: val[sel] for key, val in gpu.items()}
+    sub_params = tuple(np.asarray(x)[sel] for x in params)
+    del gpu
+    compare(sub, logits[torch.from_numpy(sel).to(cuda_device)].cpu().numpy(), sub_params, 9, 20, range(len(sel)))
+
+
 def test_sample_launch_count(cuda_device):
     """Small batches run the sampler's kernels side by side (3 launches), large ones in
     order (2): the decode and speculative-verify sizes on a 148-SM part."""

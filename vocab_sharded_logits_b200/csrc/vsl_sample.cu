@@ -37,6 +37,7 @@
 // re-compared in float64 whenever float32 cannot separate two candidates.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cfloat>
 #include <cmath>
 #include <cstdint>
@@ -211,6 +212,7 @@ struct __align__(16) SharedHeader {
   uint32_t scan_u[kWarps];
   unsigned long long scan_fx[kWarps][4];
   double exp_tab[256];
+  int32_t drows[kThreads];        // deferred-row pass: the rows of one block of marks
 };
 
 constexpr size_t kScratchBytes = kHistBins * 4;  // 16 KB: raw histogram, later mass / narrowing bins
@@ -745,14 +747,14 @@ __device__ __forceinline__ uint32_t* collect_counter(const Ctx& cx) {
 }
 
 // ---- pass 1: stats + raw-key histogram, chunk by chunk as the bulk copies land
-__device__ void pass_stats(const Ctx& cx, const int* chunk_q) {
+__device__ void pass_stats(const Ctx& cx, const int* chunk_q, uint32_t parity) {
   uint32_t* hist = reinterpret_cast<uint32_t*>(cx.scratch);
   uint32_t kmax = 0, kminf = 0xFFFFFFFFu, bad = 0;
   float m = -INFINITY, s = 0.0f;
   bool load_ok = true;
   constexpr float kLog2e = 1.4426950408889634f;
   for (int c = 0; c < kLoadChunks; ++c) {
-    if (load_ok && !mbar_wait_bounded(smem_u32(&cx.H->mbar[c]), 0)) {
+    if (load_ok && !mbar_wait_bounded(smem_u32(&cx.H->mbar[c]), parity)) {
       if (threadIdx.x == 0) atomicOr(cx.a->err, kErrSampleLoad);
       load_ok = false;
     }
@@ -2551,7 +2553,12 @@ __device__ void leader_tail(const Ctx& cx, uint32_t tail) {
   write_outputs(cx, L);
 }
 
-__global__ void __launch_bounds__(kThreads, 2) sample_kernel(const __grid_constant__ SampleArgs a) {
+// One row on the cluster (every CTA of it calls this with the same row).
+// Returns when this CTA's share of the row is done: a non-leader may return
+// while the leader still finishes the row from its own shared memory.  The
+// load barriers are initialised once per CTA; `parity` is the phase this
+// row's loads complete (the CTA's rows so far, mod 2).
+__device__ __noinline__ void sample_row(const SampleArgs& a, int row, uint32_t parity) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   SharedHeader* H = reinterpret_cast<SharedHeader*>(smem_raw);
   uint8_t* scratch = smem_raw + ((sizeof(SharedHeader) + 127) & ~size_t(127));
@@ -2565,9 +2572,7 @@ __global__ void __launch_bounds__(kThreads, 2) sample_kernel(const __grid_consta
   cx.list = list;
   cx.C = static_cast<uint32_t>(a.C);
   cx.rank = cluster_ctarank();
-  cx.row = static_cast<int>(blockIdx.x / a.C);
-  // rows the streaming kernel takes (alongside), or resolved (before), are not this kernel's
-  if (a.select == kSelectOthers ? stream_row(a.params[cx.row], a.V) : a.token_ids[cx.row] != kDeferred) return;
+  cx.row = row;
   cx.g0 = static_cast<long long>(cx.rank) * a.part;
   const long long g1 = min(cx.g0 + a.part, static_cast<long long>(a.V));
   const int n = g1 > cx.g0 ? static_cast<int>(g1 - cx.g0) : 0;
@@ -2577,10 +2582,8 @@ __global__ void __launch_bounds__(kThreads, 2) sample_kernel(const __grid_consta
   // ---- chunked load of this CTA's part (1-D bulk copies), one mbarrier per chunk
   int chunk_q[kLoadChunks + 1];
   for (int c = 0; c <= kLoadChunks; ++c) chunk_q[c] = static_cast<int>((static_cast<long long>(cx.n4) * c) / kLoadChunks);
-  if (threadIdx.x == 0) {
-    for (int c = 0; c < kLoadChunks; ++c) mbar_init(smem_u32(&H->mbar[c]), 1);
-    fence_mbar_init();
-  }
+  // a previous row's writes to the part (x in place) are ordered before the copies overwrite it
+  fence_proxy_async_smem();
   __syncthreads();
   if (threadIdx.x == 0) {
     const uint64_t pol = policy_evict_first();
@@ -2616,7 +2619,7 @@ __global__ void __launch_bounds__(kThreads, 2) sample_kernel(const __grid_consta
   __syncthreads();
 
   cluster_arrive();  // this CTA's shared memory is initialised
-  pass_stats(cx, chunk_q);
+  pass_stats(cx, chunk_q, parity);
 
   // ---- first-pass candidates from this CTA's own threshold, straight into the leader's list
   const bool greedy = cx.T == 0.0f;
@@ -2757,6 +2760,48 @@ __global__ void __launch_bounds__(kThreads, 2) sample_kernel(const __grid_consta
   }
 }
 
+// Alongside the streaming kernel (kSelectOthers): cluster g samples row g
+// unless the streaming kernel takes it; grid R * C.  After it
+// (kSelectDeferred): G clusters, cluster g samples the rows g, g + G, ...
+// that the streaming kernel marked kDeferred, one after another (the cluster
+// meets at the end of each row), so a launch costs G clusters whatever R is.
+// Only cluster g reads or writes the marks of its rows, and every CTA of it
+// reads a block of marks before the first cluster barrier of the block's
+// first row, ahead of the leader's writes.
+__global__ void __launch_bounds__(kThreads, 2) sample_kernel(const __grid_constant__ SampleArgs a) {
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  SharedHeader* H = reinterpret_cast<SharedHeader*>(smem_raw);
+  const int g = static_cast<int>(blockIdx.x / a.C);
+  const bool others = a.select == kSelectOthers;
+  if (threadIdx.x == 0) {
+    for (int c = 0; c < kLoadChunks; ++c) mbar_init(smem_u32(&H->mbar[c]), 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  uint32_t rows_done = 0;
+  const long long G = others ? 1 : gridDim.x / a.C;
+  const long long end = others ? g + 1 : a.R;
+  for (long long base = g; base < end; base += G * kThreads) {
+    uint32_t total = 0;
+    if (others) {
+      total = stream_row(a.params[g], a.V) ? 0u : 1u;
+      if (threadIdx.x == 0) H->drows[0] = g;
+    } else {
+      const long long r = base + G * threadIdx.x;
+      const uint32_t d = (r < a.R && a.token_ids[r] == kDeferred) ? 1u : 0u;
+      const uint32_t idx = block_scan_u(d, &total, H) - d;
+      if (d) H->drows[idx] = static_cast<int32_t>(r);
+    }
+    __syncthreads();
+    for (uint32_t i = 0; i < total; ++i) {
+      sample_row(a, H->drows[i], rows_done++ & 1u);
+      if (others) return;  // one row: the CTA leaves when its share is done
+      __syncthreads();
+      cluster_sync();  // the leader has finished the row: the next one may write into its memory
+    }
+  }
+}
+
 }  // namespace vsl
 
 #include "vsl_stream.cuh"
@@ -2833,21 +2878,38 @@ static void stream_geometry(int R, long long V, int sms, int* cluster, int* part
   *part = static_cast<int>(p);
 }
 
-static cudaError_t launch_with_cluster(const void* fn, const SampleArgs& a, int grid, size_t smem, cudaStream_t stream) {
+// `urgent`: the launch gets the device's greatest scheduling priority, so
+// its CTAs are placed before those of a kernel launched beside it.
+static cudaError_t launch_with_cluster(const void* fn, const SampleArgs& a, int grid, size_t smem, cudaStream_t stream,
+                                       bool urgent = false) {
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = static_cast<unsigned>(a.C);
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (urgent) {
+    int least = 0, greatest = 0;
+    const cudaError_t e = cudaDeviceGetStreamPriorityRange(&least, &greatest);
+    if (e != cudaSuccess) return e;
+    attr[1].id = cudaLaunchAttributePriority;
+    attr[1].val.priority = greatest;
+    cfg.numAttrs = 2;
+  }
   void* args[] = {const_cast<SampleArgs*>(&a)};
   return cudaLaunchKernelExC(&cfg, fn, args);
+}
+
+// Clusters of the deferred-row pass: as many as run at once (two CTAs per
+// SM), at most one per row.
+static int deferred_clusters(int R, int cluster, int sms) {
+  return std::max(1, std::min(R, 2 * sms / cluster));
 }
 
 // A batch whose cluster kernel grid covers at most 4 CTAs per SM is latency
@@ -2911,12 +2973,14 @@ cudaError_t launch_sample(const float* const* logits, int R, int S, int V_s, con
     sa.select = kStreamMarks | (sa.C == 1 ? kStreamKoff : 0);
     a.select = kSelectDeferred;
     if ((e = launch_with_cluster(fs, sa, R * sa.C, stream_smem_bytes(), stream)) != cudaSuccess) return e;
-    return launch_with_cluster(fc, a, R * c, sample_smem_bytes(part), stream);
+    return launch_with_cluster(fc, a, deferred_clusters(R, c, sms) * c, sample_smem_bytes(part), stream);
   }
   // a small batch is latency-bound: the two kernels take disjoint rows (decided
-  // by the parameters alone) and run side by side, the cluster kernel on a side
-  // stream forked from and joined back to the caller's; then the cluster kernel
-  // samples the rows the streaming kernel could not hold (marked kDeferred)
+  // by the parameters alone) and run side by side, the streaming kernel on a
+  // side stream forked from and joined back to the caller's; then the cluster
+  // kernel samples the rows the streaming kernel could not hold (marked
+  // kDeferred).  The cluster kernel's rows take the longest, so it is launched
+  // first and with the greatest priority: its CTAs get the SMs first.
   struct Side {
     cudaStream_t s = nullptr;
     cudaEvent_t fork = nullptr, join = nullptr;
@@ -2937,12 +3001,12 @@ cudaError_t launch_sample(const float* const* logits, int R, int S, int V_s, con
   a.select = kSelectOthers;
   if ((e = cudaEventRecord(sd.fork, stream)) != cudaSuccess) return e;
   if ((e = cudaStreamWaitEvent(sd.s, sd.fork, 0)) != cudaSuccess) return e;
-  if ((e = launch_with_cluster(fc, a, R * c, sample_smem_bytes(part), sd.s)) != cudaSuccess) return e;
-  if ((e = launch_with_cluster(fs, sa, R * sa.C, stream_smem_bytes(), stream)) != cudaSuccess) return e;
+  if ((e = launch_with_cluster(fc, a, R * c, sample_smem_bytes(part), stream, true)) != cudaSuccess) return e;
+  if ((e = launch_with_cluster(fs, sa, R * sa.C, stream_smem_bytes(), sd.s)) != cudaSuccess) return e;
   if ((e = cudaEventRecord(sd.join, sd.s)) != cudaSuccess) return e;
   if ((e = cudaStreamWaitEvent(stream, sd.join, 0)) != cudaSuccess) return e;
   a.select = kSelectDeferred;
-  return launch_with_cluster(fc, a, R * c, sample_smem_bytes(part), stream);
+  return launch_with_cluster(fc, a, deferred_clusters(R, c, sms) * c, sample_smem_bytes(part), stream);
 }
 
 }  // namespace vsl

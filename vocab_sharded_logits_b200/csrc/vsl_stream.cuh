@@ -220,7 +220,10 @@ __device__ bool stream_pass(const SampleArgs& a, int row, int g0, int n, float* 
   const uint64_t pol = policy_evict_first();
   int s_issue = 0;
   bool ok = true;
-  __syncthreads();  // every stage of the previous pass is consumed
+  // every stage of the previous pass is consumed, and the leader's writes to
+  // the ring (its scratch) are ordered before the copies overwrite it
+  fence_proxy_async_smem();
+  __syncthreads();
   if (threadIdx.x == 0)
     for (int c = 0; c < min(nch, kStreamStages - 1); ++c)
       stream_issue(a, row, g0, n, c, s_issue, ring, bars, pol, cg % kStreamStages);
