@@ -2866,12 +2866,13 @@ static cudaError_t prepare_sample_kernel() {
   return cudaSuccess;
 }
 
-// Streaming kernel geometry: CTAs per row so that R * C covers two CTAs per
-// SM where the batch is small (at most 8, a portable cluster), and the part
-// of each (a multiple of 4 floats: every part starts 16-byte aligned).
+// Streaming kernel geometry: the most CTAs per row (at most 8, a portable
+// cluster) for which R * C still runs in one wave of two CTAs per SM (a
+// second wave would start only once the first has streamed its parts), and
+// the part of each (a multiple of 4 floats: every part starts 16-byte aligned).
 static void stream_geometry(int R, long long V, int sms, int* cluster, int* part) {
   int c = 1;
-  while (c < 8 && static_cast<long long>(R) * c < 2LL * sms) c <<= 1;
+  while (c < 8 && static_cast<long long>(R) * c * 2 <= 2LL * sms) c <<= 1;
   long long p = (V + c - 1) / c;
   p = (p + 3) / 4 * 4;
   *cluster = c;
