@@ -371,14 +371,14 @@ __device__ __forceinline__ uint32_t word_of(const uint4& w, int i) {
 // Gumbel noise -log(-log u), u = ((w >> 9) + 0.5) * 2^-23, in float32.  -log u
 // is taken as -log1p(-(1 - u)) above one half so that it keeps full relative
 // precision near u = 1 (1 - u is exact).
-__device__ __forceinline__ float gumbel32(uint32_t w) {
+__device__ __noinline__ float gumbel32(uint32_t w) {
   const uint32_t b = w >> 9;
   const float u = (static_cast<float>(b) + 0.5f) * 0x1p-23f;
   const float v = (static_cast<float>(0x7FFFFFu - b) + 0.5f) * 0x1p-23f;  // 1 - u, exact
   const float nl = (u < 0.5f) ? -logf(u) : -log1pf(-v);
   return -logf(nl);
 }
-__device__ __forceinline__ double gumbel64(uint32_t w) {
+__device__ __noinline__ double gumbel64(uint32_t w) {
   const double u = (static_cast<double>(w >> 9) + 0.5) * 0x1p-23;
   return -log(-log(u));
 }
@@ -1219,47 +1219,74 @@ __device__ void op_exact(const Ctx& cx, const Plan& p) {
   const double* tab = cx.H->exp_tab;
   const int jlo = static_cast<int>(p.lo), jhi = static_cast<int>(p.hi);
   double above = 0.0, below = 0.0;
+  // two float4 groups per iteration (q and q + kThreads): their float64 exps
+  // and Philox words are independent chains the warp issues interleaved
   const int nq = (cx.n4 + kThreads - 1) / kThreads * kThreads;
-  for (int q = threadIdx.x; q < nq; q += kThreads) {
-    const bool valid = q < cx.n4;
-    const float4 v4 = valid ? cx.part4[q] : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-    const float v[4] = {v4.x, v4.y, v4.z, v4.w};
-    bool win[4], ab[4];
-    bool any_win = false, any_ab = false;
-    float xmax = -INFINITY;
+  for (int q0 = threadIdx.x; q0 < nq; q0 += 2 * kThreads) {
+    float v[2][4];
+    bool win[2][4], ab[2][4];
+    bool any_win[2] = {false, false}, any_ab[2] = {false, false};
+    float xmax[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const bool fin = v[i] > -INFINITY;
-      const int j = fin ? xbin(v[i], p.m, p.step) : kXBins;
-      win[i] = fin && j >= jlo && j <= jhi;
-      ab[i] = fin && j < jlo;
-      if (fin && !win[i]) {
-        const double e = exp_neg64(static_cast<double>(v[i]) - m, tab);
-        above += ab[i] ? e : 0.0;
-        below += ab[i] ? 0.0 : e;
+    for (int u = 0; u < 2; ++u) {
+      const int q = q0 + u * kThreads;
+      const float4 v4 = q < cx.n4 ? cx.part4[q] : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      v[u][0] = v4.x;
+      v[u][1] = v4.y;
+      v[u][2] = v4.z;
+      v[u][3] = v4.w;
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const bool fin = v[u][i] > -INFINITY;
+        const int j = fin ? xbin(v[u][i], p.m, p.step) : kXBins;
+        win[u][i] = fin && j >= jlo && j <= jhi;
+        ab[u][i] = fin && j < jlo;
+        // exp(-inf - m) is the clamped, negligible value: no branch around the chain
+        const double e = exp_neg64(static_cast<double>(v[u][i]) - m, tab);
+        const double ee = (fin && !win[u][i]) ? e : 0.0;
+        above += ab[u][i] ? ee : 0.0;
+        below += ab[u][i] ? 0.0 : ee;
+        any_win[u] |= win[u][i];
+        any_ab[u] |= ab[u][i];
+        if (ab[u][i]) xmax[u] = fmaxf(xmax[u], v[u][i]);
       }
-      any_win |= win[i];
-      any_ab |= ab[i];
-      if (ab[i]) xmax = fmaxf(xmax, v[i]);
-    }
-    if (__any_sync(0xFFFFFFFFu, any_win)) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        local_append(counter, cx.list, win[i],
-                     (static_cast<uint64_t>(~fkey(v[i])) << 32) | static_cast<uint32_t>(cx.g0 + 4 * q + i));
+    for (int u = 0; u < 2; ++u) {
+      const int q = q0 + u * kThreads;
+      if (__any_sync(0xFFFFFFFFu, any_win[u])) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          local_append(counter, cx.list, win[u][i],
+                       (static_cast<uint64_t>(~fkey(v[u][i])) << 32) | static_cast<uint32_t>(cx.g0 + 4 * q + i));
+      }
     }
-    if (!any_ab) continue;
+    // a group no kept element of which can beat the current best, whatever its noise, is skipped
+    bool need[2];
     {
       const float sb = b.bound_score();
-      if (sb > -INFINITY && xmax + kGMax < sb - score_tol(sb)) continue;
-    }
-    const long long gid0 = cx.g0 + 4LL * q;
-    const uint4 w = philox4x32_10(make_uint4(static_cast<uint32_t>(gid0 >> 2), cx.pos, cx.req, 0u), k0, k1);
-    const float bl = b.bound_l2e();
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      if (ab[i] && (bl == Best::kNoBound || !Best::rejects(bl, v[i], word_of(w, i))))
-        b.offer_passed(v[i], 0.0f, word_of(w, i), static_cast<int32_t>(gid0 + i));
+      for (int u = 0; u < 2; ++u) need[u] = any_ab[u] && !(sb > -INFINITY && xmax[u] + kGMax < sb - score_tol(sb));
+    }
+    if (!(need[0] || need[1])) continue;
+    uint4 w[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const long long gid0 = cx.g0 + 4LL * (q0 + u * kThreads);
+      w[u] = philox4x32_10(make_uint4(static_cast<uint32_t>(gid0 >> 2), cx.pos, cx.req, 0u), k0, k1);
+    }
+    const float bl = b.bound_l2e();  // a bound a little behind the best is still a valid one
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (!need[u]) continue;
+      const long long gid0 = cx.g0 + 4LL * (q0 + u * kThreads);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (ab[u][i] && (bl == Best::kNoBound || !Best::rejects(bl, v[u][i], word_of(w[u], i))))
+          b.offer_passed(v[u][i], 0.0f, word_of(w[u], i), static_cast<int32_t>(gid0 + i));
+    }
   }
   const double ta = block_sum_d0(above, cx.H);
   const double tb = block_sum_d0(below, cx.H);
