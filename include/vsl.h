@@ -112,11 +112,11 @@ VSL_API vsl_status vsl_logits_local(const void* hidden_bf16, const void* const* 
 VSL_API size_t vsl_sample_workspace_bytes(int32_t R, int32_t S, int32_t V_s, int32_t n_logprobs);
 
 /* Number of kernels one vsl_sample call with these sizes launches on the
- * current device (2 for a large batch: the streaming kernel, then the cluster
- * kernel on the rows it leaves; 3 for a small one, R times the cluster size at
- * most 4 per SM: the cluster kernel on a side stream beside the streaming
- * kernel, then a pass over the rows the streaming kernel could not hold), or
- * -1 for sizes vsl_sample rejects.  Host only; no device work. */
+ * current device (2 for a large batch, R above the SM count: the streaming
+ * kernel, then the cluster kernel on the rows it leaves; 3 for a small one:
+ * the cluster kernel beside the streaming kernel, which runs on a side stream,
+ * then a pass over the rows the streaming kernel could not hold), or -1 for
+ * sizes vsl_sample rejects.  Host only; no device work. */
 VSL_API int32_t vsl_sample_launches(int32_t R, int32_t S, int32_t V_s);
 
 /* vsl_sample - per-row temperature, top-k, top-p, Gumbel-max draw and top-n

@@ -64,7 +64,7 @@ def test_integer_inputs_exact(cuda_device):
         assert np.array_equal(o.cpu().numpy().astype(np.float64), r)
 
 
-@pytest.mark.parametrize("name", ["decode", "spec", "large", "peaked"])
+@pytest.mark.parametrize("name", ["decode", "spec", "large", "peaked", "wide"])
 def test_full_size_sampled_entries(cuda_device, name):
     w = W.WORKLOADS[name]
     hidden, ws = W.gemm_inputs(w, cuda_device)

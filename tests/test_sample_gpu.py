@@ -25,7 +25,7 @@ def test_tiny_config_all_rows(cuda_device):
     assert st["rows"] == 4
 
 
-@pytest.mark.parametrize("name", ["decode", "spec", "large", "peaked"])
+@pytest.mark.parametrize("name", ["decode", "spec", "large", "peaked", "wide"])
 def test_small_vocab_versions_all_rows(cuda_device, name):
     # the configs' parameter recipes at a vocabulary the oracle handles in seconds,
     # still several CTAs per row and a ragged tail
@@ -34,7 +34,7 @@ def test_small_vocab_versions_all_rows(cuda_device, name):
     assert st["mismatch_allowed"] <= max(1, st["rows"] // 50)
 
 
-@pytest.mark.parametrize("name,nrows", [("decode", 64), ("spec", 48), ("large", 24), ("peaked", 24)])
+@pytest.mark.parametrize("name,nrows", [("decode", 64), ("spec", 48), ("large", 24), ("peaked", 24), ("wide", 32)])
 def test_full_size_configs_sampled_rows(cuda_device, name, nrows):
     w = W.WORKLOADS[name]
     rows = np.random.default_rng(5).choice(w.R, min(nrows, w.R), replace=False)
@@ -229,8 +229,9 @@ def test_deferred_rows_of_a_large_batch(cuda_device):
 
 
 def test_sample_launch_count(cuda_device):
-    """Small batches run the sampler's kernels side by side (3 launches), large ones in
-    order (2): the decode and speculative-verify sizes on a 148-SM part."""
+    """Small batches (at most one row per SM) run the sampler's kernels side by side
+    (3 launches), large ones in order (2): the decode and speculative-verify sizes."""
     sms = torch.cuda.get_device_properties(cuda_device).multi_processor_count
-    assert vsl.sample_launches(64, 4, 37984) == (3 if 64 * 8 <= 4 * sms else 2)
+    assert vsl.sample_launches(64, 4, 37984) == (3 if 64 <= sms else 2)
+    assert vsl.sample_launches(64, 8, 31040) == (3 if 64 <= sms else 2)
     assert vsl.sample_launches(512, 4, 37984) == 2

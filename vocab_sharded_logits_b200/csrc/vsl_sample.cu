@@ -2940,10 +2940,14 @@ static int deferred_clusters(int R, int cluster, int sms) {
   return std::max(1, std::min(R, 2 * sms / cluster));
 }
 
-// A batch whose cluster kernel grid covers at most 4 CTAs per SM is latency
-// bound: the sampler's kernels then run side by side (three launches).
-static bool small_batch(int R, int cluster, int sms) {
-  return static_cast<long long>(R) * cluster <= 4LL * sms;
+// A batch whose streaming kernel spreads each row over more than one CTA (R
+// at most the SM count) is latency bound: the sampler's kernels then run side
+// by side (three launches), the cluster kernel taking the top-k-off rows the
+// streaming kernel leaves at that geometry.
+static bool small_batch(int R, long long V, int sms) {
+  int sc = 0, sp = 0;
+  stream_geometry(R, V, sms, &sc, &sp);
+  return sc > 1;
 }
 
 static int device_sms() {
@@ -2961,7 +2965,7 @@ int sample_launches(int R, long long V) {
   if (prepare_sample_kernel() != cudaSuccess || !sample_geometry(V, &c, &part)) return -1;
   const int sms = device_sms();
   if (sms <= 0) return -1;
-  return small_batch(R, c, sms) ? 3 : 2;
+  return small_batch(R, V, sms) ? 3 : 2;
 }
 
 cudaError_t launch_sample(const float* const* logits, int R, int S, int V_s, const vsl_row_params* params,
@@ -2995,7 +2999,7 @@ cudaError_t launch_sample(const float* const* logits, int R, int S, int V_s, con
   a.part = part;
   const void* fs = reinterpret_cast<const void*>(stream_kernel);
   const void* fc = reinterpret_cast<const void*>(sample_kernel);
-  if (!small_batch(R, c, sms)) {
+  if (!small_batch(R, a.V, sms)) {
     // a large batch: the streaming kernel first (it marks the rows it leaves),
     // then the cluster kernel on the marked rows
     sa.select = kStreamMarks | (sa.C == 1 ? kStreamKoff : 0);

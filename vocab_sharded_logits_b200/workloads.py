@@ -42,6 +42,10 @@ WORKLOADS = {
     "spec": Workload("spec", 2, 128, 4, 4096, 151936, 4, 20),
     "large": Workload("large", 3, 256, 8, 5120, 151936, 8, 20),
     "peaked": Workload("peaked", 4, 1024, 1, 4096, 262144, 8, 20),
+    # a second vocabulary shape: V = 248,320 over H = 2,560 (the wide vocabulary
+    # relative to the hidden size that makes projection sharding pay), decode-like
+    # batch and parameters, 8 slices of 31,040
+    "wide": Workload("wide", 5, 64, 1, 2560, 248320, 8, 20),
 }
 
 
@@ -61,7 +65,7 @@ def row_params(w, seed_offset=0):
         T = np.full(nreq, 1.0)
         k = np.full(nreq, 50)
         p = np.full(nreq, 0.9)
-    elif w.name == "decode":
+    elif w.name in ("decode", "wide"):
         T = rng.uniform(0.5, 1.5, nreq)
         k = rng.choice([0, 20, 50], nreq)
         p = rng.uniform(0.8, 1.0, nreq)
