@@ -1152,14 +1152,37 @@ __device__ void op_gumbel(const Ctx& cx, const Plan& p) {
 // quantised in-bin offsets; then CTA r replaces its own bins [r, r + 1) *
 // kXBins / C with their sums over the cluster (only CTA r reads that slice of
 // any CTA, so the slice can be overwritten in place).
-__device__ void op_xhist(const Ctx& cx, const Plan& p) {
+__device__ void op_xhist(const Ctx& cx, const Plan& p, uint32_t collect_lo = 0xFFFFFFFFu) {
   uint32_t* cnt = reinterpret_cast<uint32_t*>(cx.scratch);
   uint32_t* qs = cnt + kXBins;
   for (int i = threadIdx.x; i < 2 * kXBins; i += kThreads) cnt[i] = 0;
+  // collect_lo: the raw keys at or above it are this CTA's first-pass candidates,
+  // listed here (the conversion below reads every logit anyway)
+  const bool collect = collect_lo != 0xFFFFFFFFu;
+  uint32_t* counter = collect_counter(cx);
+  if (collect && cx.rank != 0 && threadIdx.x == 0) cx.H->list_aux = 0;
   __syncthreads();
-  for (int q = threadIdx.x; q < cx.n4; q += kThreads) {
-    const float4 v4 = cx.part4[q];
+  const int nq = (cx.n4 + kThreads - 1) / kThreads * kThreads;  // whole warps: the appends are warp-wide
+  for (int q = threadIdx.x; q < nq; q += kThreads) {
+    const bool valid = q < cx.n4;
+    const float4 v4 = valid ? cx.part4[q] : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
     float v[4] = {v4.x, v4.y, v4.z, v4.w};
+    if (collect) {
+      uint32_t k[4];
+      bool any = false;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        k[i] = fkey(v[i]);
+        any |= valid && k[i] >= collect_lo;
+      }
+      if (__any_sync(0xFFFFFFFFu, any)) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          local_append(counter, cx.list, valid && k[i] >= collect_lo,
+                       (static_cast<uint64_t>(~k[i]) << 32) | static_cast<uint32_t>(cx.g0 + 4 * q + i));
+      }
+    }
+    if (!valid) continue;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const bool fin = key_finite(fkey(v[i]));
@@ -1174,6 +1197,7 @@ __device__ void op_xhist(const Ctx& cx, const Plan& p) {
     }
     cx.part4[q] = make_float4(v[0], v[1], v[2], v[3]);
   }
+  if (collect) publish_local_list(cx);
   __syncthreads();
   cluster_sync();  // every CTA's counts are complete
   const int per = kXBins / static_cast<int>(cx.C);
@@ -2656,11 +2680,6 @@ __device__ __noinline__ void sample_row(const SampleArgs& a, int row, uint32_t p
   if (eligible && k_on) rank = max(rank, static_cast<uint32_t>(cx.top_k));
   const LocalPick lp = local_pick(cx, rank, eligible && k_on);
   cluster_wait();    // every CTA's shared memory is initialised: remote access is safe
-  {
-    Plan pc{};
-    pc.lo = lp.lo;
-    op_collect_raw(cx, pc);
-  }
   if (threadIdx.x < cx.C) {
     cluster_ptr(H->need_all, threadIdx.x)[cx.rank] = lp.need;
     cluster_ptr(H->ok_all, threadIdx.x)[cx.rank] = lp.ok;
@@ -2674,6 +2693,29 @@ __device__ __noinline__ void sample_row(const SampleArgs& a, int row, uint32_t p
     all_ok &= H->ok_all[r];
   }
   const bool listed = total <= static_cast<uint32_t>(kListCap);
+  // the merged statistics decide the row's path
+  uint32_t kmax = 0, kminf = 0xFFFFFFFFu, bad = 0;
+  float M = -INFINITY;
+  for (uint32_t r = 0; r < cx.C; ++r) {
+    const CtaStats& st = H->all[r];
+    bad |= st.bad;
+    kmax = max(kmax, st.kmax);
+    kminf = min(kminf, st.kminf);
+    M = fmaxf(M, st.m);
+  }
+  const bool valid_row = !bad && kmax != kKeyNegInf && cx.T > 0.0f && cx.T < INFINITY && cx.top_p > 0.0f &&
+                         cx.top_k >= 0 && !isinf(scale_x(key_value(kmax), cx.T)) &&
+                         !isinf(scale_x(key_value(kminf), cx.T));
+  // a top-k-off top-p row lists its first-pass candidates during XHIST, which
+  // reads every logit anyway; every other row lists them now
+  const bool xhist_direct = valid_row && !k_on && listed && cx.top_p < 1.0f;
+  if (!xhist_direct) {
+    Plan pc{};
+    pc.lo = lp.lo;
+    op_collect_raw(cx, pc);
+    __syncthreads();
+    cluster_sync();  // every CTA's candidates are in the leader's list
+  }
   if (eligible && listed && all_ok) {
     // the list holds the top-n and every top-k survivor: the leader finishes alone
     if (cx.rank == 0) {
@@ -2691,18 +2733,6 @@ __device__ __noinline__ void sample_row(const SampleArgs& a, int row, uint32_t p
   // ---- streamed rows with top-k off and the top-n listed: every CTA derives the
   // same first op from the merged statistics and starts it without a plan round
   {
-    uint32_t kmax = 0, kminf = 0xFFFFFFFFu, bad = 0;
-    float M = -INFINITY;
-    for (uint32_t r = 0; r < cx.C; ++r) {
-      const CtaStats& st = H->all[r];
-      bad |= st.bad;
-      kmax = max(kmax, st.kmax);
-      kminf = min(kminf, st.kminf);
-      M = fmaxf(M, st.m);
-    }
-    const bool valid_row = !bad && kmax != kKeyNegInf && cx.T > 0.0f && cx.T < INFINITY && cx.top_p > 0.0f &&
-                           cx.top_k >= 0 && !isinf(scale_x(key_value(kmax), cx.T)) &&
-                           !isinf(scale_x(key_value(kminf), cx.T));
     if (valid_row && !k_on && listed) {
       const float m = scale_x(M, cx.T);
       Plan p{};
@@ -2724,7 +2754,7 @@ __device__ __noinline__ void sample_row(const SampleArgs& a, int row, uint32_t p
         }
         __syncthreads();
       }
-      if (p.op == OP_XHIST) op_xhist(cx, p);
+      if (p.op == OP_XHIST) op_xhist(cx, p, lp.lo);
       else op_gumbel(cx, p);
       __syncthreads();
       cluster_sync();
