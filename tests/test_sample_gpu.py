@@ -228,6 +228,51 @@ def test_deferred_rows_of_a_large_batch(cuda_device):
     compare(sub, logits[torch.from_numpy(sel).to(cuda_device)].cpu().numpy(), sub_params, 9, 20, range(len(sel)))
 
 
+@pytest.mark.parametrize("requests", [64, 200])
+def test_cuda_graph_capture_replays_the_step(cuda_device, requests):
+    """The projection and the sampler captured into one CUDA graph (side-by-side
+    launches with their fork / join events at 64 rows, the serial pair at 200)
+    replay to the same outputs as the eager calls."""
+    w = W.scaled(W.WORKLOADS["decode"], V=4 * 4096, requests=requests)
+    hidden, ws = W.gemm_inputs(w, cuda_device)
+    T, k, p, req, pos = W.row_params(w)
+    params = vsl.make_row_params(T, k, p, req, pos, cuda_device)
+    logits = [torch.empty(w.R, w.V_s, device=cuda_device) for _ in range(w.S)]
+    n = w.n_logprobs
+
+    def fresh():
+        return vsl.SampleResult(torch.full((w.R,), -7, dtype=torch.int32, device=cuda_device),
+                                torch.zeros(w.R, device=cuda_device),
+                                torch.full((w.R, n), -7, dtype=torch.int32, device=cuda_device),
+                                torch.zeros(w.R, n, device=cuda_device),
+                                torch.full((w.R,), 7, dtype=torch.int32, device=cuda_device))
+
+    eager = fresh()
+    vsl.logits_local(hidden, ws, out=logits)
+    vsl.sample(logits, params, 21, n, out=eager)
+    torch.cuda.synchronize()
+    ref_logits = [t.clone() for t in logits]
+    for t in logits:
+        t.fill_(float("nan"))
+    out = fresh()
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream(cuda_device)
+    side.wait_stream(torch.cuda.current_stream(cuda_device))
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g):
+            vsl.logits_local(hidden, ws, out=logits)
+            vsl.sample(logits, params, 21, n, out=out)
+    torch.cuda.current_stream(cuda_device).wait_stream(side)
+    g.replay()
+    torch.cuda.synchronize()
+    for a, b in zip(logits, ref_logits):
+        assert torch.equal(a, b)
+    for key in ("token_ids", "token_logprob", "topn_ids", "topn_logprob", "row_flags"):
+        assert torch.equal(getattr(out, key), getattr(eager, key)), key
+    del g
+    assert vsl.device_error() == (0, 0)
+
+
 def test_sample_launch_count(cuda_device):
     """Small batches (at most one row per SM) run the sampler's kernels side by side
     (3 launches), large ones in order (2): the decode and speculative-verify sizes."""
