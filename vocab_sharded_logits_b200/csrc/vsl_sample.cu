@@ -30,6 +30,19 @@
 //                    whose edges are exact key boundaries
 //   NARROW_MASS      256-bin refinement of the top-p cut inside an x-key range
 //   GUMBEL           Philox + Gumbel scores over every kept x, per-CTA best
+//   XHIST            (top-k off, top_p < 1) x = fl(l / T) in place, 2,048 fine
+//                    bins of x below m with counts and in-bin offset sums; the
+//                    CTAs bound every bin's mass and agree on the window of
+//                    bins that may hold the cut without a leader round
+//   EXACT            float64 masses above and below the window, the window's
+//                    members listed, the draw over the certainly kept x; the
+//                    leader places the cut inside the sorted window
+//
+// Launches (host side, end of file): a batch of more rows than SMs runs the
+// streaming kernel (vsl_stream.cuh) first, then this kernel on the rows it
+// marked, on a fixed number of clusters that walk those rows; a smaller batch
+// runs this kernel beside the streaming kernel on the rows the parameters give
+// it, then the same marked-row pass.
 //
 // Exactness: x uses IEEE division; the top-k threshold is an exact integer
 // rank selection on keys; the top-p cut compares exact sums of float64 masses
