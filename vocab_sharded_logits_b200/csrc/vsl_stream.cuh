@@ -467,22 +467,34 @@ __global__ void __launch_bounds__(kThreads, 2) stream_kernel(const __grid_consta
   uint32_t grow_limit = static_cast<uint32_t>(kStreamCap - kStreamChunk);
   const uint32_t small_limit = min(grow_limit, 4u * R + 64u);
   const int lane = threadIdx.x & 31;
-  for (int c = 0; c < nch; ++c) {
-    const int stage = c % kStreamStages;
-    // refill the stage scanned in the previous iteration (its barrier has passed)
-    if (threadIdx.x == 0 && c + kStreamStages - 1 < nch)
-      stream_issue(a, cx.row, g0, n, c + kStreamStages - 1, s_issue, ring, H->ring_bar, pol);
-    if (load_ok && !mbar_wait_bounded(smem_u32(&H->ring_bar[stage]), static_cast<uint32_t>(c / kStreamStages) & 1u)) {
-      if (threadIdx.x == 0) atomicOr(a.err, kErrSampleLoad);
-      load_ok = false;
+  // Rounds of one chunk until the first compaction has set the threshold, then
+  // of two: one block barrier per round, so a warp that lists candidates holds
+  // the others up half as often.  The list then has room for one chunk of
+  // candidates per round, not two: a round that lists more (a flood of ties
+  // at the threshold) overflows it, and the row is deferred.
+  int next_issue = min(nch, kStreamStages - 1);  // thread 0: chunks issued so far
+  int step = 1;
+  for (int c = 0; c < nch;) {
+    const int cur = step;  // this round's chunks (a compaction below may widen the next rounds)
+    // refill every stage whose chunk all threads have scanned (the last barrier has passed)
+    if (threadIdx.x == 0)
+      for (; next_issue < min(nch, c + kStreamStages); ++next_issue)
+        stream_issue(a, cx.row, g0, n, next_issue, s_issue, ring, H->ring_bar, pol);
+    for (int u = 0; u < cur && c + u < nch; ++u) {
+      const int cc = c + u;
+      const int stage = cc % kStreamStages;
+      if (load_ok && !mbar_wait_bounded(smem_u32(&H->ring_bar[stage]), static_cast<uint32_t>(cc / kStreamStages) & 1u)) {
+        if (threadIdx.x == 0) atomicOr(a.err, kErrSampleLoad);
+        load_ok = false;
+      }
+      const float4* st4 = reinterpret_cast<const float4*>(ring + static_cast<size_t>(stage) * kStreamChunk);
+      const int nq = min(kStreamChunk, n - cc * kStreamChunk) >> 2;
+      const uint32_t gid = static_cast<uint32_t>(g0 + cc * kStreamChunk);
+      if (nq == kStreamChunk / 4) stream_scan<true>(st4, nq, thr, gid, st, seen, &H->list_count, list);
+      else stream_scan<false>(st4, nq, thr, gid, st, seen, &H->list_count, list);
     }
-    const float4* st4 = reinterpret_cast<const float4*>(ring + static_cast<size_t>(stage) * kStreamChunk);
-    const int nq = min(kStreamChunk, n - c * kStreamChunk) >> 2;
-    const uint32_t gid = static_cast<uint32_t>(g0 + c * kStreamChunk);
-    if (nq == kStreamChunk / 4) stream_scan<true>(st4, nq, thr, gid, st, seen, &H->list_count, list);
-    else stream_scan<false>(st4, nq, thr, gid, st, seen, &H->list_count, list);
-    // the stage is consumed and the appends are visible; the barrier also
-    // tells every thread whether the list has less than a chunk of room left
+    // the round's stages are consumed and the appends are visible; the barrier
+    // also tells every thread whether the list has less than a chunk of room left
     const bool full = __syncthreads_or(seen > grow_limit) != 0;
     seen = 0;
     if (full && !dropped) {
@@ -493,7 +505,9 @@ __global__ void __launch_bounds__(kThreads, 2) stream_kernel(const __grid_consta
       if (left > static_cast<uint32_t>(kStreamCap - kStreamChunk)) dropped = true;
       if (dropped) thr = 0xFFFFFFFFu;
       grow_limit = min(static_cast<uint32_t>(kStreamCap - kStreamChunk), max(small_limit, left + 64u));
+      step = 2;
     }
+    c += cur;
   }
 
   int cg = nch;  // chunks streamed so far (the ring's position)
