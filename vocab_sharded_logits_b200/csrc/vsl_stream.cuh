@@ -18,6 +18,7 @@
 namespace vsl {
 
 constexpr int kStreamCap = 4096;      // candidate list capacity while streaming
+constexpr int kStreamRound = 4;       // chunks per block barrier once the threshold is set
 
 constexpr size_t kStreamListBytes = static_cast<size_t>(kStreamCap) * 8;
 constexpr size_t kStreamRingBytes = static_cast<size_t>(kStreamStages) * kStreamChunk * 4;
@@ -468,10 +469,11 @@ __global__ void __launch_bounds__(kThreads, 2) stream_kernel(const __grid_consta
   const uint32_t small_limit = min(grow_limit, 4u * R + 64u);
   const int lane = threadIdx.x & 31;
   // Rounds of one chunk until the first compaction has set the threshold, then
-  // of two: one block barrier per round, so a warp that lists candidates holds
-  // the others up half as often.  The list then has room for one chunk of
-  // candidates per round, not two: a round that lists more (a flood of ties
-  // at the threshold) overflows it, and the row is deferred.
+  // of kStreamRound: one block barrier per round, so a warp that lists
+  // candidates holds the others up once per round, not once per chunk.  The
+  // list then keeps room for one chunk of candidates, not a round's: a round
+  // that lists more (a flood of ties at the threshold) overflows it, and the
+  // row is deferred.
   int next_issue = min(nch, kStreamStages - 1);  // thread 0: chunks issued so far
   int step = 1;
   for (int c = 0; c < nch;) {
@@ -505,7 +507,7 @@ __global__ void __launch_bounds__(kThreads, 2) stream_kernel(const __grid_consta
       if (left > static_cast<uint32_t>(kStreamCap - kStreamChunk)) dropped = true;
       if (dropped) thr = 0xFFFFFFFFu;
       grow_limit = min(static_cast<uint32_t>(kStreamCap - kStreamChunk), max(small_limit, left + 64u));
-      step = 2;
+      step = kStreamRound;
     }
     c += cur;
   }
