@@ -1,8 +1,9 @@
 // vsl_stream.cuh - streaming sampler for rows resolved from a candidate list
-// (greedy rows, and sampling rows with 0 < top_k <= kStreamMaxK), included by
-// vsl_sample.cu after the cluster kernel it shares the list toolkit with.
+// (greedy rows, sampling rows with 0 < top_k <= kStreamMaxK, and, in a large
+// batch with one CTA per row, top-k-off rows), included by vsl_sample.cu
+// after the cluster kernel it shares the list toolkit with.
 //
-// Such a row needs one pass over its logits: the statistics of the softmax
+// A top-k row needs one pass over its logits: the statistics of the softmax
 // (max, sum of exp, NaN / +inf, smallest finite value) and every logit that
 // can be among the top max(n, k), ties included.  Its part of the row streams
 // from HBM through a ring of shared-memory stages fed by 1-D bulk copies, so
@@ -10,9 +11,11 @@
 // in flight.  Candidates above a running threshold go to a list; when the
 // list fills up it is compacted and the threshold raised.  The cluster's
 // leader then resolves the row from the merged list with the same toolkit as
-// the cluster kernel.  A row this kernel does not take (or whose candidates
-// do not fit) gets the token id kDeferred, and the cluster kernel, launched
-// next on the same stream, samples exactly those rows.
+// the cluster kernel.  A top-k-off row streams its row up to twice more (the
+// fine bins of x, then the masses, window and draw: stream_koff).  A row this
+// kernel does not take (or whose candidates do not fit) gets the token id
+// kDeferred, and the cluster kernel's pass over marked rows, launched after
+// this kernel on the caller's stream, samples exactly those rows.
 #pragma once
 
 namespace vsl {
