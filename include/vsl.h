@@ -21,7 +21,12 @@
  *   - The caller owns every buffer.  "device" pointers are CUDA device
  *     memory of the current device; "host" arrays are ordinary host memory
  *     read during the call only.  The library never allocates device
- *     memory and never synchronises the stream.
+ *     memory and never synchronises the stream.  vsl_sample keeps, per
+ *     device, one side stream and two events (created on first use, kept
+ *     for the process) for the kernels it runs side by side; its calls are
+ *     serialised by a lock around their launches, and they can be captured
+ *     into a CUDA graph (the side stream joins the capture through the
+ *     events).
  *   - stream is a cudaStream_t (NULL = legacy default stream).  Work is
  *     enqueued asynchronously; host-side argument errors are returned before
  *     anything is enqueued, launch errors as VSL_ERR_CUDA.
