@@ -220,6 +220,26 @@ def run_reference(args, w):
     return 0
 
 
+def _e2e_sizes(R, H, n):
+    """Bytes of the packed per-step input (bf16 hidden [R, H], then int32 row
+    parameters [R, 5]) and int32 words of the packed output (token ids, token
+    logprobs, top-n ids, top-n logprobs, row flags) of the end-to-end leg."""
+    return R * H * 2 + R * 5 * 4, R * (3 + 2 * n)
+
+
+def _e2e_views(buf_in, buf_out, R, H, n):
+    """hidden, params and a SampleResult viewing one packed input buffer (uint8)
+    and one packed output buffer (int32), so each step moves one block each way."""
+    import vocab_sharded_logits_b200 as vsl
+    hid = buf_in[: R * H * 2].view(torch.bfloat16).view(R, H)
+    prm = buf_in[R * H * 2:].view(torch.int32).view(R, 5)
+    res = vsl.SampleResult(buf_out[:R], buf_out[R:2 * R].view(torch.float32),
+                           buf_out[2 * R:2 * R + R * n].view(R, n),
+                           buf_out[2 * R + R * n:2 * R + 2 * R * n].view(torch.float32).view(R, n),
+                           buf_out[2 * R + 2 * R * n:])
+    return hid, prm, res
+
+
 def _metric(w):
     return f"sampled rows/sec ({w.name}: logits_local GEMM + sampler, V={w.V})"
 
@@ -309,8 +329,7 @@ def run_gpu(args, w):
     # device and reads its results (one packed buffer of the five outputs) back.
     # The copies run on a copy stream, double-buffered, so step i + 1's inputs
     # cross PCIe while step i computes: the way a serving loop feeds the GPU.
-    in_bytes = w.R * w.H * 2 + w.R * 5 * 4
-    out_words = w.R * (3 + 2 * n)
+    in_bytes, out_words = _e2e_sizes(w.R, w.H, n)
     h2d, d2h = in_bytes, out_words * 4
     pin_in = [torch.empty(in_bytes, dtype=torch.uint8).pin_memory() for _ in range(2)]
     for b in range(2):
@@ -320,18 +339,7 @@ def run_gpu(args, w):
     dev_in = [torch.empty(in_bytes, dtype=torch.uint8, device=dev) for _ in range(2)]
     dev_out = [torch.empty(out_words, dtype=torch.int32, device=dev) for _ in range(2)]
 
-    def views(b):
-        di, do = dev_in[b], dev_out[b]
-        hid = di[: w.R * w.H * 2].view(torch.bfloat16).view(w.R, w.H)
-        prm = di[w.R * w.H * 2:].view(torch.int32).view(w.R, 5)
-        R_ = w.R
-        res = vsl.SampleResult(do[:R_], do[R_:2 * R_].view(torch.float32),
-                               do[2 * R_:2 * R_ + R_ * n].view(w.R, n),
-                               do[2 * R_ + R_ * n:2 * R_ + 2 * R_ * n].view(torch.float32).view(w.R, n),
-                               do[2 * R_ + 2 * R_ * n:])
-        return hid, prm, res
-
-    bufs = [views(0), views(1)]
+    bufs = [_e2e_views(dev_in[b], dev_out[b], w.R, w.H, n) for b in range(2)]
     copy_stream = torch.cuda.Stream(dev)
     ev_in = [torch.cuda.Event() for _ in range(2)]    # inputs of buffer b are on the device
     ev_done = [torch.cuda.Event() for _ in range(2)]  # the step using buffer b has computed

@@ -55,3 +55,29 @@ def test_reference_arm_prints_one_json_line():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["unit"] == "rows/s" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+@pytest.mark.parametrize("R,H,n", [(64, 4096, 20), (4, 64, 5), (7, 24, 0)])
+def test_e2e_packed_buffers_are_split_without_overlap(R, H, n):
+    """The end-to-end leg's packed transfers: the views of hidden, params and the
+    five outputs tile the two buffers exactly, with the shapes and dtypes the
+    binding checks, and the params block starts 16-byte aligned."""
+    import torch
+    sys.path.insert(0, ROOT)
+    import bench
+    in_bytes, out_words = bench._e2e_sizes(R, H, n)
+    bi = torch.zeros(in_bytes, dtype=torch.uint8)
+    bo = torch.zeros(out_words, dtype=torch.int32)
+    hid, prm, res = bench._e2e_views(bi, bo, R, H, n)
+    assert hid.dtype == torch.bfloat16 and tuple(hid.shape) == (R, H) and hid.is_contiguous()
+    assert prm.dtype == torch.int32 and tuple(prm.shape) == (R, 5) and prm.is_contiguous()
+    assert (prm.data_ptr() - bi.data_ptr()) % 16 == 0
+    outs = [res.token_ids, res.token_logprob, res.topn_ids, res.topn_logprob, res.row_flags]
+    assert [t.dtype for t in outs] == [torch.int32, torch.float32, torch.int32, torch.float32, torch.int32]
+    assert [tuple(t.shape) for t in outs] == [(R,), (R,), (R, n), (R, n), (R,)]
+    def spans(ts, base):
+        return sorted((t.data_ptr() - base, t.data_ptr() - base + t.numel() * t.element_size()) for t in ts)
+    for parts, buf in (([hid, prm], bi), (outs, bo)):
+        sp = [x for x in spans(parts, buf.data_ptr()) if x[0] != x[1]]
+        assert sp[0][0] == 0 and sp[-1][1] == buf.numel() * buf.element_size()
+        assert all(a[1] == b[0] for a, b in zip(sp, sp[1:]))
