@@ -709,21 +709,6 @@ __device__ uint32_t raw_prefilter(float theta, float T) {
   return fkey(lo32);
 }
 
-// Warp-aggregated append of sort keys to the leader's list.
-__device__ __forceinline__ void list_append(const Ctx& cx, bool pred, uint64_t key) {
-  const uint32_t mask = __ballot_sync(0xFFFFFFFFu, pred);
-  if (mask == 0) return;
-  const int lane = threadIdx.x & 31;
-  uint32_t base = 0;
-  if (lane == __ffs(mask) - 1)
-    base = atom_add_dsmem_u32(mapa(smem_u32(&cx.H->list_count), 0), __popc(mask));
-  base = __shfl_sync(0xFFFFFFFFu, base, __ffs(mask) - 1);
-  if (pred) {
-    const uint32_t idx = base + __popc(mask & ((1u << lane) - 1u));
-    if (idx < static_cast<uint32_t>(kListCap)) st_dsmem_u64(mapa(smem_u32(cx.list + idx), 0), key);
-  }
-}
-
 // Warp-aggregated append of sort keys to a list in this CTA's own shared memory.
 __device__ __forceinline__ void local_append(uint32_t* counter, uint64_t* list, bool pred, uint64_t key) {
   const uint32_t mask = __ballot_sync(0xFFFFFFFFu, pred);
@@ -1096,15 +1081,6 @@ __device__ void op_collect_x(const Ctx& cx, const Plan& p) {
   }
   publish_local_list(cx);
   push_best(cx, b);
-}
-
-// Cheap test that a candidate with x <= xu cannot beat a score s: that
-// needs -log u < exp(x - bound) for any bound below the best's exact score, and
-// -log u >= 1 - u.
-__device__ __forceinline__ bool gumbel_rejects(float s, float xu, uint32_t w) {
-  const float bound = s - score_tol(s) - 3e-5f;
-  const float q = fast_exp2((xu - bound) * 1.4426950408889634f);
-  return one_minus_u(w) > q * 1.0001f + 1e-30f;
 }
 
 // ---- GUMBEL: argmax of x + g over kept elements (x >= theta), float64-exact;
@@ -1736,19 +1712,6 @@ __device__ void list_gumbel(const Ctx& cx, LeaderState& L, int count, bool x_key
     L.token_l = ok ? l : __int_as_float(0x7FC00000);
   }
   __syncthreads();
-}
-
-// List resolution for a sampling row: the raw list holds the top-n and every
-// top-k survivor.  theta_k by rank, exact top-p by mass narrowing, the draw.
-__device__ void list_sample_tail(const Ctx& cx, LeaderState& L, int count) {
-  float theta = -INFINITY;
-  if (L.r_k > 0) theta = scale_x(key_value(list_rank_key(cx, count, static_cast<uint32_t>(L.r_k))), L.T);
-  if (L.top_p < 1.0f) {
-    const Fx4 z = list_mass_total(cx, L, count, theta);
-    const float theta_p = list_mass_cut(cx, L, count, false, theta, fx_zero(), z);
-    theta = fmaxf(theta, theta_p);
-  }
-  list_gumbel(cx, L, count, false, theta);
 }
 
 // Sorts `count` distinct sort keys (~key << 32 | id) ascending from `in` into
