@@ -23,11 +23,14 @@ reordering beyond what the definition states:
   (same page, section "batch-sharded sampling in one paragraph"); the draw
   (Gumbel-max keyed by Philox4x32 on (seed, request, position, token)) and the
   exact tie / threshold readings are the plainest readings stated in each
-  function's docstring.
+  function's docstring.  ``processed_logprobs`` gives the log-probabilities of
+  the distribution the draw samples from (after temperature, top-k, top-p).
 
 Pins (see ``tests/test_oracle_*.py``): the Philox known-answer vectors of the
 Random123 distribution, brute-force enumeration on tiny vocabularies, closed
 forms (greedy == argmax, top_k=1, top_p -> 0, top_p=1 keeps all, sum of
 probabilities == 1), exact integer GEMMs, and chi-square tests of the draw
-frequencies.  No function here is "parity unpinned".
+frequencies; the processed logprobs against the library log-softmax (full
+vocabulary), point masses, and the frequencies of the oracle's own draws.
+No function here is "parity unpinned".
 """

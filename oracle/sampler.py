@@ -198,6 +198,62 @@ def sample_row(l, temperature, top_k, top_p, request_id, position, seed, n_logpr
     return res
 
 
+@dataclass
+class ProcessedResult:
+    kept: np.ndarray          # bool mask over V of the set the draw is over
+    logprob: np.ndarray       # float64 over V: log q_i on the kept set, -inf elsewhere
+    topn_ids: np.ndarray      # n ids, -1 past the kept set
+    topn_logprob: np.ndarray  # n values, -inf past the kept set
+    flags: int
+
+
+def processed_logprobs(l, temperature, top_k, top_p, n):
+    """Log-probabilities of the distribution the token is drawn from (the
+    "processed" logprobs, after temperature, top-k and top-p).
+
+    Readings (the pages only name logprobs; these restate what the draw above
+    samples from): for a sampling row the kept set K is the draw's (the same
+    top-k and top-p rules), q_i = exp(x_i - m) / sum_{j in K} exp(x_j - m) with
+    m = max_K x, in float64, and log q_i = -inf outside K; a greedy row draws
+    its argmax with certainty, so its kept set is that one token with log q
+    = 0.  The top-n lists the n largest log q (the n largest x of K), lower id
+    first on equal x, then (-1, -inf) once K is exhausted.  A flagged row gets
+    NaN values and ids -1, as for the raw logprobs.
+    """
+    l = np.asarray(l, dtype=np.float32)
+    V = l.size
+    flags = validate(l, temperature, top_k, top_p)
+    if flags:
+        return ProcessedResult(np.zeros(V, bool), np.full(V, np.nan), np.full(n, -1, np.int64),
+                               np.full(n, np.nan), flags)
+    lp = np.full(V, -np.inf)
+    keep = np.zeros(V, bool)
+    if np.float32(temperature) == 0:
+        token = int(np.argmax(l))            # first maximum = lowest id
+        keep[token] = True
+        lp[token] = 0.0
+        x = l
+    else:
+        x = scale(l, temperature)
+        keep = np.isfinite(l).copy()
+        if 0 < top_k < V:
+            keep &= x >= top_k_threshold(x, top_k)
+        if np.float32(top_p) < 1:
+            theta_p, _ = top_p_threshold(x[keep], top_p)
+            keep &= x >= theta_p
+        xk = x[keep].astype(np.float64)
+        m = xk.max()
+        lp[keep] = (xk - m) - np.log(np.sum(np.exp(xk - m)))
+    ids = np.nonzero(keep)[0]
+    order = ids[np.lexsort((ids, -x[ids].astype(np.float64)))]
+    take = order[:n]
+    topn_ids = np.full(n, -1, np.int64)
+    topn_lp = np.full(n, -np.inf)
+    topn_ids[:take.size] = take
+    topn_lp[:take.size] = lp[take]
+    return ProcessedResult(keep, lp, topn_ids, topn_lp, 0)
+
+
 def sample_rows(logits, params, seed, n_logprobs, rows=None):
     """Apply ``sample_row`` to each selected row of a (R, V) float32 array.
 
