@@ -53,14 +53,14 @@ typedef enum {
   VSL_OK = 0,
   VSL_ERR_INVALID_ARG = 1,          /* null pointer, non-positive size, out-of-range value */
   VSL_ERR_ALIGNMENT = 2,            /* pointer or row pitch not 16-byte aligned            */
-  VSL_ERR_UNSUPPORTED = 3,          /* size beyond what this build handles (see limits)    */
+  VSL_ERR_UNSUPPORTED = 3,          /* size beyond the library's limits (see below)        */
   VSL_ERR_WORKSPACE_TOO_SMALL = 4,  /* workspace_bytes below vsl_sample_workspace_bytes()  */
   VSL_ERR_CUDA = 5,                 /* a CUDA runtime / driver call failed                 */
   VSL_ERR_DEVICE_TIMEOUT = 6        /* a kernel gave up a bounded wait (reported later by
                                        vsl_device_error)                                    */
 } vsl_status;
 
-/* Limits of this build. */
+/* Limits of the library. */
 #define VSL_MAX_SLICES 16       /* S <= 16                                  */
 #define VSL_MAX_LOGPROBS 20     /* 0 <= n_logprobs <= 20 (and <= S * V_s)   */
 

@@ -32,7 +32,7 @@ const char* vsl_status_string(vsl_status status) {
     case VSL_OK: return "ok";
     case VSL_ERR_INVALID_ARG: return "invalid argument";
     case VSL_ERR_ALIGNMENT: return "pointer or row pitch not 16-byte aligned";
-    case VSL_ERR_UNSUPPORTED: return "size not supported by this build";
+    case VSL_ERR_UNSUPPORTED: return "size beyond the library's limits";
     case VSL_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
     case VSL_ERR_CUDA: return "CUDA call failed";
     case VSL_ERR_DEVICE_TIMEOUT: return "a kernel gave up a bounded wait";
