@@ -124,6 +124,39 @@ VSL_API size_t vsl_sample_workspace_bytes(int32_t R, int32_t S, int32_t V_s, int
  * sizes vsl_sample rejects.  Host only; no device work. */
 VSL_API int32_t vsl_sample_launches(int32_t R, int32_t S, int32_t V_s);
 
+/* The launches of one vsl_sample call, as plain data (host only, no device
+ * work; vsl_sample makes the same choices on the current device):
+ *   launches       : 2 (serial) or 3 (side by side)
+ *   side_by_side   : 1 when R is at most the SM count: the streaming kernel
+ *                    then splits rows, and the cluster kernel takes the rows
+ *                    it leaves beside it
+ *   stream_cluster : CTAs per row of the streaming kernel (1, 2, 4 or 8: the
+ *                    most for which R times it fits two CTAs per SM)
+ *   stream_part    : logits per streaming CTA;  stream_grid = R * stream_cluster
+ *   cluster, part  : CTAs per row (cluster size) and logits per CTA of the
+ *                    cluster kernel
+ *   others_grid    : its grid beside the streaming kernel (R * cluster; 0 when
+ *                    serial)
+ *   deferred_grid  : the grid of its pass over the rows the streaming kernel
+ *                    marked: min(R, 2 * sms / cluster) clusters
+ * sms is the device's SM count and max_cluster the largest cluster size it
+ * schedules for the cluster kernel (a power of two).  Returns VSL_OK,
+ * VSL_ERR_INVALID_ARG (null out, non-positive sizes), VSL_ERR_ALIGNMENT
+ * (V_s % 4 != 0) or VSL_ERR_UNSUPPORTED (a vocabulary beyond the limits). */
+typedef struct {
+  int32_t launches;
+  int32_t side_by_side;
+  int32_t stream_cluster;
+  int32_t stream_part;
+  int32_t stream_grid;
+  int32_t cluster;
+  int32_t part;
+  int32_t others_grid;
+  int32_t deferred_grid;
+} vsl_sample_plan;
+VSL_API vsl_status vsl_sample_plan_for(int32_t R, int32_t S, int32_t V_s, int32_t sms, int32_t max_cluster,
+                                       vsl_sample_plan* out);
+
 /* vsl_sample - per-row temperature, top-k, top-p, Gumbel-max draw and top-n
  * raw logprobs.
  *   logits_slices : host array of S device pointers, slice s = [R][V_s] fp32

@@ -11,7 +11,7 @@ import os
 import torch
 
 __all__ = [
-    "logits_local", "sample", "sample_launches", "make_row_params", "SampleResult", "lib", "status_string",
+    "logits_local", "sample", "sample_launches", "sample_plan", "make_row_params", "SampleResult", "lib", "status_string",
     "device_error", "VslError", "ROW_NONFINITE", "ROW_ALL_NEG_INF", "ROW_BAD_TEMPERATURE",
     "ROW_BAD_TOP_P", "ROW_BAD_TOP_K", "ROW_SCALE_OVERFLOW", "MAX_SLICES", "MAX_LOGPROBS",
 ]
@@ -38,6 +38,12 @@ class VslError(RuntimeError):
         super().__init__(f"{where}: {_STATUS_NAMES.get(status, status)} ({status_string(status)})")
 
 
+class _Plan(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_int32) for name in (
+        "launches", "side_by_side", "stream_cluster", "stream_part", "stream_grid", "cluster", "part",
+        "others_grid", "deferred_grid")]
+
+
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"libvsl.so not built at {LIB_PATH}; run vocab_sharded_logits_b200/build.py")
@@ -49,6 +55,8 @@ def _load():
     l.vsl_sample_workspace_bytes.argtypes = [i32, i32, i32, i32]
     l.vsl_sample_launches.restype = i32
     l.vsl_sample_launches.argtypes = [i32, i32, i32]
+    l.vsl_sample_plan_for.restype = ctypes.c_int
+    l.vsl_sample_plan_for.argtypes = [i32, i32, i32, i32, i32, ctypes.POINTER(_Plan)]
     l.vsl_sample.restype = ctypes.c_int
     l.vsl_sample.argtypes = [ctypes.POINTER(vp), i32, i32, i32, vp, u64, i32, vp, vp, vp, vp, vp, vp, sz, vp]
     l.vsl_device_error.restype = ctypes.c_int
@@ -181,6 +189,15 @@ def sample_launches(R, S, V_s):
     if n < 0:
         raise VslError(f"vsl_sample_launches: sizes rejected (R={R}, S={S}, V_s={V_s})")
     return n
+
+
+def sample_plan(R, S, V_s, sms, max_cluster):
+    """The launches ``sample`` makes for these sizes on a device with ``sms`` SMs that
+    schedules clusters of at most ``max_cluster`` CTAs, as a dict (host only)."""
+    p = _Plan()
+    _check(lib.vsl_sample_plan_for(int(R), int(S), int(V_s), int(sms), int(max_cluster), ctypes.byref(p)),
+           "vsl_sample_plan_for")
+    return {name: getattr(p, name) for name, _ in _Plan._fields_}
 
 
 def device_error():

@@ -69,6 +69,16 @@ int32_t vsl_sample_launches(int32_t R, int32_t S, int32_t V_s) {
   return vsl::sample_launches(R, static_cast<long long>(S) * V_s);
 }
 
+vsl_status vsl_sample_plan_for(int32_t R, int32_t S, int32_t V_s, int32_t sms, int32_t max_cluster,
+                               vsl_sample_plan* out) {
+  if (out == nullptr || R <= 0 || S <= 0 || V_s <= 0 || sms <= 0 || max_cluster <= 0) return VSL_ERR_INVALID_ARG;
+  if (S > VSL_MAX_SLICES) return VSL_ERR_UNSUPPORTED;
+  if (V_s % 4 != 0) return VSL_ERR_ALIGNMENT;
+  const long long V = static_cast<long long>(S) * V_s;
+  if (V > 0x7FFFFFFFLL || !vsl::sample_plan(R, V, sms, max_cluster, out)) return VSL_ERR_UNSUPPORTED;
+  return VSL_OK;
+}
+
 vsl_status vsl_sample(const float* const* logits_slices, int32_t R, int32_t S, int32_t V_s,
                       const vsl_row_params* params_dev, uint64_t seed, int32_t n_logprobs, int32_t* token_ids,
                       float* token_logprob, int32_t* topn_ids, float* topn_logprob, uint32_t* row_flags,

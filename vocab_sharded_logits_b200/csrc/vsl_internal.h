@@ -27,5 +27,6 @@ cudaError_t launch_sample(const float* const* logits, int R, int S, int V_s,
 // size) and elements per CTA.  Returns false if V cannot be handled.
 bool sample_geometry(long long V, int* cluster, int* part);
 int sample_launches(int R, long long V);
+bool sample_plan(int R, long long V, int sms, int maxc, vsl_sample_plan* out);
 
 }  // namespace vsl

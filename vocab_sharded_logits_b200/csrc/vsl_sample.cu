@@ -2849,11 +2849,11 @@ size_t sample_smem_bytes(int part) {
 
 static int g_max_cluster = -1;  // largest cluster size the device schedules for this kernel
 
-bool sample_geometry(long long V, int* cluster, int* part) {
-  if (V <= 0 || V > static_cast<long long>(kMaxCluster) * kMaxPart) return false;
+// The same for a device that schedules clusters of at most maxc CTAs.
+static bool sample_geometry_for(long long V, int maxc, int* cluster, int* part) {
+  if (V <= 0 || V > static_cast<long long>(kMaxCluster) * kMaxPart || maxc < 1) return false;
   int c = 1;
   while (c < kMaxCluster && (V + c - 1) / c > kPreferredPart) c <<= 1;
-  const int maxc = g_max_cluster > 0 ? g_max_cluster : 8;
   while (c > maxc) c >>= 1;
   long long p = (V + c - 1) / c;
   p = (p + 3) / 4 * 4;
@@ -2861,6 +2861,10 @@ bool sample_geometry(long long V, int* cluster, int* part) {
   *cluster = c;
   *part = static_cast<int>(p);
   return true;
+}
+
+bool sample_geometry(long long V, int* cluster, int* part) {
+  return sample_geometry_for(V, g_max_cluster > 0 ? g_max_cluster : 8, cluster, part);
 }
 
 static cudaError_t prepare_sample_kernel() {
@@ -2966,12 +2970,33 @@ static int device_sms() {
   return sms;
 }
 
-int sample_launches(int R, long long V) {
+// The launches of one call for R rows of V tokens on a device with `sms` SMs
+// that schedules clusters of at most `maxc` CTAs: the choices launch_sample
+// makes, as plain data.  Returns false if V cannot be handled.
+bool sample_plan(int R, long long V, int sms, int maxc, vsl_sample_plan* out) {
   int c = 0, part = 0;
-  if (prepare_sample_kernel() != cudaSuccess || !sample_geometry(V, &c, &part)) return -1;
+  if (R <= 0 || sms <= 0 || !sample_geometry_for(V, maxc, &c, &part)) return false;
+  int sc = 0, sp = 0;
+  stream_geometry(R, V, sms, &sc, &sp);
+  const bool side = small_batch(R, V, sms);
+  out->launches = side ? 3 : 2;
+  out->side_by_side = side ? 1 : 0;
+  out->stream_cluster = sc;
+  out->stream_part = sp;
+  out->stream_grid = R * sc;
+  out->cluster = c;
+  out->part = part;
+  out->others_grid = side ? R * c : 0;
+  out->deferred_grid = deferred_clusters(R, c, sms) * c;
+  return true;
+}
+
+int sample_launches(int R, long long V) {
+  if (prepare_sample_kernel() != cudaSuccess) return -1;
   const int sms = device_sms();
-  if (sms <= 0) return -1;
-  return small_batch(R, V, sms) ? 3 : 2;
+  vsl_sample_plan p{};
+  if (sms <= 0 || !sample_plan(R, V, sms, g_max_cluster > 0 ? g_max_cluster : 8, &p)) return -1;
+  return p.launches;
 }
 
 cudaError_t launch_sample(const float* const* logits, int R, int S, int V_s, const vsl_row_params* params,
