@@ -81,3 +81,43 @@ def test_e2e_packed_buffers_are_split_without_overlap(R, H, n):
         sp = [x for x in spans(parts, buf.data_ptr()) if x[0] != x[1]]
         assert sp[0][0] == 0 and sp[-1][1] == buf.numel() * buf.element_size()
         assert all(a[1] == b[0] for a, b in zip(sp, sp[1:]))
+
+
+def test_clock_sampler_reads_clocks_and_throttle_reasons(tmp_path):
+    """The clocks line of the JSON: median SM clock under load, the max clock and
+    every throttle reason seen active, from nvidia-smi's CSV (samples taken
+    before the timed steps are skipped)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    csv = tmp_path / "clocks.csv"
+    csv.write_text("\n".join([
+        "0, 1200, 1965, 150.0, 0x0, Not Active, Not Active, Not Active, Not Active",   # before the steps
+        "0, 1965, 1965, 700.5, 0x4, Not Active, Not Active, Not Active, Active",
+        "0, 1950, 1965, 710.0, 0x4, Not Active, Not Active, Not Active, Active",
+        "0, 1935, 1965, 690.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "garbage line",
+    ]) + "\n")
+
+    class _Proc:
+        def send_signal(self, sig):
+            pass
+
+        def wait(self, timeout=None):
+            return 0
+
+    c = bench.ClockSampler(0)
+    c.proc, c.path, c.skip = _Proc(), str(csv), 1
+    got = c.stop()
+    assert got == {"sm_mhz": 1950.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
+
+
+def test_recorded_traffic_needs_the_sources_it_was_captured_from(monkeypatch):
+    """A profile's DRAM bytes are used only while the kernel's sources hash to
+    the value recorded beside them."""
+    sys.path.insert(0, ROOT)
+    import bench
+    got = bench._recorded_traffic("logits_local_kernel", "decode")
+    assert isinstance(got, int) and got > 0
+    monkeypatch.setattr(bench, "_source_sha", lambda kernel: "0" * 64)
+    assert bench._recorded_traffic("logits_local_kernel", "decode") is None
+    assert bench._recorded_traffic("logits_local_kernel", "no_such_workload") is None
