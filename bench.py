@@ -2,15 +2,18 @@
 
 One step = one pass of the whole hot path over one batch: ``logits_local``
 (tcgen05 GEMM, every vocab slice, no gather) followed by ``sample``
-(temperature / top-k / top-p / Gumbel-max draw / top-n logprobs) on the
-"decode" workload by default: 64 requests x 1 row, hidden 4096, vocab 151936
-in 4 slices, bf16 hidden N(0,1) and lm_head N(0,0.02), per-request
-T ~ U[0.5,1.5], top_k in {off,20,50}, top_p ~ U[0.8,1.0], top-20 logprobs.
+(temperature / top-k / top-p / Gumbel-max draw / top-n logprobs).  The
+headline line is the "large batch" workload by default: 256 requests x 8 rows
+(7 speculative tokens + 1) = 2048 rows, hidden 5120, vocab 151936 in 8 slices,
+bf16 hidden N(0,1) and lm_head N(0,0.02), per-request T ~ U[0.3,1.2],
+top_p ~ U[0.5,1.0], top_k off, top-20 logprobs.  The same line carries
+``per_config``: every workload measured in the same run (projection TFLOP/s,
+sampler GB/s with L2 flushed, rows/s in the step and end to end).
 
-Prints ONE JSON line (rank 0).  ``--impl reference`` times the CPU oracle on
-the same workload instead.  Multi-GPU (torchrun): every rank runs its own
-batch (weak scaling, no collective on the data path); the timed region is
-bracketed by barriers and the max over ranks is reported.
+Prints ONE JSON line (rank 0).  ``--impl reference`` times the CPU sampler
+oracle on the same workload instead.  Multi-GPU (torchrun): every rank runs its
+own batch (weak scaling, no collective on the data path); every timed region
+is bracketed by barriers and the max over ranks is reported.
 """
 import argparse
 import json
@@ -29,12 +32,17 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from vocab_sharded_logits_b200 import workloads as W  # noqa: E402
+import workloads as W  # noqa: E402
 
 L2_BYTES = 126 * 1024 * 1024
+METRIC = "sampled rows/sec and sampler HBM GB/s at V=151936; logits-GEMM TFLOPS on 1 B200"
+# every workload measured into per_config, in this order (the headline's first)
+PER_CONFIG = ["tiny", "decode", "spec", "large", "peaked", "wide"]
+PARITY_SEED = 777
 
 
 def _peaks():
+    """(HBM GB/s, bf16 TF/s burst, bf16 TF/s sustained, source)."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
@@ -45,8 +53,7 @@ def _peaks():
 
 
 # The timed units of a step and the sources each is built from.  "sample" is
-# one call of the sampler: the streaming kernel (greedy and top-k <= 1024 rows)
-# followed by the cluster kernel (the other rows).
+# one call of the sampler (the streaming kernel and the cluster kernel).
 _KERNEL_SOURCES = {"logits_local_kernel": ["vsl_gemm.cu"], "sample": ["vsl_sample.cu", "vsl_stream.cuh"]}
 
 
@@ -59,10 +66,10 @@ def _source_sha(kernel):
     return h.hexdigest()
 
 
-def _recorded_traffic(kernel, workload):
+def _recorded_traffic(kernel, workload, profiles_dir=None):
     """DRAM bytes per call recorded from an ncu capture in profiles/<kernel>_<workload>.md,
     or None when there is none or the sources changed since (sha256 over them differs)."""
-    prof = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+    prof = os.path.join(profiles_dir or os.path.join(ROOT, "profiles"), f"{kernel}_{workload}.md")
     if not os.path.exists(prof):
         return None
     fields = {}
@@ -169,56 +176,99 @@ def _barrier(world):
         dist.barrier()
 
 
-def cpu_oracle_rows(w, n_rows, seed=0):
-    """Times the oracle on ``n_rows`` rows of workload ``w`` (projection + sampler).
+# ------------------------------------------------------------------ the CPU oracle
 
-    Returns (seconds, rows, threads).  Inputs are made on the CPU from the same
-    seeded recipe; only the oracle calls are timed.
-    """
-    from oracle.gemm import logits_local as ref_logits
-    from oracle.sampler import sample_row
-    hidden, ws = W.gemm_inputs(W.scaled(w, requests=max(1, n_rows // w.rows_per_request)), "cpu")
-    h = hidden.float().numpy()[:n_rows]
-    ws_np = [x.float().numpy() for x in ws]
-    T, k, p, req, pos = W.row_params(w)
+def _nproc():
     try:
-        from threadpoolctl import threadpool_info
-        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    except Exception:
-        threads = os.cpu_count() or 1
-    t0 = time.perf_counter()
-    logits = np.concatenate(ref_logits(h, ws_np), axis=1).astype(np.float32)
-    for r in range(n_rows):
-        sample_row(logits[r], T[r], int(k[r]), p[r], int(req[r]), int(pos[r]), seed, w.n_logprobs)
-    return time.perf_counter() - t0, n_rows, threads
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def oracle_baseline(logits_np, params, seed, n_logprobs, label, gpu_tokens=None, budget_s=2.0, reps=5):
+    """The sampler oracle, as it stands, timed on this host's cores over rows of
+    ``logits_np`` (float32 [rows, V]): one thread, then one worker per core (rows
+    split between them), wall clock, median of ``reps`` runs of about ``budget_s``
+    each.  Returns the ``cpu_baseline`` object and, when ``gpu_tokens`` is given,
+    a token parity summary of the GPU's draw (same logits, same seed) against the
+    oracle's on every row the all-cores runs sampled."""
+    from oracle.timing import OracleSampler, cpu_model
+    rows_avail = logits_np.shape[0]
+    nproc = _nproc()
+    orc = OracleSampler(logits_np, params, seed, n_logprobs, workers=nproc)
+    try:
+        t, _ = orc.run([0], parallel=False)          # warm-up and a first estimate
+        t, _ = orc.run([min(1, rows_avail - 1)], parallel=False)
+        per_row = max(t, 1e-4)
+        n1 = max(2, min(rows_avail, int(budget_s / per_row)))
+        rate1, med1, _ = orc.median_rate(range(n1), parallel=False, reps=reps)
+        orc.start_workers()
+        n_all = max(nproc, min(4 * rows_avail, nproc * max(1, int(budget_s / per_row))))
+        rows_all = [r % rows_avail for r in range(n_all)]
+        rate_all, med_all, res = orc.median_rate(rows_all, parallel=True, reps=reps)
+    finally:
+        orc.close()
+    base = {"value": rate_all, "unit": "rows/s", "cores": nproc, "kind": "oracle",
+            "sample": f"{label}: the sampler oracle (float64, sort based) over rows of the same fp32 logits; "
+                      f"all cores: {n_all} rows per run on {nproc} worker processes ({med_all:.2f} s); one thread: "
+                      f"{n1} rows per run ({med1:.2f} s); median of {reps} runs each",
+            "threads_1": rate1, "threads_all": rate_all, "nproc": nproc, "cpu_model": cpu_model()}
+    parity = None
+    if gpu_tokens is not None:
+        seen = {}
+        for r, tok, near, cut, flags in res:
+            seen[r] = (tok, near, cut, flags)
+        eq = sum(1 for r, (tok, _, _, _) in seen.items() if int(gpu_tokens[r]) == tok)
+        near = sum(1 for v in seen.values() if v[1])
+        cut = sum(1 for v in seen.values() if v[2])
+        unexplained = sum(1 for r, (tok, nt, ct, _) in seen.items() if int(gpu_tokens[r]) != tok and not (nt or ct))
+        parity = {"rows": len(seen), "token_equal": eq, "near_tie": near, "cut_tie": cut,
+                  "mismatch_unexplained": unexplained, "seed": seed}
+    return base, parity
 
 
 def run_reference(args, w):
+    """The oracle arm: the sampler oracle on the host's cores, each step a bounded
+    sample of the workload's rows (synthetic fp32 logits with the spread of the
+    projection's output), all cores."""
     world, rank, _ = _dist_setup(args.gpus)
     if rank != 0:
         return 0
-    for _ in range(args.warmup):
-        cpu_oracle_rows(w, 1)
-    times, rows = [], 0
-    for _ in range(args.steps):
-        t, n, threads = cpu_oracle_rows(w, args.reference_rows)
-        times.append(t)
-        rows += n
+    from oracle.timing import OracleSampler, cpu_model
+    nproc = _nproc()
+    rows = max(1, min(w.R, args.reference_rows * nproc))
+    wl = W.scaled(w, requests=max(1, -(-rows // w.rows_per_request)))
+    logits = W.sampler_logits(wl, "cpu").numpy()[:rows]
+    params = W.row_params(w)
+    orc = OracleSampler(logits, params, 0, w.n_logprobs, workers=nproc)
+    try:
+        orc.start_workers()
+        for _ in range(args.warmup):
+            orc.run(range(min(rows, nproc)), parallel=True)
+        times = []
+        for _ in range(args.steps):
+            t, _ = orc.run(range(rows), parallel=True)
+            times.append(t)
+    finally:
+        orc.close()
     total = sum(times)
-    value = rows / total
+    value = rows * args.steps / total
+    sample = (f"{rows} rows per step of the {w.name} workload (V={w.V}): the sampler oracle over synthetic fp32 "
+              f"logits with the projection's spread, {nproc} worker processes")
     line = {
-        "impl": "reference", "metric": _metric(w), "value": value, "unit": "rows/s", "n_gpus": args.gpus,
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "rows/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": _config(w),
-        "cpu_baseline": {"value": value, "unit": "rows/s", "cores": threads, "kind": "oracle",
-                         "sample": f"{args.reference_rows} rows per step of the {w.name} workload "
-                                   f"(float64 projection of those rows over all {w.V} tokens + the sampler oracle)"},
+        "cpu_baseline": {"value": value, "unit": "rows/s", "cores": nproc, "kind": "oracle", "sample": sample,
+                         "nproc": nproc, "cpu_model": cpu_model()},
         "e2e": {"value": value, "unit": "rows/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
 
+
+# ------------------------------------------------------------------ the GPU arm
 
 def _e2e_sizes(R, H, n):
     """Bytes of the packed per-step input (bf16 hidden [R, H], then int32 row
@@ -240,28 +290,35 @@ def _e2e_views(buf_in, buf_out, R, H, n):
     return hid, prm, res
 
 
-def _metric(w):
-    return f"sampled rows/sec ({w.name}: logits_local GEMM + sampler, V={w.V})"
-
-
 def _config(w):
     return {"workload": w.name, "requests": w.requests, "rows": w.R, "hidden": w.H, "vocab": w.V, "slices": w.S,
-            "n_logprobs": w.n_logprobs, "l2": "inputs larger than L2 (lm_head weights "
-            f"{w.V * w.H * 2 / 1e9:.3f} GB read per step); sampler-only figure flushes L2 between reps"}
+            "n_logprobs": w.n_logprobs,
+            "sampler_input": "synthetic peaked / long-tail logits" if w.name == "peaked" else "the projection's output",
+            "l2": "inputs larger than L2 in the step (lm_head weights "
+                  f"{w.V * w.H * 2 / 1e9:.3f} GB read per step); the sampler-alone figures flush L2 (a 252 MB "
+                  "write) before every rep"}
 
 
-def run_gpu(args, w):
+def _events(n):
+    return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+
+
+def measure_config(w, dev, world, rank, steps, warmup, peaks):
+    """One workload on this rank: the timed steps (projection + sampler, events per
+    kernel on the launching stream), the sampler alone with L2 flushed, the end-to-end
+    leg through the public API with host buffers.  Times are maxima over ranks.
+    Returns (summary dict, state for the headline's extra legs)."""
     import vocab_sharded_logits_b200 as vsl
-    world, rank, local = _dist_setup(args.gpus)
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
+    hbm_peak, tf_peak, _, _ = peaks
     stream = torch.cuda.current_stream(dev)
-    hbm_peak, tf_peak, tf_sus, peak_kind = _peaks()
-
     hidden, ws = W.gemm_inputs(w, dev)
     T, k, p, req, pos = W.row_params(w)
     params = vsl.make_row_params(T, k, p, req + rank * w.requests, pos, dev)
     logits = [torch.empty(w.R, w.V_s, dtype=torch.float32, device=dev) for _ in range(w.S)]
+    # the peaked workload's sampler reads its own synthetic logits; the others sample the projection's output
+    samp_in = logits
+    if w.name == "peaked":
+        samp_in = [t.contiguous() for t in torch.tensor_split(W.sampler_logits(w, dev), w.S, dim=1)]
     n = w.n_logprobs
     out = vsl.SampleResult(torch.empty(w.R, dtype=torch.int32, device=dev), torch.empty(w.R, device=dev),
                            torch.empty(w.R, n, dtype=torch.int32, device=dev), torch.empty(w.R, n, device=dev),
@@ -269,68 +326,49 @@ def run_gpu(args, w):
 
     def step(seed):
         vsl.logits_local(hidden, ws, out=logits, stream=stream)
-        vsl.sample(logits, params, seed, n, out=out, stream=stream)
+        vsl.sample(samp_in, params, seed, n, out=out, stream=stream)
 
-    for i in range(args.warmup):
+    for i in range(warmup):
         step(i)
     torch.cuda.synchronize()
-
-    # ---- timed region: K steps, per-kernel events on the launching stream
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    clocks = ClockSampler(local)
-    clocks.start()
+    ev = [_events(3) for _ in range(steps)]
     _barrier(world)
     torch.cuda.synchronize()
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-    t_start.record(stream)
-    for i in range(args.steps):
+    t0, t1 = _events(2)
+    t0.record(stream)
+    for i in range(steps):
         a, b, c = ev[i]
         a.record(stream)
         vsl.logits_local(hidden, ws, out=logits, stream=stream)
         b.record(stream)
-        vsl.sample(logits, params, 1000 + i, n, out=out, stream=stream)
+        vsl.sample(samp_in, params, 1000 + i, n, out=out, stream=stream)
         c.record(stream)
-    t_end.record(stream)
+    t1.record(stream)
     torch.cuda.synchronize()
-    # a timed region shorter than the sampling period still gets samples: keep
-    # running the same step (untimed) until three samples under load exist
-    t0 = time.time()
-    while clocks.proc is not None and clocks.count() - clocks.skip < 3 and time.time() - t0 < 10:
-        for i in range(20):
-            step(5000 + i)
-        torch.cuda.synchronize()
-    _barrier(world)
-    clk = clocks.stop()
-    total_ms = t_start.elapsed_time(t_end)
-    gemm_ms = sum(a.elapsed_time(b) for a, b, _ in ev) / args.steps
-    samp_ms = sum(b.elapsed_time(c) for _, b, c in ev) / args.steps
-    total_ms = _max_over_ranks(total_ms, world, dev)
-    ms_per_step = total_ms / args.steps
-    value = world * w.R * args.steps / (total_ms / 1e3)
+    total_ms = _max_over_ranks(t0.elapsed_time(t1), world, dev)
+    gemm_ms = _max_over_ranks(sum(a.elapsed_time(b) for a, b, _ in ev) / steps, world, dev)
+    samp_ms = _max_over_ranks(sum(b.elapsed_time(c) for _, b, c in ev) / steps, world, dev)
 
-    # ---- sampler alone with L2 flushed between reps (its HBM figure)
+    # the sampler alone, L2 flushed before every rep (its HBM figure)
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
     s_times = []
-    for i in range(max(3, args.steps)):
+    for i in range(max(5, steps)):
         flush.fill_(float(i))
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0, e1 = _events(2)
         e0.record(stream)
-        vsl.sample(logits, params, 2000 + i, n, out=out, stream=stream)
+        vsl.sample(samp_in, params, 2000 + i, n, out=out, stream=stream)
         e1.record(stream)
         torch.cuda.synchronize()
         s_times.append(e0.elapsed_time(e1))
-    samp_cold_ms = statistics.median(s_times)
     del flush
+    samp_cold_ms = _max_over_ranks(statistics.median(s_times), world, dev)
 
-    # ---- end to end through the public API with host buffers.  Every step copies
-    # its inputs (hidden states + row parameters, one packed pinned buffer) to the
-    # device and reads its results (one packed buffer of the five outputs) back.
-    # The copies run on a copy stream, double-buffered, so step i + 1's inputs
-    # cross PCIe while step i computes: the way a serving loop feeds the GPU.
+    # end to end through the public API with host buffers: every step copies its
+    # inputs (hidden states + row parameters, one packed pinned buffer) to the
+    # device and reads its results (one packed buffer of the five outputs) back,
+    # on a copy stream, double-buffered, so step i + 1's inputs cross PCIe while
+    # step i computes: the way a serving loop feeds the GPU
     in_bytes, out_words = _e2e_sizes(w.R, w.H, n)
-    h2d, d2h = in_bytes, out_words * 4
     pin_in = [torch.empty(in_bytes, dtype=torch.uint8).pin_memory() for _ in range(2)]
     for b in range(2):
         pin_in[b][: w.R * w.H * 2].view(torch.bfloat16).view(w.R, w.H).copy_(hidden.cpu())
@@ -338,19 +376,18 @@ def run_gpu(args, w):
     pin_out = [torch.empty(out_words, dtype=torch.int32).pin_memory() for _ in range(2)]
     dev_in = [torch.empty(in_bytes, dtype=torch.uint8, device=dev) for _ in range(2)]
     dev_out = [torch.empty(out_words, dtype=torch.int32, device=dev) for _ in range(2)]
-
     bufs = [_e2e_views(dev_in[b], dev_out[b], w.R, w.H, n) for b in range(2)]
     copy_stream = torch.cuda.Stream(dev)
     ev_in = [torch.cuda.Event() for _ in range(2)]    # inputs of buffer b are on the device
     ev_done = [torch.cuda.Event() for _ in range(2)]  # the step using buffer b has computed
     ev_out = [torch.cuda.Event() for _ in range(2)]   # results of buffer b are on the host
 
-    def e2e_run(first_seed, steps, start=None):
+    def e2e_run(first_seed, nsteps, start=None):
         if start is not None:
             copy_stream.wait_event(start)  # no copy of the timed steps starts before the clock
         for b in range(2):
             ev_out[b].record(copy_stream)
-        for i in range(steps):
+        for i in range(nsteps):
             b = i & 1
             hid, prm, res = bufs[b]
             with torch.cuda.stream(copy_stream):
@@ -359,7 +396,7 @@ def run_gpu(args, w):
                 ev_in[b].record(copy_stream)
             stream.wait_event(ev_in[b])
             vsl.logits_local(hid, ws, out=logits, stream=stream)
-            vsl.sample(logits, prm, first_seed + i, n, out=res, stream=stream)
+            vsl.sample(samp_in, prm, first_seed + i, n, out=res, stream=stream)
             ev_done[b].record(stream)
             with torch.cuda.stream(copy_stream):
                 copy_stream.wait_event(ev_done[b])
@@ -368,65 +405,123 @@ def run_gpu(args, w):
         for b in range(2):
             stream.wait_event(ev_out[b])  # every result is on the host
 
-    e2e_run(0, args.warmup)
+    e2e_run(0, warmup)
     torch.cuda.synchronize()
     _barrier(world)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0, e1 = _events(2)
     e0.record(stream)
-    e2e_run(3000, args.steps, e0)
+    e2e_run(3000, steps, e0)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = _max_over_ranks(e0.elapsed_time(e1), world, dev)
-    e2e_value = world * w.R * args.steps / (e2e_ms / 1e3)
+    _barrier(world)
+
+    gemm_bytes = w.V * w.H * 2 + w.R * w.H * 2 + w.R * w.V * 4
+    gemm_flops = 2.0 * w.R * w.H * w.V
+    samp_bytes = w.R * w.V * 4
+    ridge = tf_peak * 1e12 / (hbm_peak * 1e9)
+    gemm_hbm = gemm_flops / gemm_bytes < ridge
+    gemm_tf = gemm_flops / (gemm_ms / 1e3) / 1e12
+    gemm_gbs = gemm_bytes / (gemm_ms / 1e3) / 1e9
+    samp_gbs_cold = samp_bytes / (samp_cold_ms / 1e3) / 1e9
+    summary = {
+        "rows": w.R, "vocab": w.V, "hidden": w.H, "slices": w.S,
+        "step_ms": total_ms / steps, "rows_per_s": world * w.R * steps / (total_ms / 1e3),
+        "e2e_rows_per_s": world * w.R * steps / (e2e_ms / 1e3),
+        "gemm_ms": gemm_ms, "gemm_tflops": gemm_tf, "gemm_hbm_gbs": gemm_gbs,
+        "gemm_bound": "hbm" if gemm_hbm else "tensor",
+        "gemm_frac": (gemm_gbs / hbm_peak) if gemm_hbm else (gemm_tf / tf_peak),
+        "gemm_frac_of": "measured HBM copy GB/s" if gemm_hbm else "measured bf16 burst TF/s",
+        "sample_ms_in_step": samp_ms, "sample_ms_cold_l2": samp_cold_ms,
+        "sampler_hbm_gbs_cold_l2": samp_gbs_cold, "sampler_frac_cold_l2": samp_gbs_cold / hbm_peak,
+        "sampler_rows_per_s_cold_l2": w.R / (samp_cold_ms / 1e3),
+    }
+    state = {"samp_in": samp_in, "params": params, "T": T, "k": k, "p": p, "req": req + rank * w.requests,
+             "pos": pos, "total_ms": total_ms, "gemm_ms": gemm_ms, "samp_ms": samp_ms, "e2e_ms": e2e_ms,
+             "h2d": in_bytes, "d2h": out_words * 4, "gemm_bytes": gemm_bytes, "gemm_flops": gemm_flops,
+             "samp_bytes": samp_bytes, "gemm_hbm": gemm_hbm, "out": out}
+    return summary, state
+
+
+def run_gpu(args, w):
+    import vocab_sharded_logits_b200 as vsl
+    world, rank, local = _dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks = _peaks()
+    hbm_peak, tf_peak, _, peak_kind = peaks
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    head, st = measure_config(w, dev, world, rank, args.steps, args.warmup, peaks)
+    # a timed region shorter than the sampling period still gets samples
+    t0 = time.time()
+    while clocks.proc is not None and clocks.count() - clocks.skip < 3 and time.time() - t0 < 10:
+        for i in range(10):
+            vsl.sample(st["samp_in"], st["params"], 5000 + i, w.n_logprobs, out=st["out"])
+        torch.cuda.synchronize()
+
+    # the GPU's draw on the headline's logits for the bench-side parity count
+    parity_out = vsl.sample(st["samp_in"], st["params"], PARITY_SEED, w.n_logprobs)
+    gpu_tokens = parity_out.token_ids.cpu().numpy()
+    logits_host = None
+    if rank == 0 and world == 1 and not args.skip_cpu:
+        logits_host = torch.cat([t.cpu() for t in st["samp_in"]], dim=1).numpy()
+    del parity_out
+
+    per_config = {w.name: head}
+    if not args.no_per_config:
+        for name in PER_CONFIG:
+            if name == w.name:
+                continue
+            torch.cuda.empty_cache()
+            per_config[name], _ = measure_config(W.WORKLOADS[name], dev, world, rank, max(5, args.steps // 2),
+                                                 max(3, args.warmup), peaks)
+    clk = clocks.stop()
     _barrier(world)
 
     status = vsl.device_error()
     if status != (0, 0):
         print(f"device error word set: {status}", file=sys.stderr)
 
-    # ---- roofline of the dominant kernel
-    gemm_bytes = w.V * w.H * 2 + w.R * w.H * 2 + w.R * w.V * 4
-    gemm_flops = 2.0 * w.R * w.H * w.V
-    samp_bytes = w.R * w.V * 4
-    intensity = gemm_flops / gemm_bytes
-    ridge = tf_peak * 1e12 / (hbm_peak * 1e9)
-    if gemm_ms >= samp_ms:
-        if intensity < ridge:
-            roof = {"kernel": "logits_local_kernel", "bound": "hbm", "achieved": gemm_bytes / (gemm_ms / 1e3) / 1e9,
-                    "peak": hbm_peak, "unit": "GB/s"}
+    # roofline of the step's dominant kernel (a per-kernel event time inside a
+    # millisecond-scale region: the burst peaks)
+    if st["gemm_ms"] >= st["samp_ms"]:
+        if st["gemm_hbm"]:
+            roof = {"kernel": "logits_local_kernel", "bound": "hbm",
+                    "achieved": st["gemm_bytes"] / (st["gemm_ms"] / 1e3) / 1e9, "peak": hbm_peak, "unit": "GB/s"}
         else:
-            roof = {"kernel": "logits_local_kernel", "bound": "tensor", "achieved": gemm_flops / (gemm_ms / 1e3) / 1e12,
-                    "peak": tf_sus, "unit": "TFLOP/s"}
+            roof = {"kernel": "logits_local_kernel", "bound": "tensor",
+                    "achieved": st["gemm_flops"] / (st["gemm_ms"] / 1e3) / 1e12, "peak": tf_peak, "unit": "TFLOP/s"}
     else:
-        roof = {"kernel": "sample", "bound": "hbm", "achieved": samp_bytes / (samp_ms / 1e3) / 1e9,
+        roof = {"kernel": "sample", "bound": "hbm", "achieved": st["samp_bytes"] / (st["samp_ms"] / 1e3) / 1e9,
                 "peak": hbm_peak, "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["peak_source"] = peak_kind
     roof["traffic"] = _recorded_traffic(roof["kernel"], w.name)
+    samp_roof = {"kernel": "sample", "bound": "hbm", "achieved": head["sampler_hbm_gbs_cold_l2"], "peak": hbm_peak,
+                 "unit": "GB/s", "frac": head["sampler_frac_cold_l2"], "peak_source": peak_kind,
+                 "timing": "sampler alone, L2 flushed before every rep", "traffic": _recorded_traffic("sample", w.name)}
 
     line = {
-        "metric": _metric(w), "value": value, "unit": "rows/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "metric": METRIC, "value": head["rows_per_s"], "unit": "rows/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": head["step_ms"], "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": _config(w),
-        "roofline": roof,
-        "kernels": {
-            "logits_local_ms": gemm_ms, "sample_ms": samp_ms, "sample_cold_l2_ms": samp_cold_ms,
-            "gemm_tflops": gemm_flops / (gemm_ms / 1e3) / 1e12,
-            "gemm_hbm_gbs": gemm_bytes / (gemm_ms / 1e3) / 1e9,
-            "sampler_rows_per_s": w.R / (samp_ms / 1e3),
-            "sampler_hbm_gbs_cold_l2": samp_bytes / (samp_cold_ms / 1e3) / 1e9,
-            "sampler_hbm_gbs_in_step": samp_bytes / (samp_ms / 1e3) / 1e9,
-        },
-        "e2e": {"value": e2e_value, "unit": "rows/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "roofline": roof, "sampler_roofline": samp_roof,
+        "kernels": {"logits_local_ms": st["gemm_ms"], "sample_ms": st["samp_ms"],
+                    "sample_cold_l2_ms": head["sample_ms_cold_l2"], "gemm_tflops": head["gemm_tflops"],
+                    "sampler_hbm_gbs_cold_l2": head["sampler_hbm_gbs_cold_l2"]},
+        "e2e": {"value": head["e2e_rows_per_s"], "unit": "rows/s", "h2d_bytes_per_step": st["h2d"],
+                "d2h_bytes_per_step": st["d2h"]},
         "gpu_launches": (1 + vsl.sample_launches(w.R, w.S, w.V_s)) * args.steps,  # projection + sampler kernels
-        "clocks": clk,
-        "cpu_baseline": None,
+        "clocks": clk, "per_config": per_config, "cpu_baseline": None, "parity": None,
     }
-    if rank == 0 and world == 1 and not args.skip_cpu:
-        secs, rows, threads = cpu_oracle_rows(w, args.cpu_rows)
-        line["cpu_baseline"] = {"value": rows / secs, "unit": "rows/s", "cores": threads, "kind": "oracle",
-                                "sample": f"{rows} rows of the {w.name} workload: float64 projection of those rows "
-                                          f"over all {w.V} tokens + the sampler oracle ({secs:.1f} s)"}
+    if logits_host is not None:
+        params = (st["T"], st["k"], st["p"], st["req"], st["pos"])
+        line["cpu_baseline"], line["parity"] = oracle_baseline(
+            logits_host, params, PARITY_SEED, w.n_logprobs,
+            f"the {w.name} workload's projection output (R={w.R}, V={w.V})", gpu_tokens=gpu_tokens,
+            budget_s=args.cpu_seconds)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -437,7 +532,7 @@ def run_gpu(args, w):
 
 def run_sampler_only(args, w):
     """Times ``sample`` alone on the workload's synthetic fp32 logits (the recipe of
-    the parity tests), L2 flushed before every rep; prints one JSON line."""
+    the parity tests), L2 flushed before every rep, clocks sampled; one JSON line."""
     import vocab_sharded_logits_b200 as vsl
     dev = torch.device("cuda", 0)
     hbm_peak, _, _, peak_kind = _peaks()
@@ -450,15 +545,23 @@ def run_sampler_only(args, w):
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
     for i in range(args.warmup):
         vsl.sample(slices, params, i, w.n_logprobs, out=out)
+    clocks = ClockSampler(0)
+    clocks.start()
     times = []
-    for i in range(args.steps):
+    t_start = time.time()
+    i = 0
+    while i < args.steps or (clocks.proc is not None and clocks.count() - clocks.skip < 3
+                             and time.time() - t_start < 10):
         flush.fill_(float(i))
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0, e1 = _events(2)
         e0.record()
         vsl.sample(slices, params, 100 + i, w.n_logprobs, out=out)
         e1.record()
         torch.cuda.synchronize()
-        times.append(e0.elapsed_time(e1))
+        if i < args.steps:
+            times.append(e0.elapsed_time(e1))
+        i += 1
+    clk = clocks.stop()
     ms = statistics.median(times)
     nbytes = w.R * w.V * 4
     print(json.dumps({"metric": f"sampler rows/sec ({w.name}, V={w.V}, L2 flushed)", "value": w.R / (ms / 1e3),
@@ -466,6 +569,7 @@ def run_sampler_only(args, w):
                       "roofline": {"bound": "hbm", "achieved": nbytes / (ms / 1e3) / 1e9, "peak": hbm_peak,
                                    "unit": "GB/s", "frac": nbytes / (ms / 1e3) / 1e9 / hbm_peak,
                                    "peak_source": peak_kind},
+                      "clocks": clk,
                       "config": {"workload": w.name, "rows": w.R, "vocab": w.V, "slices": w.S}}), flush=True)
     return 0
 
@@ -476,10 +580,11 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["vsl", "reference"], default="vsl")
-    ap.add_argument("--workload", default="decode", choices=sorted(W.WORKLOADS))
-    ap.add_argument("--cpu-rows", type=int, default=4)
-    ap.add_argument("--reference-rows", type=int, default=2)
+    ap.add_argument("--workload", default="large", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--reference-rows", type=int, default=2, help="oracle arm: rows per worker process per step")
+    ap.add_argument("--cpu-seconds", type=float, default=2.0, help="cpu_baseline: seconds per timed oracle run")
     ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true", help="measure the headline workload only")
     ap.add_argument("--sampler-only", action="store_true",
                     help="time the sampler alone on the workload's synthetic logits (profiling aid)")
     args = ap.parse_args()

@@ -21,12 +21,14 @@
  *   - The caller owns every buffer.  "device" pointers are CUDA device
  *     memory of the current device; "host" arrays are ordinary host memory
  *     read during the call only.  The library never allocates device
- *     memory and never synchronises the stream.  vsl_sample keeps, per
- *     device, one side stream and two events (created on first use, kept
- *     for the process) for the kernels it runs side by side; its calls are
- *     serialised by a lock around their launches, and they can be captured
- *     into a CUDA graph (the side stream joins the capture through the
- *     events).
+ *     memory and never synchronises the stream.  Per device the library
+ *     keeps its kernels' launch attributes, the SM count and the largest
+ *     cluster the device schedules (read once, on the first call made with
+ *     that device current), and vsl_sample keeps one side stream and two
+ *     events (created on the first call that runs its kernels side by side,
+ *     kept for the process); the side-by-side launches of one device are
+ *     serialised by a lock, and they can be captured into a CUDA graph (the
+ *     side stream joins the capture through the events).
  *   - stream is a cudaStream_t (NULL = legacy default stream).  Work is
  *     enqueued asynchronously; host-side argument errors are returned before
  *     anything is enqueued, launch errors as VSL_ERR_CUDA.
@@ -181,6 +183,31 @@ VSL_API vsl_status vsl_sample(const float* const* logits_slices, int32_t R, int3
                       int32_t* token_ids, float* token_logprob, int32_t* topn_ids,
                       float* topn_logprob, uint32_t* row_flags, void* workspace,
                       size_t workspace_bytes, void* stream);
+
+/* Optional outputs of vsl_sample_ex (every pointer may be NULL: not written).
+ *   kept_theta : device fp32 [R][2], 8-byte aligned.  Row r gets
+ *                (theta_k, theta_p), the two thresholds on x = fl(logit / T)
+ *                the draw used: theta_k the top_k-th largest x (counted with
+ *                multiplicity), theta_p the smallest x the top-p rule keeps
+ *                among the top-k survivors; -inf for a rule that is off (top_k
+ *                0 or >= S * V_s, top_p >= 1) and NaN for a greedy or a
+ *                flagged row.  The kept set the token is drawn from is exactly
+ *                { i : x_i finite and x_i >= max(theta_k, theta_p) }.
+ * Source: "Qwen4Exp batch-sharded sampling: inside vLLM PR #61018"
+ * (orcarouter.ai blog), section "batch-sharded sampling in one paragraph": the
+ * sampler's top-k and top-p work per request. */
+typedef struct {
+  float* kept_theta;
+} vsl_sample_extras;
+
+/* vsl_sample_ex - vsl_sample with optional outputs (extras may be NULL, which
+ * is vsl_sample).  Same arguments, ownership and errors as vsl_sample, plus
+ * VSL_ERR_ALIGNMENT for a kept_theta that is not 8-byte aligned. */
+VSL_API vsl_status vsl_sample_ex(const float* const* logits_slices, int32_t R, int32_t S, int32_t V_s,
+                         const vsl_row_params* params_dev, uint64_t seed, int32_t n_logprobs,
+                         int32_t* token_ids, float* token_logprob, int32_t* topn_ids,
+                         float* topn_logprob, uint32_t* row_flags, void* workspace,
+                         size_t workspace_bytes, const vsl_sample_extras* extras, void* stream);
 
 /* Reads and clears the device error word the kernels set when a bounded wait
  * gives up (a bug, never expected).  Synchronises the current device.

@@ -1,4 +1,6 @@
 """Shared checks of the CUDA sampler against the oracle, row by row."""
+import os
+
 import numpy as np
 import torch
 
@@ -8,13 +10,17 @@ from oracle import sampler as S
 LOGPROB_TOL = 1e-4      # raw logprobs: fp32 online log-sum-exp vs float64
 LOGIT_TOL = 2e-2        # projection: bf16 inputs, fp32 accumulation vs float64
 
+# per-test counts of the allowed exceptions, printed in pytest's terminal summary
+REPORT = []
+
 
 def run_sampler(logits, params_np, seed, n, S_slices, device):
-    """Runs the CUDA sampler on [R, V] fp32 logits split into S_slices slices."""
+    """Runs the CUDA sampler on [R, V] fp32 logits split into S_slices slices,
+    with the kept-set thresholds requested."""
     T, k, p, req, pos = params_np
     slices = [t.contiguous() for t in torch.tensor_split(logits.to(device), S_slices, dim=1)]
     prm = vsl.make_row_params(T, k, p, req, pos, device)
-    out = vsl.sample(slices, prm, seed, n)
+    out = vsl.sample(slices, prm, seed, n, kept_theta=True)
     torch.cuda.synchronize()
     return {
         "token": out.token_ids.cpu().numpy(),
@@ -22,20 +28,30 @@ def run_sampler(logits, params_np, seed, n, S_slices, device):
         "topn_ids": out.topn_ids.cpu().numpy(),
         "topn_lp": out.topn_logprob.cpu().numpy(),
         "flags": out.row_flags.cpu().numpy().astype(np.uint32),
+        "theta": out.kept_theta.cpu().numpy(),
     }
 
 
+def _expected_theta(v):
+    return np.float32(-np.inf) if v is None else np.float32(v)
+
+
 def compare(gpu, logits_np, params_np, seed, n, rows):
-    """Element-by-element comparison on ``rows``; returns counts of the
-    allowed exceptions (near-ties of the draw, cut-ties of top-p)."""
+    """Element-by-element comparison on ``rows``: flags, top-n ids (exact) and
+    logprobs (1e-4), the kept-set thresholds theta_k and theta_p (bit-exact) and
+    the kept set they define (every element), and the token (exact).  Returns
+    counts of the allowed exceptions: near-ties of the draw (the token only) and
+    cut-ties of top-p (theta_p, the kept set and the token)."""
     T, k, p, req, pos = params_np
-    stats = {"rows": 0, "near_tie": 0, "cut_tie": 0, "mismatch_allowed": 0}
+    stats = {"rows": 0, "near_tie": 0, "cut_tie": 0, "mismatch_allowed": 0, "kept_checked": 0}
     for r in rows:
         o = S.sample_row(logits_np[r], T[r], int(k[r]), p[r], int(req[r]), int(pos[r]), seed, n)
         stats["rows"] += 1
+        th = gpu["theta"][r]
         assert int(gpu["flags"][r]) == o.flags, (r, gpu["flags"][r], o.flags)
         if o.flags:
             assert gpu["token"][r] == -1 and np.isnan(gpu["token_lp"][r])
+            assert np.isnan(th).all(), (r, th)
             if n:
                 assert np.all(gpu["topn_ids"][r] == -1)
             continue
@@ -44,6 +60,17 @@ def compare(gpu, logits_np, params_np, seed, n, rows):
             assert np.allclose(gpu["topn_lp"][r], o.topn_logprob, atol=LOGPROB_TOL, rtol=0), r
         stats["near_tie"] += int(o.near_tie)
         stats["cut_tie"] += int(o.cut_tie)
+        if np.float32(T[r]) == 0:
+            assert np.isnan(th).all(), (r, th)          # greedy: no kept set
+        else:
+            assert th[0] == _expected_theta(o.theta_k), (r, "theta_k", th[0], o.theta_k)
+            if not o.cut_tie:
+                assert th[1] == _expected_theta(o.theta_p), (r, "theta_p", th[1], o.theta_p)
+                l = logits_np[r]
+                x = S.scale(l, T[r])
+                kept = np.isfinite(l) & (x >= max(th[0], th[1]))
+                assert np.array_equal(kept, o.kept), (r, int(kept.sum()), int(o.kept.sum()))
+                stats["kept_checked"] += 1
         tok = int(gpu["token"][r])
         if tok != o.token:
             assert o.near_tie or o.cut_tie, (r, tok, o.token, o.score_gap, o.cut_margin)
@@ -53,4 +80,5 @@ def compare(gpu, logits_np, params_np, seed, n, rows):
                 assert o.kept[tok]
         ref_lp = S.log_softmax(logits_np[r])[tok]
         assert abs(float(gpu["token_lp"][r]) - ref_lp) <= LOGPROB_TOL, (r, gpu["token_lp"][r], ref_lp)
+    REPORT.append((os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0], dict(stats)))
     return stats

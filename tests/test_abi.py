@@ -70,6 +70,11 @@ def test_host_validation_rejects_bad_arguments_without_a_device():
     assert L.vsl_sample(*args(S=17)) == 3
     assert L.vsl_sample(*args(V_s=1 << 20, S=1)) == 3         # beyond the largest vocabulary
     assert L.vsl_sample_workspace_bytes(2048, 8, 18992, 20) == 0
+    # vsl_sample_ex: the same checks, plus the optional outputs' alignment
+    ex = lambda extras, **kw: L.vsl_sample_ex(*args(**kw)[:-1], extras, None)
+    assert ex(None, R=0) == 1
+    assert ex(ctypes.byref(v._Extras(0x10004)), V_s=512) == 2         # kept_theta not 8-byte aligned
+    assert ex(ctypes.byref(v._Extras(0x10008)), V_s=1 << 20) == 3     # aligned: the size check follows
 
 
 def test_binding_has_no_cpu_fallback(monkeypatch, tmp_path):

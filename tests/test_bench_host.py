@@ -55,6 +55,7 @@ def test_reference_arm_prints_one_json_line():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["unit"] == "rows/s" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0
+    assert d["cpu_baseline"]["nproc"] >= 1 and "cpu_model" in d["cpu_baseline"]
 
 
 @pytest.mark.parametrize("R,H,n", [(64, 4096, 20), (4, 64, 5), (7, 24, 0)])
@@ -111,13 +112,57 @@ def test_clock_sampler_reads_clocks_and_throttle_reasons(tmp_path):
     assert got == {"sm_mhz": 1950.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
 
 
-def test_recorded_traffic_needs_the_sources_it_was_captured_from(monkeypatch):
+def test_recorded_traffic_needs_the_sources_it_was_captured_from(monkeypatch, tmp_path):
     """A profile's DRAM bytes are used only while the kernel's sources hash to
     the value recorded beside them."""
     sys.path.insert(0, ROOT)
     import bench
-    got = bench._recorded_traffic("logits_local_kernel", "decode")
-    assert isinstance(got, int) and got > 0
+    (tmp_path / "logits_local_kernel_decode.md").write_text(
+        "# capture\n"
+        f"source_sha256: {bench._source_sha('logits_local_kernel')}\n"
+        "traffic_bytes_per_launch: 1253643368\n")
+    got = bench._recorded_traffic("logits_local_kernel", "decode", str(tmp_path))
+    assert got == 1253643368
     monkeypatch.setattr(bench, "_source_sha", lambda kernel: "0" * 64)
-    assert bench._recorded_traffic("logits_local_kernel", "decode") is None
-    assert bench._recorded_traffic("logits_local_kernel", "no_such_workload") is None
+    assert bench._recorded_traffic("logits_local_kernel", "decode", str(tmp_path)) is None
+    assert bench._recorded_traffic("logits_local_kernel", "no_such_workload", str(tmp_path)) is None
+
+
+def test_reference_arm_loads_no_repository_library():
+    """The oracle arm imports neither the binding nor libvsl.so: its process maps
+    no shared object of this repository."""
+    code = ("import sys, runpy; sys.argv = ['bench.py', '--impl', 'reference', '--workload', 'tiny', '--steps', '1', "
+            "'--warmup', '0', '--reference-rows', '1']\n"
+            "try:\n    runpy.run_path('bench.py', run_name='__main__')\n"
+            "except SystemExit as e:\n    assert not e.code, e.code\n"
+            "maps = open('/proc/self/maps').read()\n"
+            "print('checked')\n"
+            "assert 'libvsl' not in maps, 'libvsl mapped'\n"
+            "assert 'vocab_sharded_logits_b200' not in sys.modules\n")
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert out.returncode == 0, out.stderr
+    assert "checked" in out.stdout
+
+
+def test_oracle_timing_harness_matches_the_oracle_on_every_row():
+    """The baseline's worker processes run the oracle itself: their tokens equal
+    sample_row's on the same rows, in one process and split over workers."""
+    import numpy as np
+    sys.path.insert(0, ROOT)
+    import workloads as W
+    from oracle.sampler import sample_row
+    from oracle.timing import OracleSampler
+    w = W.scaled(W.WORKLOADS["decode"], V=4096, requests=6)
+    logits = W.sampler_logits(w, "cpu").numpy()
+    T, k, p, req, pos = W.row_params(w)
+    want = [sample_row(logits[r], T[r], int(k[r]), p[r], int(req[r]), int(pos[r]), 5, w.n_logprobs).token
+            for r in range(w.R)]
+    orc = OracleSampler(logits, (T, k, p, req, pos), 5, w.n_logprobs, workers=2)
+    try:
+        _, one = orc.run(range(w.R), parallel=False)
+        orc.start_workers()
+        _, many = orc.run(range(w.R), parallel=True)
+    finally:
+        orc.close()
+    assert [t for _, t, _, _, _ in sorted(one)] == want
+    assert [t for _, t, _, _, _ in sorted(many)] == want

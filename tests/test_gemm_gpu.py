@@ -8,7 +8,7 @@ import torch
 
 import vocab_sharded_logits_b200 as vsl
 from oracle.gemm import logits_local as ref_logits, logits_local_entries
-from vocab_sharded_logits_b200 import workloads as W
+import workloads as W
 from parity_helpers import LOGIT_TOL
 
 pytestmark = pytest.mark.gpu

@@ -6,7 +6,7 @@ import pytest
 import torch
 
 import vocab_sharded_logits_b200 as vsl
-from vocab_sharded_logits_b200 import workloads as W
+import workloads as W
 from parity_helpers import compare, run_sampler
 
 pytestmark = pytest.mark.gpu
@@ -40,6 +40,25 @@ def test_full_size_configs_sampled_rows(cuda_device, name, nrows):
     rows = np.random.default_rng(5).choice(w.R, min(nrows, w.R), replace=False)
     st, _ = _case(w, cuda_device, rows=sorted(rows.tolist()))
     assert st["rows"] == len(rows)
+
+
+def test_peaked_full_size_seed_sweep(cuda_device):
+    """The peaked / long-tail configuration at full size, draw seeds 0..15: the
+    whole batch sampled per seed, 12 rows per seed compared with the oracle
+    (tokens, kept sets, thresholds, top-n)."""
+    w = W.WORKLOADS["peaked"]
+    logits = W.sampler_logits(w, cuda_device)
+    params = W.row_params(w)
+    logits_np = logits.cpu().numpy()
+    total = {"rows": 0, "mismatch_allowed": 0}
+    for seed in range(16):
+        gpu = run_sampler(logits, params, seed, w.n_logprobs, w.S, cuda_device)
+        rows = sorted(np.random.default_rng(100 + seed).choice(w.R, 12, replace=False).tolist())
+        st = compare(gpu, logits_np, params, seed, w.n_logprobs, rows)
+        total["rows"] += st["rows"]
+        total["mismatch_allowed"] += st["mismatch_allowed"]
+    assert total["rows"] == 16 * 12
+    assert total["mismatch_allowed"] <= 4
 
 
 @pytest.mark.parametrize("S", [1, 2, 4, 8])

@@ -33,9 +33,15 @@ _STATUS_NAMES = {0: "VSL_OK", 1: "VSL_ERR_INVALID_ARG", 2: "VSL_ERR_ALIGNMENT", 
 
 
 class VslError(RuntimeError):
+    """A libvsl call returned a status other than VSL_OK (``status`` is the code)."""
+
     def __init__(self, status, where):
         self.status = status
         super().__init__(f"{where}: {_STATUS_NAMES.get(status, status)} ({status_string(status)})")
+
+
+class _Extras(ctypes.Structure):
+    _fields_ = [("kept_theta", ctypes.c_void_p)]
 
 
 class _Plan(ctypes.Structure):
@@ -59,6 +65,9 @@ def _load():
     l.vsl_sample_plan_for.argtypes = [i32, i32, i32, i32, i32, ctypes.POINTER(_Plan)]
     l.vsl_sample.restype = ctypes.c_int
     l.vsl_sample.argtypes = [ctypes.POINTER(vp), i32, i32, i32, vp, u64, i32, vp, vp, vp, vp, vp, vp, sz, vp]
+    l.vsl_sample_ex.restype = ctypes.c_int
+    l.vsl_sample_ex.argtypes = [ctypes.POINTER(vp), i32, i32, i32, vp, u64, i32, vp, vp, vp, vp, vp, vp, sz,
+                                ctypes.POINTER(_Extras), vp]
     l.vsl_device_error.restype = ctypes.c_int
     l.vsl_device_error.argtypes = [ctypes.POINTER(u32)]
     l.vsl_status_string.restype = ctypes.c_char_p
@@ -96,6 +105,13 @@ def _check(status, where):
         raise VslError(status, where)
 
 
+def _on_device(device):
+    """The library launches on the current device: make the tensors' device current."""
+    if device.type != "cuda":
+        raise ValueError(f"libvsl needs CUDA tensors, got a tensor on {device}")
+    return torch.cuda.device(device)
+
+
 def logits_local(hidden, w_slices, out=None, stream=None):
     """Vocab-slice projection with no gather: ``out[s] = hidden @ w_slices[s].T`` in fp32.
 
@@ -112,8 +128,12 @@ def logits_local(hidden, w_slices, out=None, stream=None):
             raise ValueError("logits_local needs contiguous tensors")
     if hidden.dtype != torch.bfloat16 or any(w.dtype != torch.bfloat16 for w in w_slices):
         raise TypeError("hidden and weights must be bfloat16")
-    status = lib.vsl_logits_local(_ptr(hidden), _ptr_array(w_slices), _ptr_array(out), R, H, S, V_s,
-                                  _stream_handle(stream, hidden.device))
+    for t in [*w_slices, *out]:
+        if t.device != hidden.device:
+            raise ValueError("logits_local: every tensor must be on the hidden states' device")
+    with _on_device(hidden.device):
+        status = lib.vsl_logits_local(_ptr(hidden), _ptr_array(w_slices), _ptr_array(out), R, H, S, V_s,
+                                      _stream_handle(stream, hidden.device))
     _check(status, "vsl_logits_local")
     return out
 
@@ -141,28 +161,33 @@ def _u32_to_i32(x):
 
 
 class SampleResult:
-    """Outputs of ``sample``: token ids, their raw logprobs, top-n ids / logprobs, row flags."""
+    """Outputs of ``sample``: token ids, their raw logprobs, top-n ids / logprobs, row
+    flags, and (when asked for) the kept-set thresholds ``kept_theta`` [R, 2]."""
 
-    def __init__(self, token_ids, token_logprob, topn_ids, topn_logprob, row_flags):
+    def __init__(self, token_ids, token_logprob, topn_ids, topn_logprob, row_flags, kept_theta=None):
         self.token_ids = token_ids
         self.token_logprob = token_logprob
         self.topn_ids = topn_ids
         self.topn_logprob = topn_logprob
         self.row_flags = row_flags
+        self.kept_theta = kept_theta
 
 
-def sample(logits_slices, params, seed, n_logprobs, out=None, stream=None):
+def sample(logits_slices, params, seed, n_logprobs, out=None, stream=None, kept_theta=False):
     """Per-row temperature / top-k / top-p / Gumbel-max draw / top-n raw logprobs.
 
     logits_slices: list of fp32 [R, V_s] CUDA tensors (row r = concatenation over slices).
     params: int32 [R, 5] CUDA tensor from ``make_row_params``.
+    kept_theta: also return each row's (theta_k, theta_p) on x = fl(l / T) (fp32 [R, 2]):
+    the draw's kept set is every finite x >= max(theta_k, theta_p); -inf for a rule
+    that is off, NaN for greedy and flagged rows.
     """
     R, V_s = logits_slices[0].shape
     S = len(logits_slices)
     dev = logits_slices[0].device
     for t in logits_slices:
-        if t.dtype != torch.float32 or not t.is_contiguous() or tuple(t.shape) != (R, V_s):
-            raise ValueError("logits slices must be contiguous fp32 [R, V_s]")
+        if t.dtype != torch.float32 or not t.is_contiguous() or tuple(t.shape) != (R, V_s) or t.device != dev:
+            raise ValueError("logits slices must be contiguous fp32 [R, V_s] on one device")
     if params.dtype != torch.int32 or tuple(params.shape) != (R, 5) or not params.is_contiguous():
         raise ValueError("params must be a contiguous int32 [R, 5] tensor (make_row_params)")
     if out is None:
@@ -172,13 +197,26 @@ def sample(logits_slices, params, seed, n_logprobs, out=None, stream=None):
                            torch.empty(R, n, dtype=torch.int32, device=dev)[:, :n_logprobs],
                            torch.empty(R, n, dtype=torch.float32, device=dev)[:, :n_logprobs],
                            torch.empty(R, dtype=torch.int32, device=dev))
+    if params.device != dev:
+        raise ValueError("params must be on the logits' device")
+    if kept_theta and out.kept_theta is None:
+        out.kept_theta = torch.empty(R, 2, dtype=torch.float32, device=dev)
+    extras = None
+    if kept_theta:
+        if out.kept_theta.dtype != torch.float32 or tuple(out.kept_theta.shape) != (R, 2) or \
+                not out.kept_theta.is_contiguous():
+            raise ValueError("kept_theta must be a contiguous fp32 [R, 2] tensor")
+        extras = _Extras(out.kept_theta.data_ptr())
     ws_bytes = lib.vsl_sample_workspace_bytes(R, S, V_s, n_logprobs)
-    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev) if ws_bytes else None
-    topn_ids = out.topn_ids if n_logprobs > 0 else None
-    topn_lp = out.topn_logprob if n_logprobs > 0 else None
-    status = lib.vsl_sample(_ptr_array(logits_slices), R, S, V_s, _ptr(params), ctypes.c_uint64(seed & (2 ** 64 - 1)),
-                            n_logprobs, _ptr(out.token_ids), _ptr(out.token_logprob), _ptr(topn_ids),
-                            _ptr(topn_lp), _ptr(out.row_flags), _ptr(ws), ws_bytes, _stream_handle(stream, dev))
+    with _on_device(dev):
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev) if ws_bytes else None
+        topn_ids = out.topn_ids if n_logprobs > 0 else None
+        topn_lp = out.topn_logprob if n_logprobs > 0 else None
+        status = lib.vsl_sample_ex(_ptr_array(logits_slices), R, S, V_s, _ptr(params),
+                                   ctypes.c_uint64(seed & (2 ** 64 - 1)), n_logprobs, _ptr(out.token_ids),
+                                   _ptr(out.token_logprob), _ptr(topn_ids), _ptr(topn_lp), _ptr(out.row_flags),
+                                   _ptr(ws), ws_bytes, ctypes.byref(extras) if extras is not None else None,
+                                   _stream_handle(stream, dev))
     _check(status, "vsl_sample")
     return out
 
@@ -187,7 +225,7 @@ def sample_launches(R, S, V_s):
     """Kernels one ``sample`` call with these sizes launches on the current device."""
     n = lib.vsl_sample_launches(int(R), int(S), int(V_s))
     if n < 0:
-        raise VslError(f"vsl_sample_launches: sizes rejected (R={R}, S={S}, V_s={V_s})")
+        raise ValueError(f"vsl_sample_launches: sizes rejected (R={R}, S={S}, V_s={V_s})")
     return n
 
 

@@ -79,10 +79,10 @@ vsl_status vsl_sample_plan_for(int32_t R, int32_t S, int32_t V_s, int32_t sms, i
   return VSL_OK;
 }
 
-vsl_status vsl_sample(const float* const* logits_slices, int32_t R, int32_t S, int32_t V_s,
-                      const vsl_row_params* params_dev, uint64_t seed, int32_t n_logprobs, int32_t* token_ids,
-                      float* token_logprob, int32_t* topn_ids, float* topn_logprob, uint32_t* row_flags,
-                      void* workspace, size_t workspace_bytes, void* stream) {
+vsl_status vsl_sample_ex(const float* const* logits_slices, int32_t R, int32_t S, int32_t V_s,
+                         const vsl_row_params* params_dev, uint64_t seed, int32_t n_logprobs, int32_t* token_ids,
+                         float* token_logprob, int32_t* topn_ids, float* topn_logprob, uint32_t* row_flags,
+                         void* workspace, size_t workspace_bytes, const vsl_sample_extras* extras, void* stream) {
   (void)workspace;
   if (logits_slices == nullptr || params_dev == nullptr || token_ids == nullptr || token_logprob == nullptr ||
       row_flags == nullptr)
@@ -97,13 +97,25 @@ vsl_status vsl_sample(const float* const* logits_slices, int32_t R, int32_t S, i
     if (logits_slices[s] == nullptr) return VSL_ERR_INVALID_ARG;
     if (!vsl::aligned16(logits_slices[s])) return VSL_ERR_ALIGNMENT;
   }
-  int c = 0, part = 0;
-  if (!vsl::sample_geometry(V, &c, &part) || V > 0x7FFFFFFFLL) return VSL_ERR_UNSUPPORTED;
+  float* kept_theta = extras != nullptr ? extras->kept_theta : nullptr;
+  if (kept_theta != nullptr && (reinterpret_cast<uintptr_t>(kept_theta) & 7u) != 0) return VSL_ERR_ALIGNMENT;
+  if (V > vsl::sample_max_vocab()) return VSL_ERR_UNSUPPORTED;
+  int maxc = 0, c = 0, part = 0;
+  if (vsl::sample_max_cluster(&maxc) != cudaSuccess) return VSL_ERR_CUDA;
+  if (!vsl::sample_geometry_for(V, maxc, &c, &part)) return VSL_ERR_UNSUPPORTED;
   if (workspace_bytes < vsl_sample_workspace_bytes(R, S, V_s, n_logprobs)) return VSL_ERR_WORKSPACE_TOO_SMALL;
   const cudaError_t e = vsl::launch_sample(logits_slices, R, S, V_s, params_dev, seed, n_logprobs, token_ids,
-                                           token_logprob, topn_ids, topn_logprob, row_flags,
+                                           token_logprob, topn_ids, topn_logprob, row_flags, kept_theta,
                                            static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? VSL_OK : VSL_ERR_CUDA;
+}
+
+vsl_status vsl_sample(const float* const* logits_slices, int32_t R, int32_t S, int32_t V_s,
+                      const vsl_row_params* params_dev, uint64_t seed, int32_t n_logprobs, int32_t* token_ids,
+                      float* token_logprob, int32_t* topn_ids, float* topn_logprob, uint32_t* row_flags,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+  return vsl_sample_ex(logits_slices, R, S, V_s, params_dev, seed, n_logprobs, token_ids, token_logprob, topn_ids,
+                       topn_logprob, row_flags, workspace, workspace_bytes, nullptr, stream);
 }
 
 vsl_status vsl_device_error(uint32_t* code_out) {

@@ -246,12 +246,18 @@ cudaError_t launch_bn(GemmArgs& args, const void* hidden, const void* const* w, 
   args.w_evict_first = args.n_tiles == 1;
   constexpr size_t smem = gemm_smem_bytes<BN, STAGES>();
   auto kern = logits_local_kernel<BN, STAGES>;
-  static bool attr_set = false;  // per template instance; idempotent if raced
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  // the shared-memory attribute is per device: set once on each, with it current
+  constexpr int kMaxDevices = 64;
+  static std::once_flag once[kMaxDevices];
+  static cudaError_t attr_status[kMaxDevices];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::call_once(once[dev], [&] {
+    attr_status[dev] = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  });
+  if (attr_status[dev] != cudaSuccess) return attr_status[dev];
   const long long grid = static_cast<long long>(S) * args.m_tiles * args.n_tiles;
   if (grid > 0x7FFFFFFF) return cudaErrorInvalidConfiguration;
   kern<<<static_cast<unsigned>(grid), kGemmThreads, smem, stream>>>(args);

@@ -21,11 +21,17 @@ cudaError_t launch_logits_local(const void* hidden, const void* const* w_slices,
 cudaError_t launch_sample(const float* const* logits, int R, int S, int V_s,
                           const vsl_row_params* params, uint64_t seed, int n_logprobs,
                           int32_t* token_ids, float* token_logprob, int32_t* topn_ids,
-                          float* topn_logprob, uint32_t* row_flags, cudaStream_t stream);
+                          float* topn_logprob, uint32_t* row_flags, float* kept_theta, cudaStream_t stream);
 
-// Sampler launch geometry for a vocabulary of V tokens: CTAs per row (cluster
-// size) and elements per CTA.  Returns false if V cannot be handled.
-bool sample_geometry(long long V, int* cluster, int* part);
+// Sampler launch geometry for a vocabulary of V tokens on a device that
+// schedules clusters of at most maxc CTAs: CTAs per row (cluster size) and
+// elements per CTA.  Returns false if V cannot be handled.
+bool sample_geometry_for(long long V, int maxc, int* cluster, int* part);
+// Largest vocabulary the sampler handles on any device (host only).
+long long sample_max_vocab();
+// Largest cluster the current device schedules for the cluster kernel (the
+// device's launch state is prepared on first use).
+cudaError_t sample_max_cluster(int* maxc);
 int sample_launches(int R, long long V);
 bool sample_plan(int R, long long V, int sms, int maxc, vsl_sample_plan* out);
 

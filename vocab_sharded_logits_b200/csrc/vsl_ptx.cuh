@@ -19,6 +19,7 @@ enum : uint32_t {
   kErrGemmEpilogue = 1u << 2,
   kErrSampleLoad = 1u << 8,
   kErrSampleList = 1u << 9,
+  kErrWaitProbe = 1u << 16,  // the test library's wait probe (never set by the product kernels)
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -50,14 +51,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Returns false if the phase did not complete within kWaitLimitCycles.
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+// Returns false if the phase did not complete within `limit` SM clock cycles.
+__device__ __forceinline__ bool mbar_wait_bounded_for(uint32_t bar, uint32_t parity, long long limit) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > kWaitLimitCycles) return false;
+    if (clock64() - t0 > limit) return false;
   }
   return true;
+}
+// Returns false if the phase did not complete within kWaitLimitCycles.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+  return mbar_wait_bounded_for(bar, parity, kWaitLimitCycles);
 }
 
 // ---------------------------------------------------------------- TMA / bulk copies

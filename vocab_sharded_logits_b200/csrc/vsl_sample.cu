@@ -115,6 +115,7 @@ struct SampleArgs {
   int32_t* topn_ids;
   float* topn_logprob;
   uint32_t* row_flags;
+  float* kept_theta;  // optional [R][2]: theta_k, theta_p of each row (nullptr: not written)
   uint32_t* err;
   unsigned long long seed;
   int R, S, V_s, V, C, part, n_logprobs;
@@ -203,6 +204,7 @@ struct __align__(16) SharedHeader {
   BestSlot best[kMaxCluster];
   double ex_above[kMaxCluster];    // leader only: EXACT sums pushed by every CTA
   double ex_below[kMaxCluster];
+  float ex_xmin[kMaxCluster];      // leader only: EXACT's smallest x above the window, per CTA
   double win_lo[kMaxCluster];      // every CTA: each slice's lower / upper mass bound
   double win_hi[kMaxCluster];
   int32_t win_jlo[kMaxCluster];    // every CTA: each slice's window edges and count
@@ -1212,6 +1214,18 @@ __device__ __forceinline__ double block_sum_d0(double v, SharedHeader* H) {
   return t;
 }
 
+// Block minimum of a float; thread 0 gets it.
+__device__ __forceinline__ float block_min_f0(float v, SharedHeader* H) {
+  v = warp_reduce(v, [](float a, float b) { return fminf(a, b); });
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) H->red_f[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float t = INFINITY;
+  if (threadIdx.x == 0)
+    for (int i = 0; i < kWarps; ++i) t = fminf(t, H->red_f[i]);
+  return t;
+}
+
 // ---- EXACT: with the window of fine bins [lo, hi] that may hold the top-p
 // cut, every finite x above the window is kept for certain (its float64 mass
 // summed, the draw run over it here), every x below it is dropped (mass
@@ -1232,6 +1246,7 @@ __device__ void op_exact(const Ctx& cx, const Plan& p) {
   const double* tab = cx.H->exp_tab;
   const int jlo = static_cast<int>(p.lo), jhi = static_cast<int>(p.hi);
   double above = 0.0, below = 0.0;
+  float xmin_ab = INFINITY;  // smallest x above the window (theta_p when the window keeps nothing)
   // two float4 groups per iteration (q and q + kThreads): their float64 exps
   // and Philox words are independent chains the warp issues interleaved
   const int nq = (cx.n4 + kThreads - 1) / kThreads * kThreads;
@@ -1264,7 +1279,10 @@ __device__ void op_exact(const Ctx& cx, const Plan& p) {
         below += ab[u][i] ? 0.0 : ee;
         any_win[u] |= win[u][i];
         any_ab[u] |= ab[u][i];
-        if (ab[u][i]) xmax[u] = fmaxf(xmax[u], v[u][i]);
+        if (ab[u][i]) {
+          xmax[u] = fmaxf(xmax[u], v[u][i]);
+          xmin_ab = fminf(xmin_ab, v[u][i]);
+        }
       }
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
@@ -1303,9 +1321,11 @@ __device__ void op_exact(const Ctx& cx, const Plan& p) {
   }
   const double ta = block_sum_d0(above, cx.H);
   const double tb = block_sum_d0(below, cx.H);
+  const float tx = block_min_f0(xmin_ab, cx.H);
   if (threadIdx.x == 0) {
     *cluster_ptr(&cx.H->ex_above[cx.rank], 0) = ta;
     *cluster_ptr(&cx.H->ex_below[cx.rank], 0) = tb;
+    *cluster_ptr(&cx.H->ex_xmin[cx.rank], 0) = tx;
   }
   publish_local_list(cx);
   push_best(cx, b);
@@ -1423,12 +1443,24 @@ __device__ void find_mass_bin(const Ctx& cx, int nbins, LeaderState& L) {
   __syncthreads();
 }
 
+// The kept-set thresholds of a row (optional output): theta_k and theta_p on
+// x = fl(l / T); -inf for a rule that is off, NaN for a greedy or flagged row.
+// The draw's kept set is every finite x >= max(theta_k, theta_p).
+__device__ __forceinline__ void write_kept_theta(const SampleArgs& a, int row, float theta_k, float theta_p) {
+  if (a.kept_theta != nullptr) {
+    a.kept_theta[2 * static_cast<size_t>(row)] = theta_k;
+    a.kept_theta[2 * static_cast<size_t>(row) + 1] = theta_p;
+  }
+}
+
 __device__ void write_outputs(const Ctx& cx, LeaderState& L) {
   if (threadIdx.x == 0) {
     const SampleArgs& a = *cx.a;
     a.token_ids[cx.row] = L.token;
     a.token_logprob[cx.row] = L.token_l - L.lse;
     a.row_flags[cx.row] = 0;
+    const float nan = __int_as_float(0x7FC00000);
+    write_kept_theta(a, cx.row, L.greedy ? nan : L.theta_k, L.greedy ? nan : L.theta_p);
   }
 }
 
@@ -1794,8 +1826,13 @@ __device__ void list_resolve_sorted(const Ctx& cx, LeaderState& L, const uint64_
       prev = x;
     }
     const int cut = block_max_i(cand, H);
-    if (cut >= 0) theta = fmaxf(theta, scale_x(key_value(entry_key(buf[cut])), T));
+    if (cut >= 0) {
+      const float theta_p = scale_x(key_value(entry_key(buf[cut])), T);
+      theta = fmaxf(theta, theta_p);
+      if (threadIdx.x == 0) L.theta_p = theta_p;
+    }
   }
+  if (threadIdx.x == 0) L.theta_k = theta_k;
   // the draw over the kept prefix
   Ctx sub = cx;
   sub.list = const_cast<uint64_t*>(buf);
@@ -2215,6 +2252,14 @@ __device__ void exact_tail(const Ctx& cx, LeaderState& L) {
     const int best = block_max_i(cand, H);
     if (best >= 0) theta_p = key_value(entry_key(buf[best]));
   }
+  if (threadIdx.x == 0) {
+    // the kept set's smallest x: the window's cut, else (the window keeps
+    // nothing) the smallest x above the window
+    float t = theta_p;
+    if (!(t < INFINITY))
+      for (uint32_t r = 0; r < cx.C; ++r) t = fminf(t, H->ex_xmin[r]);
+    L.theta_p = t;
+  }
   double sd;
   int32_t id;
   float l;
@@ -2283,6 +2328,7 @@ __device__ bool leader_merge(const Ctx& cx, LeaderState& L, bool topn_now = true
           a.token_ids[cx.row] = -1;
           a.token_logprob[cx.row] = __int_as_float(0x7FC00000);
           a.row_flags[cx.row] = L.flags;
+          write_kept_theta(a, cx.row, __int_as_float(0x7FC00000), __int_as_float(0x7FC00000));
         }
         for (int j = threadIdx.x; j < a.n_logprobs; j += kThreads) {
           a.topn_ids[static_cast<size_t>(cx.row) * a.n_logprobs + j] = -1;
@@ -2847,10 +2893,24 @@ size_t sample_smem_bytes(int part) {
          static_cast<size_t>(part) * 4;
 }
 
-static int g_max_cluster = -1;  // largest cluster size the device schedules for this kernel
+// Per-device launch state: the kernels' attributes are set, and the largest
+// schedulable cluster and the SM count are read, once per device (with that
+// device current); the side stream and its two events are created on the
+// first side-by-side call on the device.
+struct DeviceState {
+  std::once_flag once;
+  cudaError_t status = cudaSuccess;
+  int max_cluster = 8;  // largest cluster size the device schedules for the cluster kernel
+  int sms = 0;
+  std::mutex mu;        // orders the fork / join event pairs of concurrent calls
+  cudaStream_t side = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+constexpr int kMaxDevices = 64;
+static DeviceState g_devices[kMaxDevices];
 
 // The same for a device that schedules clusters of at most maxc CTAs.
-static bool sample_geometry_for(long long V, int maxc, int* cluster, int* part) {
+bool sample_geometry_for(long long V, int maxc, int* cluster, int* part) {
   if (V <= 0 || V > static_cast<long long>(kMaxCluster) * kMaxPart || maxc < 1) return false;
   int c = 1;
   while (c < kMaxCluster && (V + c - 1) / c > kPreferredPart) c <<= 1;
@@ -2863,20 +2923,19 @@ static bool sample_geometry_for(long long V, int maxc, int* cluster, int* part) 
   return true;
 }
 
-bool sample_geometry(long long V, int* cluster, int* part) {
-  return sample_geometry_for(V, g_max_cluster > 0 ? g_max_cluster : 8, cluster, part);
-}
-
-static cudaError_t prepare_sample_kernel() {
-  static bool done = false;
-  if (done) return cudaSuccess;
+static cudaError_t prepare_device(DeviceState& d, int dev) {
   cudaError_t e = cudaFuncSetAttribute(sample_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(sample_smem_bytes(kMaxPart)));
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(sample_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(stream_smem_bytes()));
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
   // largest schedulable cluster at the preferred part size
-  g_max_cluster = 8;
+  d.max_cluster = 8;
   for (int c = kMaxCluster; c >= 8; c >>= 1) {
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(c, 1, 1);
@@ -2891,16 +2950,34 @@ static cudaError_t prepare_sample_kernel() {
     cfg.numAttrs = 1;
     int nclusters = 0;
     if (cudaOccupancyMaxActiveClusters(&nclusters, sample_kernel, &cfg) == cudaSuccess && nclusters > 0) {
-      g_max_cluster = c;
+      d.max_cluster = c;
       break;
     }
     cudaGetLastError();
   }
-  e = cudaFuncSetAttribute(stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(stream_smem_bytes()));
-  if (e != cudaSuccess) return e;
-  done = true;
   return cudaSuccess;
+}
+
+// The current device's state, prepared on first use.
+static cudaError_t current_device_state(DeviceState** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  DeviceState& d = g_devices[dev];
+  std::call_once(d.once, [&] { d.status = prepare_device(d, dev); });
+  if (d.status != cudaSuccess) return d.status;
+  *out = &d;
+  return cudaSuccess;
+}
+
+long long sample_max_vocab() { return static_cast<long long>(kMaxCluster) * kMaxPart; }
+
+cudaError_t sample_max_cluster(int* maxc) {
+  DeviceState* d = nullptr;
+  const cudaError_t e = current_device_state(&d);
+  if (e == cudaSuccess) *maxc = d->max_cluster;
+  return e;
 }
 
 // Streaming kernel geometry: the most CTAs per row (at most 8, a portable
@@ -2960,16 +3037,6 @@ static bool small_batch(int R, long long V, int sms) {
   return sc > 1;
 }
 
-static int device_sms() {
-  static int sms = 0;
-  if (sms == 0) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-  }
-  return sms;
-}
-
 // The launches of one call for R rows of V tokens on a device with `sms` SMs
 // that schedules clusters of at most `maxc` CTAs: the choices launch_sample
 // makes, as plain data.  Returns false if V cannot be handled.
@@ -2992,17 +3059,19 @@ bool sample_plan(int R, long long V, int sms, int maxc, vsl_sample_plan* out) {
 }
 
 int sample_launches(int R, long long V) {
-  if (prepare_sample_kernel() != cudaSuccess) return -1;
-  const int sms = device_sms();
+  DeviceState* d = nullptr;
+  if (current_device_state(&d) != cudaSuccess) return -1;
   vsl_sample_plan p{};
-  if (sms <= 0 || !sample_plan(R, V, sms, g_max_cluster > 0 ? g_max_cluster : 8, &p)) return -1;
+  if (!sample_plan(R, V, d->sms, d->max_cluster, &p)) return -1;
   return p.launches;
 }
 
 cudaError_t launch_sample(const float* const* logits, int R, int S, int V_s, const vsl_row_params* params,
                           uint64_t seed, int n_logprobs, int32_t* token_ids, float* token_logprob,
-                          int32_t* topn_ids, float* topn_logprob, uint32_t* row_flags, cudaStream_t stream) {
-  cudaError_t e = prepare_sample_kernel();
+                          int32_t* topn_ids, float* topn_logprob, uint32_t* row_flags, float* kept_theta,
+                          cudaStream_t stream) {
+  DeviceState* d = nullptr;
+  cudaError_t e = current_device_state(&d);
   if (e != cudaSuccess) return e;
   SampleArgs a{};
   for (int s = 0; s < S; ++s) a.slices[s] = logits[s];
@@ -3012,6 +3081,7 @@ cudaError_t launch_sample(const float* const* logits, int R, int S, int V_s, con
   a.topn_ids = topn_ids;
   a.topn_logprob = topn_logprob;
   a.row_flags = row_flags;
+  a.kept_theta = kept_theta;
   a.err = device_error_word();
   if (a.err == nullptr) return cudaErrorUnknown;
   a.seed = seed;
@@ -3021,9 +3091,8 @@ cudaError_t launch_sample(const float* const* logits, int R, int S, int V_s, con
   a.V = S * V_s;
   a.n_logprobs = n_logprobs;
   int c = 0, part = 0;
-  if (!sample_geometry(a.V, &c, &part)) return cudaErrorInvalidValue;
-  const int sms = device_sms();
-  if (sms <= 0) return cudaErrorInvalidDevice;
+  if (!sample_geometry_for(a.V, d->max_cluster, &c, &part)) return cudaErrorInvalidValue;
+  const int sms = d->sms;
   SampleArgs sa = a;
   stream_geometry(R, a.V, sms, &sa.C, &sa.part);
   a.C = c;
@@ -3044,30 +3113,24 @@ cudaError_t launch_sample(const float* const* logits, int R, int S, int V_s, con
   // kernel samples the rows the streaming kernel could not hold (marked
   // kDeferred).  The cluster kernel's rows take the longest, so it is launched
   // first and with the greatest priority: its CTAs get the SMs first.
-  struct Side {
-    cudaStream_t s = nullptr;
-    cudaEvent_t fork = nullptr, join = nullptr;
-  };
-  static std::mutex mu;
-  static Side sides[64];
-  int dev = 0;
-  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(mu);
-  Side& sd = sides[dev];
-  if (sd.s == nullptr) {
-    if ((e = cudaStreamCreateWithFlags(&sd.s, cudaStreamNonBlocking)) != cudaSuccess) return e;
-    if ((e = cudaEventCreateWithFlags(&sd.fork, cudaEventDisableTiming)) != cudaSuccess) return e;
-    if ((e = cudaEventCreateWithFlags(&sd.join, cudaEventDisableTiming)) != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(d->mu);
+  if (d->side == nullptr) {
+    if ((e = cudaStreamCreateWithFlags(&d->side, cudaStreamNonBlocking)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&d->fork, cudaEventDisableTiming)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&d->join, cudaEventDisableTiming)) != cudaSuccess) return e;
   }
   sa.select = 0;  // the streaming kernel leaves the other rows untouched
   a.select = kSelectOthers;
-  if ((e = cudaEventRecord(sd.fork, stream)) != cudaSuccess) return e;
-  if ((e = cudaStreamWaitEvent(sd.s, sd.fork, 0)) != cudaSuccess) return e;
-  if ((e = launch_with_cluster(fc, a, R * c, sample_smem_bytes(part), stream, true)) != cudaSuccess) return e;
-  if ((e = launch_with_cluster(fs, sa, R * sa.C, stream_smem_bytes(), sd.s)) != cudaSuccess) return e;
-  if ((e = cudaEventRecord(sd.join, sd.s)) != cudaSuccess) return e;
-  if ((e = cudaStreamWaitEvent(stream, sd.join, 0)) != cudaSuccess) return e;
+  if ((e = cudaEventRecord(d->fork, stream)) != cudaSuccess) return e;
+  if ((e = cudaStreamWaitEvent(d->side, d->fork, 0)) != cudaSuccess) return e;
+  // once forked, the side stream is always joined back (also when a launch
+  // fails), so a capture in progress stays well-formed and reports the error
+  e = launch_with_cluster(fc, a, R * c, sample_smem_bytes(part), stream, true);
+  if (e == cudaSuccess) e = launch_with_cluster(fs, sa, R * sa.C, stream_smem_bytes(), d->side);
+  cudaError_t ej = cudaEventRecord(d->join, d->side);
+  if (ej == cudaSuccess) ej = cudaStreamWaitEvent(stream, d->join, 0);
+  if (e != cudaSuccess) return e;
+  if (ej != cudaSuccess) return ej;
   a.select = kSelectDeferred;
   return launch_with_cluster(fc, a, deferred_clusters(R, c, sms) * c, sample_smem_bytes(part), stream);
 }

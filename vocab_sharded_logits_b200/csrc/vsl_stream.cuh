@@ -352,6 +352,7 @@ __device__ bool stream_koff(const Ctx& cx, LeaderState& L, const SampleArgs& a, 
   const double* tab = H->exp_tab;
   const int jlo = static_cast<int>(e.lo), jhi = static_cast<int>(e.hi);
   double above = 0.0, below = 0.0;
+  float xmin_ab = INFINITY;  // smallest x above the window
   stream_pass(a, cx.row, g0, n, ring, H->ring_bar, cg, [&](const float4* st4, int nq, uint32_t gid) {
 #pragma unroll
     for (int it = 0; it < kStreamChunk / 4 / kThreads; ++it) {
@@ -375,7 +376,10 @@ __device__ bool stream_koff(const Ctx& cx, LeaderState& L, const SampleArgs& a, 
         below += (fin && !ab[i] && !win[i]) ? ev : 0.0;
         any_win |= win[i];
         any_ab |= ab[i];
-        if (ab[i]) xmax = fmaxf(xmax, v[i]);
+        if (ab[i]) {
+          xmax = fmaxf(xmax, v[i]);
+          xmin_ab = fminf(xmin_ab, v[i]);
+        }
       }
       const uint32_t gq = gid + 4u * static_cast<uint32_t>(q);
       if (__any_sync(0xFFFFFFFFu, any_win)) {
@@ -396,9 +400,11 @@ __device__ bool stream_koff(const Ctx& cx, LeaderState& L, const SampleArgs& a, 
   });
   const double ta = block_sum_d0(above, H);
   const double tb = block_sum_d0(below, H);
+  const float tx = block_min_f0(xmin_ab, H);
   if (t == 0) {
     H->ex_above[0] = ta;
     H->ex_below[0] = tb;
+    H->ex_xmin[0] = tx;
     L.topn_count = 0;  // the window list starts at wc.list[0]
   }
   push_best(wc, b);

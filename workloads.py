@@ -1,10 +1,13 @@
 """Seeded synthetic workloads: the shapes, sizes and value distributions of the
-five named configurations, shared by the tests and the bench.
+five named configurations, shared by the tests, the bench and the oracle's
+baseline leg.
 
 Holds no arithmetic of the method itself: only random inputs and per-row
-parameters.  Every generator is seeded: parameters with numpy PCG64
-(``data_seed = 1000 + config index``), tensors with a torch generator on the
-target device (the same seed gives the same tensor on the same device type).
+parameters.  It sits outside the product package so that the oracle's timed
+baseline imports neither the binding nor the CUDA library.  Every generator is
+seeded: parameters with numpy PCG64 (``data_seed = 1000 + config index``),
+tensors with a torch generator on the target device (the same seed gives the
+same tensor on the same device type).
 """
 from dataclasses import dataclass
 
