@@ -1,6 +1,6 @@
 """Builds libvsl.so (the C-ABI library) in-tree with nvcc for sm_100a, and the
-test library tests/libvsl_test.so (the same objects plus a test-only probe of
-the bounded waits, tests/csrc/vsl_wait_probe.cu; never part of libvsl.so)."""
+test library tests/libvsl_test.so (the same objects plus the test-only probes
+of tests/csrc/vsl_test_probes.cu; never part of libvsl.so)."""
 import os
 import subprocess
 import sys
@@ -9,7 +9,7 @@ PKG_DIR = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG_DIR)
 CSRC = os.path.join(PKG_DIR, "csrc")
 LIB_PATH = os.path.join(PKG_DIR, "libvsl.so")
-TEST_SRC = os.path.join(ROOT, "tests", "csrc", "vsl_wait_probe.cu")
+TEST_SRC = os.path.join(ROOT, "tests", "csrc", "vsl_test_probes.cu")
 TEST_LIB_PATH = os.path.join(ROOT, "tests", "libvsl_test.so")
 SOURCES = ["vsl_api.cu", "vsl_gemm.cu", "vsl_sample.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -55,7 +55,7 @@ def build(force=False, verbose=False):
         _compile(os.path.join(CSRC, src), obj, verbose)
         objs.append(obj)
     _link(objs, LIB_PATH)
-    probe = os.path.join(objdir, "vsl_wait_probe.o")
+    probe = os.path.join(objdir, "vsl_test_probes.o")
     _compile(TEST_SRC, probe, verbose)
     _link(objs + [probe], TEST_LIB_PATH)
     return LIB_PATH

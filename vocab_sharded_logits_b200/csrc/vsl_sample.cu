@@ -57,6 +57,7 @@
 #include <mutex>
 
 #include "vsl_internal.h"
+#include "vsl_math.cuh"
 #include "vsl_ptx.cuh"
 
 namespace vsl {
@@ -228,6 +229,7 @@ struct __align__(16) SharedHeader {
   unsigned long long scan_fx[kWarps][4];
   double exp_tab[256];
   int32_t drows[kThreads];        // deferred-row pass: the rows of one block of marks
+  uint32_t row_amin;               // streaming kernel: smallest bit pattern of a nonzero |l| (top-k-off rows)
 };
 
 constexpr size_t kScratchBytes = kHistBins * 4;  // 16 KB: raw histogram, later mass / narrowing bins
@@ -260,7 +262,6 @@ __device__ __forceinline__ bool nan_or_pos_inf(uint32_t b) {
   return (b & 0x7FFFFFFFu) > 0x7F800000u || b == 0x7F800000u;
 }
 __device__ __forceinline__ bool key_finite(uint32_t k) { return k > kKeyNegInf && k < kKeyPosInf; }
-__device__ __forceinline__ float scale_x(float l, float T) { return __fdiv_rn(l, T); }
 
 __device__ __forceinline__ float fast_exp2(float t) {
   float r;

@@ -18,6 +18,8 @@
 // this kernel on the caller's stream, samples exactly those rows.
 #pragma once
 
+#include <type_traits>
+
 namespace vsl {
 
 constexpr int kStreamCap = 4096;      // candidate list capacity while streaming
@@ -139,6 +141,7 @@ __device__ __forceinline__ void stream_issue(const SampleArgs& a, int row, int g
 struct ScanStats {
   uint32_t kmax;   // largest key
   uint32_t kmf;    // smallest (key - key(-inf) - 1) mod 2^32: the smallest key above key(-inf)
+  uint32_t amin;   // (kAmin scans) smallest bit pattern of a nonzero |l|
   float m, mL, s;
 };
 constexpr float kScanNoMax = -1e30f;
@@ -147,7 +150,7 @@ constexpr float kScanNoMax = -1e30f;
 // candidates (key >= thr) appended to the list (`seen`: this warp's list end).
 // A thread takes kPer float4; a warp with any candidate reserves the slots of
 // all of them with one atomic.
-template <bool kFull>
+template <bool kFull, bool kAmin>
 __device__ __forceinline__ void stream_scan(const float4* st4, int nq, uint32_t thr, uint32_t gid, ScanStats& st,
                                             uint32_t& seen, uint32_t* counter, uint64_t* list) {
   constexpr float kLog2e = 1.4426950408889634f;
@@ -167,6 +170,10 @@ __device__ __forceinline__ void stream_scan(const float4* st4, int nq, uint32_t 
       const uint32_t b = __float_as_uint(__fadd_rn(v[i], 0.0f));
       k[it][i] = valid ? b ^ (static_cast<uint32_t>(static_cast<int32_t>(b) >> 31) | 0x80000000u) : 0u;
       st.kmf = min(st.kmf, valid ? k[it][i] - (kKeyNegInf + 1u) : 0xFFFFFFFFu);
+      if (kAmin) {
+        const uint32_t ab = __float_as_uint(v[i]) & 0x7FFFFFFFu;
+        st.amin = min(st.amin, (valid && ab != 0u) ? ab : 0xFFFFFFFFu);
+      }
     }
     const uint32_t kq = max(max(k[it][0], k[it][1]), max(k[it][2], k[it][3]));
     if (kq > st.kmax) {
@@ -309,29 +316,40 @@ __device__ bool stream_koff(const Ctx& cx, LeaderState& L, const SampleArgs& a, 
     finish_draw(cx, L, -INFINITY, 0x7FFFFFFF);
     return true;
   }
+  // passes 2 and 3 divide every logit by T: with scale_x_fast when the row's
+  // temperature and the range of its nonzero |l| allow it (decided once per
+  // row: each pass is instantiated for both quotients)
+  const float y = __frcp_rn(T);
+  const bool fast = fast_division_ok(T, fmaxf(fabsf(key_value(L.kmax)), fabsf(key_value(L.kminf))),
+                                     H->row_amin == 0xFFFFFFFFu ? INFINITY : __uint_as_float(H->row_amin));
   // ---- pass 2: fine bins of x below m (the list area's first 16 KB)
   uint32_t* cnt = reinterpret_cast<uint32_t*>(cx.list);
   uint32_t* qs = cnt + kXBins;
   for (int i = t; i < 2 * kXBins; i += kThreads) cnt[i] = 0;
   const float m = L.m;
   const float inv_w = xbin_scale(m, scale_x(key_value(L.kminf), T));
-  stream_pass(a, cx.row, g0, n, ring, H->ring_bar, cg, [&](const float4* st4, int nq, uint32_t) {
+  auto pass2 = [&](auto fast_tag) {
+    constexpr bool kF = decltype(fast_tag)::value;
+    stream_pass(a, cx.row, g0, n, ring, H->ring_bar, cg, [&](const float4* st4, int nq, uint32_t) {
 #pragma unroll
-    for (int it = 0; it < kStreamChunk / 4 / kThreads; ++it) {
-      const int q = t + it * kThreads;
-      if (q >= nq) continue;
-      const float4 v4 = st4[q];
-      const float v[4] = {v4.x, v4.y, v4.z, v4.w};
+      for (int it = 0; it < kStreamChunk / 4 / kThreads; ++it) {
+        const int q = t + it * kThreads;
+        if (q >= nq) continue;
+        const float4 v4 = st4[q];
+        const float v[4] = {v4.x, v4.y, v4.z, v4.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        if (!key_finite(fkey(v[i]))) continue;
-        uint32_t qo;
-        const int j = xbin_q(scale_x(v[i], T), m, inv_w, qo);
-        atomicAdd(&cnt[j], 1u);
-        atomicAdd(&qs[j], qo);
+        for (int i = 0; i < 4; ++i) {
+          if (!key_finite(fkey(v[i]))) continue;
+          uint32_t qo;
+          const int j = xbin_q((kF ? scale_x_fast(v[i], T, y) : scale_x(v[i], T)), m, inv_w, qo);
+          atomicAdd(&cnt[j], 1u);
+          atomicAdd(&qs[j], qo);
+        }
       }
-    }
-  });
+    });
+  };
+  if (fast) pass2(std::true_type{});
+  else pass2(std::false_type{});
   // ---- the window (a cluster of one CTA)
   Ctx wc = cx;
   wc.scratch = reinterpret_cast<uint8_t*>(cnt);
@@ -353,51 +371,56 @@ __device__ bool stream_koff(const Ctx& cx, LeaderState& L, const SampleArgs& a, 
   const int jlo = static_cast<int>(e.lo), jhi = static_cast<int>(e.hi);
   double above = 0.0, below = 0.0;
   float xmin_ab = INFINITY;  // smallest x above the window
-  stream_pass(a, cx.row, g0, n, ring, H->ring_bar, cg, [&](const float4* st4, int nq, uint32_t gid) {
+  auto pass3 = [&](auto fast_tag) {
+    constexpr bool kF = decltype(fast_tag)::value;
+    stream_pass(a, cx.row, g0, n, ring, H->ring_bar, cg, [&](const float4* st4, int nq, uint32_t gid) {
 #pragma unroll
-    for (int it = 0; it < kStreamChunk / 4 / kThreads; ++it) {
-      const int q = t + it * kThreads;
-      const bool valid = q < nq;
-      const float4 v4 = valid ? st4[q] : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-      const float l[4] = {v4.x, v4.y, v4.z, v4.w};
-      float v[4];
-      bool win[4], ab[4];
-      bool any_win = false, any_ab = false;
-      float xmax = -INFINITY;
+      for (int it = 0; it < kStreamChunk / 4 / kThreads; ++it) {
+        const int q = t + it * kThreads;
+        const bool valid = q < nq;
+        const float4 v4 = valid ? st4[q] : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+        const float l[4] = {v4.x, v4.y, v4.z, v4.w};
+        float v[4];
+        bool win[4], ab[4];
+        bool any_win = false, any_ab = false;
+        float xmax = -INFINITY;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const bool fin = key_finite(fkey(l[i]));
-        v[i] = fin ? scale_x(l[i], T) : -INFINITY;
-        const int j = fin ? xbin(v[i], m, inv_w) : kXBins;
-        win[i] = fin && j >= jlo && j <= jhi;
-        ab[i] = fin && j < jlo;
-        const double ev = exp_neg64(static_cast<double>(v[i]) - md, tab);
-        above += ab[i] ? ev : 0.0;
-        below += (fin && !ab[i] && !win[i]) ? ev : 0.0;
-        any_win |= win[i];
-        any_ab |= ab[i];
-        if (ab[i]) {
-          xmax = fmaxf(xmax, v[i]);
-          xmin_ab = fminf(xmin_ab, v[i]);
+        for (int i = 0; i < 4; ++i) {
+          const bool fin = key_finite(fkey(l[i]));
+          v[i] = fin ? (kF ? scale_x_fast(l[i], T, y) : scale_x(l[i], T)) : -INFINITY;
+          const int j = fin ? xbin(v[i], m, inv_w) : kXBins;
+          win[i] = fin && j >= jlo && j <= jhi;
+          ab[i] = fin && j < jlo;
+          const double ev = exp_neg64(static_cast<double>(v[i]) - md, tab);
+          above += ab[i] ? ev : 0.0;
+          below += (fin && !ab[i] && !win[i]) ? ev : 0.0;
+          any_win |= win[i];
+          any_ab |= ab[i];
+          if (ab[i]) {
+            xmax = fmaxf(xmax, v[i]);
+            xmin_ab = fminf(xmin_ab, v[i]);
+          }
         }
-      }
-      const uint32_t gq = gid + 4u * static_cast<uint32_t>(q);
-      if (__any_sync(0xFFFFFFFFu, any_win)) {
+        const uint32_t gq = gid + 4u * static_cast<uint32_t>(q);
+        if (__any_sync(0xFFFFFFFFu, any_win)) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            local_append(&H->list_count, wc.list, win[i], (static_cast<uint64_t>(~fkey(v[i])) << 32) | (gq + i));
+        }
+        if (!any_ab) continue;
+        const float sb = b.bound_score();
+        if (sb > -INFINITY && xmax + kGMax < sb - score_tol(sb)) continue;
+        const uint4 w = philox4x32_10(make_uint4(gq >> 2, cx.pos, cx.req, 0u), k0, k1);
+        const float bl = b.bound_l2e();
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-          local_append(&H->list_count, wc.list, win[i], (static_cast<uint64_t>(~fkey(v[i])) << 32) | (gq + i));
+          if (ab[i] && (bl == Best::kNoBound || !Best::rejects(bl, v[i], word_of(w, i))))
+            b.offer_passed(v[i], 0.0f, word_of(w, i), static_cast<int32_t>(gq + i));
       }
-      if (!any_ab) continue;
-      const float sb = b.bound_score();
-      if (sb > -INFINITY && xmax + kGMax < sb - score_tol(sb)) continue;
-      const uint4 w = philox4x32_10(make_uint4(gq >> 2, cx.pos, cx.req, 0u), k0, k1);
-      const float bl = b.bound_l2e();
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        if (ab[i] && (bl == Best::kNoBound || !Best::rejects(bl, v[i], word_of(w, i))))
-          b.offer_passed(v[i], 0.0f, word_of(w, i), static_cast<int32_t>(gq + i));
-    }
-  });
+    });
+  };
+  if (fast) pass3(std::true_type{});
+  else pass3(std::false_type{});
   const double ta = block_sum_d0(above, H);
   const double tb = block_sum_d0(below, H);
   const float tx = block_min_f0(xmin_ab, H);
@@ -467,7 +490,10 @@ __global__ void __launch_bounds__(kThreads, 2) stream_kernel(const __grid_consta
 
   constexpr float kLog2e = 1.4426950408889634f;
   uint32_t thr = 0;  // every key (-inf included) is a candidate until the first compaction
-  ScanStats st{0u, 0xFFFFFFFFu, kScanNoMax, kScanNoMax * kLog2e, 0.0f};
+  ScanStats st{0u, 0xFFFFFFFFu, 0xFFFFFFFFu, kScanNoMax, kScanNoMax * kLog2e, 0.0f};
+  // a top-k-off row on one CTA also finds its smallest nonzero |l| (the
+  // domain check of the later passes' division)
+  const bool amin_scan = take_koff && !greedy && !k_on;
   bool load_ok = true;
   bool dropped = false;  // some candidate was not listed: the row goes to the cluster kernel
   uint32_t seen = 0;     // this warp's list end after its appends of the current chunk
@@ -501,8 +527,13 @@ __global__ void __launch_bounds__(kThreads, 2) stream_kernel(const __grid_consta
       const float4* st4 = reinterpret_cast<const float4*>(ring + static_cast<size_t>(stage) * kStreamChunk);
       const int nq = min(kStreamChunk, n - cc * kStreamChunk) >> 2;
       const uint32_t gid = static_cast<uint32_t>(g0 + cc * kStreamChunk);
-      if (nq == kStreamChunk / 4) stream_scan<true>(st4, nq, thr, gid, st, seen, &H->list_count, list);
-      else stream_scan<false>(st4, nq, thr, gid, st, seen, &H->list_count, list);
+      if (amin_scan) {
+        if (nq == kStreamChunk / 4) stream_scan<true, true>(st4, nq, thr, gid, st, seen, &H->list_count, list);
+        else stream_scan<false, true>(st4, nq, thr, gid, st, seen, &H->list_count, list);
+      } else {
+        if (nq == kStreamChunk / 4) stream_scan<true, false>(st4, nq, thr, gid, st, seen, &H->list_count, list);
+        else stream_scan<false, false>(st4, nq, thr, gid, st, seen, &H->list_count, list);
+      }
     }
     // the round's stages are consumed and the appends are visible; the barrier
     // also tells every thread whether the list has less than a chunk of room left
@@ -528,6 +559,7 @@ __global__ void __launch_bounds__(kThreads, 2) stream_kernel(const __grid_consta
   for (int o = 16; o > 0; o >>= 1) {
     st.kmax = max(st.kmax, __shfl_xor_sync(0xFFFFFFFFu, st.kmax, o));
     st.kmf = min(st.kmf, __shfl_xor_sync(0xFFFFFFFFu, st.kmf, o));
+    st.amin = min(st.amin, __shfl_xor_sync(0xFFFFFFFFu, st.amin, o));
     const float om = __shfl_xor_sync(0xFFFFFFFFu, st.m, o);
     const float os = __shfl_xor_sync(0xFFFFFFFFu, st.s, o);
     const float nm = fmaxf(st.m, om);
@@ -537,6 +569,7 @@ __global__ void __launch_bounds__(kThreads, 2) stream_kernel(const __grid_consta
   const int warp = threadIdx.x >> 5;
   if (lane == 0) {
     H->red_u[warp * 4 + 0] = st.kmax;
+    H->red_u[warp * 4 + 1] = st.amin;
     H->red_u[warp * 4 + 2] = st.kmf;
     H->red_u[warp * 4 + 3] = load_ok ? 0u : 1u;
     H->red_f[warp * 2 + 0] = st.m;
@@ -544,10 +577,11 @@ __global__ void __launch_bounds__(kThreads, 2) stream_kernel(const __grid_consta
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    uint32_t ka = 0, kf = 0xFFFFFFFFu, bad = 0;
+    uint32_t ka = 0, kf = 0xFFFFFFFFu, bad = 0, am = 0xFFFFFFFFu;
     float M = kScanNoMax;
     for (int i = 0; i < kWarps; ++i) {
       ka = max(ka, H->red_u[i * 4 + 0]);
+      am = min(am, H->red_u[i * 4 + 1]);
       kf = min(kf, H->red_u[i * 4 + 2]);
       bad |= H->red_u[i * 4 + 3];
       M = fmaxf(M, H->red_f[i * 2]);
@@ -556,6 +590,7 @@ __global__ void __launch_bounds__(kThreads, 2) stream_kernel(const __grid_consta
     for (int i = 0; i < kWarps; ++i) S += H->red_f[i * 2 + 1] * fast_exp2((H->red_f[i * 2] - M) * kLog2e);
     // NaN of either sign turns the sum NaN; +inf (and a NaN's key) lies at or above key(+inf)
     bad |= (ka >= kKeyPosInf || isnan(S)) ? 1u : 0u;
+    H->row_amin = am;
     H->stats.kmax = ka;
     H->stats.kminf = kf == 0xFFFFFFFFu ? kf : kf + (kKeyNegInf + 1u);  // smallest finite key
     H->stats.bad = bad;
