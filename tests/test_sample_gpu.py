@@ -209,24 +209,26 @@ def test_streaming_geometries(cuda_device, R):
     compare(gpu, logits.numpy(), params, 99, 20, rows)
 
 
-def _binned_rows(V, R, rng):
-    """Top-k-off top-p rows for the streaming kernel's binned path, and the rows
-    that must leave it (three-pass path): a maximum far beyond the first chunk
-    (the slots slide), |x| > 1e5, a window larger than the list (very flat),
-    a cut in the open bottom slot, -inf mixes, ties, x on bin edges."""
+def _koff_rows(V, R, rng):
+    """Top-k-off top-p rows for the streaming kernel's one-CTA-per-row path: a
+    maximum at the end of the row, huge logits (the IEEE quotient instead of
+    the fused one), very flat rows (a top-p window larger than the list: the
+    cluster kernel takes the row), a cut ~18 units below the maximum, -inf
+    mixes, two finite tokens, ties, values on a 5/256 grid, all equal."""
     rows, prm = [], []
     add = lambda l, T, p: (rows.append(np.asarray(l, np.float32)), prm.append((T, p)))
     base = lambda s=1.4: rng.normal(0, s, V).astype(np.float32)
-    add(base() + np.linspace(0, 30, V, dtype=np.float32), 0.7, 0.9)      # max at the end: slides
-    add(base() + np.linspace(0, 300, V, dtype=np.float32), 1.0, 0.95)    # many slides
-    add(base() * 1e6, 1.0, 0.9)                                          # |x| > 1e5: three-pass path
+    add(base() + np.linspace(0, 30, V, dtype=np.float32), 0.7, 0.9)      # max at the end
+    add(base() + np.linspace(0, 300, V, dtype=np.float32), 1.0, 0.95)    # a steep trend
+    add(base() * 1e30, 1.0, 0.9)                                         # |l| > 2^100: the IEEE quotient
     add(base(), 50.0, 0.95)                                              # very flat: window too large
-    add(base(1.43), 0.3, 0.99999)                                        # cut ~18 below the max: the open slot
+    add(base(1.43), 0.3, 0.99999)                                        # cut ~18 below the max
     add(base(4.0), 0.05, 0.5)                                            # very peaked
     l = base(); l[::3] = -np.inf; add(l, 0.8, 0.8)                       # -inf mixed in
     l = np.full(V, -np.inf, np.float32); l[7] = 1.0; l[V // 2] = 1.5; add(l, 1.0, 0.5)  # two finite
     add(np.round(base() * 4) / 4, 0.9, 0.7)                              # ties
-    add(rng.integers(-300, 300, V).astype(np.float32) * np.float32(5 / 256), 1.0, 0.9)  # x on bin edges
+    add(rng.integers(-300, 300, V).astype(np.float32) * np.float32(5 / 256), 1.0, 0.9)  # a coarse grid
+    l = base(); l[::5] = 1e-30; add(l, 0.9, 0.8)                         # tiny |l|: the IEEE quotient
     add(np.zeros(V, np.float32), 1.0, 0.5)                               # all equal
     while len(rows) < R:
         add(base(rng.uniform(0.5, 3.0)), float(rng.uniform(0.3, 1.5)), float(rng.uniform(0.3, 0.999)))
@@ -236,14 +238,14 @@ def _binned_rows(V, R, rng):
 
 
 @pytest.mark.parametrize("V,S", [(12000, 4), (151936, 8)])
-def test_binned_top_p_large_batch_all_rows(cuda_device, V, S):
+def test_large_batch_top_k_off_all_rows(cuda_device, V, S):
     """A batch of more rows than SMs, every row top-k off with top_p < 1: the
-    streaming kernel's binned path (and its fallbacks), every row (V = 12,000)
-    or 40 rows (V = 151,936) compared with the oracle: tokens, thresholds and
-    kept sets, top-n."""
+    streaming kernel's one-CTA-per-row path (both quotients) and the rows it
+    passes on, every row (V = 12,000) or 40 rows (V = 151,936) compared with
+    the oracle: tokens, thresholds and kept sets, top-n."""
     R = 300
     rng = np.random.default_rng(V)
-    logits, params = _binned_rows(V, R, rng)
+    logits, params = _koff_rows(V, R, rng)
     gpu = run_sampler(torch.from_numpy(logits), params, 4242, 20, S, cuda_device)
     rows = range(R) if V <= 12000 else sorted(set(range(12)) | set(rng.choice(R, 28, replace=False).tolist()))
     st = compare(gpu, logits, params, 4242, 20, rows)
