@@ -110,6 +110,9 @@ def _edge_rows(V, rng):
     add(base(), 1.0, -3, 1.0)                          # bad top_k
     l = base(); l[0] = 3e38; add(l, 0.5, 0, 1.0)       # l / T overflows
     l = base(); l[::2] = -0.0; l[1::2] = 0.0; add(l, 1.0, 2, 1.0)  # signed zeros tie
+    add(base() * np.float32(1e35) - np.float32(3e37), 1.0, 0, 0.9)  # finite, all far below -1e30
+    l = base(); l[1] = -3.0e38; add(l, 1.0, 0, 0.9)        # |l| > 2.4e38: l log2(e) would overflow
+    l = base(); l[2] = 3.0e38; add(l, 1.0, 0, 0.9)         # a huge finite maximum (x finite at T = 1)
     return np.stack(rows), params
 
 

@@ -5,19 +5,25 @@
 // orcarouter.ai blog, sections "batch-sharded sampling in one paragraph" and
 // "why three lines were the whole job").
 //
-// Design (one CTA per output tile):
+// Design (each CTA walks the output tiles t = blockIdx.x, blockIdx.x +
+// gridDim.x, ...; for batch tiles of 128 and 256 rows, which keep the tensor
+// cores busy, the grid is as many CTAs as the SMs hold, so the kernel is
+// persistent; for narrower ones, bound by the weight read, one CTA per tile):
 //   * The MMA M side is the vocabulary (128 rows of W_s per tile) and the N side
 //     is the batch rows (BN in {16, 32, 64, 128, 256}), so a small batch still
 //     issues full-height tcgen05.mma instructions ("swap-AB").
 //   * Warp 0 (one lane) streams K-slabs of 64 bf16 (one 128-byte swizzle row)
 //     of W_s and hidden into a STAGES-deep shared-memory ring with 2-D TMA
-//     loads (128B swizzle, zero fill past the edges, no multicast).
+//     loads (128B swizzle, zero fill past the edges, no multicast), running
+//     ahead across tile boundaries.
 //   * Warp 1 (one lane) issues tcgen05.mma.kind::f16 (bf16 x bf16 -> fp32) into
-//     a 128 x BN fp32 accumulator in tensor memory, releasing each ring slot
-//     with tcgen05.commit.
-//   * Warps 2..5 read the accumulator with tcgen05.ld (one TMEM lane = one
-//     vocab row per thread) and store fp32 logits; for each batch row a warp
-//     writes 32 consecutive floats (128 coalesced bytes).
+//     one of two 128 x BN fp32 accumulators in tensor memory (tile i uses
+//     accumulator i mod 2), releasing each ring slot with tcgen05.commit.
+//   * Warps 2..5 read the accumulator of the previous tile with tcgen05.ld
+//     (one TMEM lane = one vocab row per thread) and store fp32 logits while
+//     the next tile's MMAs run; for each batch row a warp writes 32 consecutive
+//     floats (128 coalesced bytes).  They hand the accumulator back through an
+//     mbarrier.
 // Every wait is bounded; a wait that gives up sets the device error word and
 // the CTA drains its own copies, frees its tensor memory and returns.
 #include <cuda.h>
@@ -40,7 +46,7 @@ struct GemmArgs {
   CUtensorMap tmap_w[VSL_MAX_SLICES];
   CUtensorMap tmap_h;
   float* out[VSL_MAX_SLICES];
-  int R, H, V_s;
+  int R, H, V_s, S;
   int m_tiles;       // vocab tiles per slice
   int n_tiles;       // batch tiles
   int k_iters;       // K slabs
@@ -75,7 +81,7 @@ __host__ __device__ constexpr int tmem_cols() {
 template <int BN, int STAGES>
 constexpr size_t gemm_smem_bytes() {
   return 1024 /*alignment slack*/ + static_cast<size_t>(STAGES) * (kBM + BN) * kBK * 2 +
-         (2 * STAGES + 1) * 8 + 16;
+         (2 * STAGES + 5) * 8 + 16;
 }
 
 template <int BN, int STAGES>
@@ -84,33 +90,36 @@ __global__ void __launch_bounds__(kGemmThreads, 1) logits_local_kernel(const __g
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   constexpr uint32_t kABytes = kBM * kBK * 2;
   constexpr uint32_t kBBytes = BN * kBK * 2;
+  constexpr uint32_t kAccCols = static_cast<uint32_t>(tmem_cols<BN>());
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * kABytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * (kABytes + kBBytes));
   uint64_t* empty = full + STAGES;
-  uint64_t* accf = empty + STAGES;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+  uint64_t* acc_full = empty + STAGES;   // [2]: MMA -> epilogue
+  uint64_t* acc_empty = acc_full + 2;    // [2]: epilogue (4 warps) -> MMA
+  uint64_t* done = acc_empty + 2;        // every MMA of the CTA has completed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile uint32_t* abort_flag = tmem_slot + 1;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int n_tile = blockIdx.x % a.n_tiles;
-  const int mt = blockIdx.x / a.n_tiles;
-  const int slice = mt / a.m_tiles;
-  const int m0 = (mt % a.m_tiles) * kBM;
-  const int n0 = n_tile * BN;
+  const int total = a.S * a.m_tiles * a.n_tiles;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(smem_u32(&full[s]), 1);
       mbar_init(smem_u32(&empty[s]), 1);
     }
-    mbar_init(smem_u32(accf), 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&acc_full[b]), 1);
+      mbar_init(smem_u32(&acc_empty[b]), 4);
+    }
+    mbar_init(smem_u32(done), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), tmem_cols<BN>());
+    tmem_alloc(smem_u32(tmem_slot), 2 * kAccCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -119,90 +128,116 @@ __global__ void __launch_bounds__(kGemmThreads, 1) logits_local_kernel(const __g
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0 && lane == 0) {
-    // ---------------- TMA producer
-    prefetch_tmap(&a.tmap_w[slice]);
+    // ---------------- TMA producer: every K slab of every tile of this CTA
     prefetch_tmap(&a.tmap_h);
     const uint64_t pol_w = a.w_evict_first ? policy_evict_first() : policy_evict_last();
     const uint64_t pol_h = policy_evict_last();
-    int issued = 0;
-    for (int k = 0; k < a.k_iters; ++k) {
-      const int s = k % STAGES;
-      const uint32_t ph = (k / STAGES) & 1;
-      if (k >= STAGES && !mbar_wait_bounded(smem_u32(&empty[s]), ph ^ 1)) {
-        atomicOr(a.err, kErrGemmProducer);
-        *abort_flag = 1;
-        break;
+    int it = 0;
+    for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
+      const int mt = t / a.n_tiles;
+      const int slice = mt / a.m_tiles;
+      const int m0 = (mt % a.m_tiles) * kBM;
+      const int n0 = (t % a.n_tiles) * BN;
+      for (int k = 0; k < a.k_iters; ++k, ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1;
+        if (it >= STAGES && !mbar_wait_bounded(smem_u32(&empty[s]), ph ^ 1)) {
+          atomicOr(a.err, kErrGemmProducer);
+          *abort_flag = 1;
+        }
+        if (*abort_flag) break;
+        mbar_arrive_expect_tx(smem_u32(&full[s]), kABytes + kBBytes);
+        tma_load_2d(smem_u32(sA + s * kABytes), &a.tmap_w[slice], k * kBK, m0, smem_u32(&full[s]), pol_w);
+        tma_load_2d(smem_u32(sB + s * kBBytes), &a.tmap_h, k * kBK, n0, smem_u32(&full[s]), pol_h);
       }
-      if (*abort_flag) break;
-      mbar_arrive_expect_tx(smem_u32(&full[s]), kABytes + kBBytes);
-      tma_load_2d(smem_u32(sA + s * kABytes), &a.tmap_w[slice], k * kBK, m0, smem_u32(&full[s]), pol_w);
-      tma_load_2d(smem_u32(sB + s * kBBytes), &a.tmap_h, k * kBK, n0, smem_u32(&full[s]), pol_h);
-      issued = k + 1;
     }
     if (*abort_flag) {
       // drain our own copies: the last load issued to each slot must land
-      for (int k = issued - 1; k >= 0 && k >= issued - STAGES; --k)
-        mbar_wait_bounded(smem_u32(&full[k % STAGES]), (k / STAGES) & 1);
+      for (int j = it - 1; j >= 0 && j >= it - STAGES; --j)
+        mbar_wait_bounded(smem_u32(&full[j % STAGES]), (j / STAGES) & 1);
     }
   } else if (warp == 1 && lane == 0) {
-    // ---------------- MMA issuer
+    // ---------------- MMA issuer: tile i into accumulator i mod 2
     const uint32_t idesc = idesc_bf16_f32<BN>();
-    for (int k = 0; k < a.k_iters; ++k) {
-      const int s = k % STAGES;
-      const uint32_t ph = (k / STAGES) & 1;
-      if (!mbar_wait_bounded(smem_u32(&full[s]), ph)) {
+    int it = 0, i = 0;
+    for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x, ++i) {
+      const int b = i & 1;
+      // the epilogue has drained this accumulator (tile i - 2)
+      if (!mbar_wait_bounded(smem_u32(&acc_empty[b]), ((i >> 1) & 1) ^ 1)) {
         atomicOr(a.err, kErrGemmMma);
         *abort_flag = 1;
         break;
       }
-      if (*abort_flag) break;
       tc_fence_after();
-      const uint64_t da = sw128_desc(smem_u32(sA + s * kABytes));
-      const uint64_t db = sw128_desc(smem_u32(sB + s * kBBytes));
+      const uint32_t acc = tmem + static_cast<uint32_t>(b) * kAccCols;
+      for (int k = 0; k < a.k_iters; ++k, ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1;
+        if (!mbar_wait_bounded(smem_u32(&full[s]), ph)) {
+          atomicOr(a.err, kErrGemmMma);
+          *abort_flag = 1;
+        }
+        if (*abort_flag) break;
+        tc_fence_after();
+        const uint64_t da = sw128_desc(smem_u32(sA + s * kABytes));
+        const uint64_t db = sw128_desc(smem_u32(sB + s * kBBytes));
 #pragma unroll
-      for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
-        // advancing K by 16 bf16 = 32 bytes moves the start address by 2 (16-byte units)
-        umma_f16(tmem, da + 2 * kk, db + 2 * kk, idesc, (k | kk) != 0);
+        for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
+          // advancing K by 16 bf16 = 32 bytes moves the start address by 2 (16-byte units)
+          umma_f16(acc, da + 2 * kk, db + 2 * kk, idesc, (k | kk) != 0);
+        }
+        umma_commit(smem_u32(&empty[s]));
       }
-      umma_commit(smem_u32(&empty[s]));
+      umma_commit(smem_u32(&acc_full[b]));
     }
-    umma_commit(smem_u32(accf));
-    // the accumulator must be complete before tensor memory is freed below
-    mbar_wait_bounded(smem_u32(accf), 0);
+    // every MMA must be complete before tensor memory is freed below
+    umma_commit(smem_u32(done));
+    mbar_wait_bounded(smem_u32(done), 0);
   } else if (warp >= 2) {
-    // ---------------- epilogue: TMEM -> registers -> global fp32
-    const bool ok = mbar_wait_bounded(smem_u32(accf), 0);
-    if (!ok) {
-      atomicOr(a.err, kErrGemmEpilogue);
-      *abort_flag = 1;
-    }
-    tc_fence_after();
-    // tcgen05.ld is warp-collective: decide for the whole warp
-    if (__all_sync(0xFFFFFFFFu, ok && !*abort_flag)) {
-      const int q = warp & 3;                  // TMEM lane quarter this warp may access
-      const int m = m0 + q * 32 + lane;        // vocab row of this thread
+    // ---------------- epilogue: TMEM -> registers -> global fp32, one tile behind the MMAs
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    int i = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++i) {
+      const int b = i & 1;
+      const bool ok = mbar_wait_bounded(smem_u32(&acc_full[b]), (i >> 1) & 1);
+      if (!ok) {
+        if (lane == 0) atomicOr(a.err, kErrGemmEpilogue);
+        *abort_flag = 1;
+      }
+      tc_fence_after();
+      // tcgen05.ld is warp-collective: decide for the whole warp
+      if (!__all_sync(0xFFFFFFFFu, ok && !*abort_flag)) break;
+      const int mt = t / a.n_tiles;
+      const int slice = mt / a.m_tiles;
+      const int m = (mt % a.m_tiles) * kBM + q * 32 + lane;  // vocab row of this thread
+      const int n0 = (t % a.n_tiles) * BN;
       float* out = a.out[slice];
       const bool m_ok = m < a.V_s;
+      const uint32_t acc = tmem + static_cast<uint32_t>(b) * kAccCols + (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll 1
       for (int c = 0; c < BN; c += 16) {
         uint32_t r[16];
-        tmem_ld_x16(tmem + (static_cast<uint32_t>(q * 32) << 16) + c, r);
+        tmem_ld_x16(acc + c, r);
         tmem_ld_wait();
         if (m_ok) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int n = n0 + c + i;
-            if (n < a.R) out[static_cast<size_t>(n) * a.V_s + m] = __uint_as_float(r[i]);
+          for (int j = 0; j < 16; ++j) {
+            const int n = n0 + c + j;
+            if (n < a.R) out[static_cast<size_t>(n) * a.V_s + m] = __uint_as_float(r[j]);
           }
         }
       }
+      // the accumulator's reads are complete: hand it back to the MMA warp
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&acc_empty[b]));
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, tmem_cols<BN>());
+    tmem_dealloc(tmem, 2 * kAccCols);
   }
 }
 
@@ -246,21 +281,36 @@ cudaError_t launch_bn(GemmArgs& args, const void* hidden, const void* const* w, 
   args.w_evict_first = args.n_tiles == 1;
   constexpr size_t smem = gemm_smem_bytes<BN, STAGES>();
   auto kern = logits_local_kernel<BN, STAGES>;
-  // the shared-memory attribute is per device: set once on each, with it current
+  // per device, with it current: the shared-memory attribute and the number of
+  // CTAs that run at once (the persistent grid)
   constexpr int kMaxDevices = 64;
   static std::once_flag once[kMaxDevices];
   static cudaError_t attr_status[kMaxDevices];
+  static int slots[kMaxDevices];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::call_once(once[dev], [&] {
+    int sms = 0, per_sm = 0;
     attr_status[dev] = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (attr_status[dev] == cudaSuccess)
+      attr_status[dev] = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (attr_status[dev] == cudaSuccess)
+      attr_status[dev] = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kGemmThreads, smem);
+    slots[dev] = sms * per_sm;
+    if (attr_status[dev] == cudaSuccess && slots[dev] <= 0) attr_status[dev] = cudaErrorInvalidConfiguration;
   });
   if (attr_status[dev] != cudaSuccess) return attr_status[dev];
-  const long long grid = static_cast<long long>(S) * args.m_tiles * args.n_tiles;
-  if (grid > 0x7FFFFFFF) return cudaErrorInvalidConfiguration;
-  kern<<<static_cast<unsigned>(grid), kGemmThreads, smem, stream>>>(args);
+  const long long tiles = static_cast<long long>(S) * args.m_tiles * args.n_tiles;
+  if (tiles > 0x7FFFFFFF) return cudaErrorInvalidConfiguration;
+  args.S = S;
+  // tensor-bound widths (BN >= 128) run persistent, one CTA per slot, so each
+  // tile's epilogue overlaps the next tile's MMAs; the narrow widths are bound
+  // by the weight read and keep one CTA per tile (the hardware then hands a
+  // free slot the next tile, whatever the pace of each SM)
+  const int grid = static_cast<int>(BN < 128 || tiles < slots[dev] ? tiles : slots[dev]);
+  kern<<<grid, kGemmThreads, smem, stream>>>(args);
   return cudaGetLastError();
 }
 

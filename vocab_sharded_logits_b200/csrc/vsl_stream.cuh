@@ -135,14 +135,17 @@ __device__ __forceinline__ void stream_issue(const SampleArgs& a, int row, int g
 }
 
 // Statistics a thread keeps over the logits it scans.  The sum of exp runs
-// against the thread's largest finite value m (prescaled: mL = m log2 e); m
-// starts at -1e30 so that a thread that never sees a finite value adds only
-// exp(-inf) = 0.  NaN of either sign makes the sum NaN; +inf shows in kmax.
+// against the thread's largest finite value m (each term exp2((v - m) log2 e),
+// so no product overflows whatever the logits' size).  m starts at a finite
+// stand-in, so a thread that has seen only -inf adds exp(-inf) = 0; a sum that
+// is still 0 has no maximum yet (the stand-in may lie above a row's values):
+// it is never rescaled, and the merges ignore its m.  NaN of either sign
+// makes the sum NaN; +inf shows in kmax.
 struct ScanStats {
   uint32_t kmax;   // largest key
   uint32_t kmf;    // smallest (key - key(-inf) - 1) mod 2^32: the smallest key above key(-inf)
   uint32_t amin;   // (kAmin scans) smallest bit pattern of a nonzero |l|
-  float m, mL, s;
+  float m, s;
 };
 constexpr float kScanNoMax = -1e30f;
 
@@ -180,14 +183,12 @@ __device__ __forceinline__ void stream_scan(const float4* st4, int nq, uint32_t 
       st.kmax = kq;
       if (kq > kKeyNegInf) {  // a new largest value: rescale the sum to it
         const float mn = key_value(kq);
-        const float mnL = mn * kLog2e;
-        st.s *= fast_exp2(st.mL - mnL);
+        st.s = st.s == 0.0f ? 0.0f : st.s * fast_exp2((st.m - mn) * kLog2e);
         st.m = mn;
-        st.mL = mnL;
       }
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) st.s += fast_exp2(fmaf(v[i], kLog2e, -st.mL));
+    for (int i = 0; i < 4; ++i) st.s += fast_exp2((v[i] - st.m) * kLog2e);
     any |= kq >= thr && valid;
   }
   if (!__any_sync(0xFFFFFFFFu, any)) return;
@@ -490,7 +491,7 @@ __global__ void __launch_bounds__(kThreads, 2) stream_kernel(const __grid_consta
 
   constexpr float kLog2e = 1.4426950408889634f;
   uint32_t thr = 0;  // every key (-inf included) is a candidate until the first compaction
-  ScanStats st{0u, 0xFFFFFFFFu, 0xFFFFFFFFu, kScanNoMax, kScanNoMax * kLog2e, 0.0f};
+  ScanStats st{0u, 0xFFFFFFFFu, 0xFFFFFFFFu, kScanNoMax, 0.0f};
   // a top-k-off row on one CTA also finds its smallest nonzero |l| (the
   // domain check of the later passes' division)
   const bool amin_scan = take_koff && !greedy && !k_on;
@@ -554,7 +555,7 @@ __global__ void __launch_bounds__(kThreads, 2) stream_kernel(const __grid_consta
 
   int cg = nch;  // chunks streamed so far (the ring's position)
   // ---- CTA statistics (the cluster kernel's CtaStats layout)
-  // (m, s) pairs merge by rescaling to the larger m; kScanNoMax pairs add 0
+  // (m, s) pairs merge by rescaling to the larger m; empty sums add 0
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     st.kmax = max(st.kmax, __shfl_xor_sync(0xFFFFFFFFu, st.kmax, o));
@@ -562,9 +563,11 @@ __global__ void __launch_bounds__(kThreads, 2) stream_kernel(const __grid_consta
     st.amin = min(st.amin, __shfl_xor_sync(0xFFFFFFFFu, st.amin, o));
     const float om = __shfl_xor_sync(0xFFFFFFFFu, st.m, o);
     const float os = __shfl_xor_sync(0xFFFFFFFFu, st.s, o);
-    const float nm = fmaxf(st.m, om);
-    st.s = st.s * fast_exp2((st.m - nm) * kLog2e) + os * fast_exp2((om - nm) * kLog2e);
-    st.m = nm;
+    // a lane with an empty sum has no maximum to keep
+    const float nm = fmaxf(st.s != 0.0f ? st.m : -INFINITY, os != 0.0f ? om : -INFINITY);
+    st.s = (st.s == 0.0f ? 0.0f : st.s * fast_exp2((st.m - nm) * kLog2e)) +
+           (os == 0.0f ? 0.0f : os * fast_exp2((om - nm) * kLog2e));
+    st.m = nm > -INFINITY ? nm : kScanNoMax;
   }
   const int warp = threadIdx.x >> 5;
   if (lane == 0) {
@@ -578,23 +581,24 @@ __global__ void __launch_bounds__(kThreads, 2) stream_kernel(const __grid_consta
   __syncthreads();
   if (threadIdx.x == 0) {
     uint32_t ka = 0, kf = 0xFFFFFFFFu, bad = 0, am = 0xFFFFFFFFu;
-    float M = kScanNoMax;
+    float M = -INFINITY;  // over the warps whose sum is not empty
     for (int i = 0; i < kWarps; ++i) {
       ka = max(ka, H->red_u[i * 4 + 0]);
       am = min(am, H->red_u[i * 4 + 1]);
       kf = min(kf, H->red_u[i * 4 + 2]);
       bad |= H->red_u[i * 4 + 3];
-      M = fmaxf(M, H->red_f[i * 2]);
+      if (H->red_f[i * 2 + 1] != 0.0f) M = fmaxf(M, H->red_f[i * 2]);
     }
     float S = 0.0f;
-    for (int i = 0; i < kWarps; ++i) S += H->red_f[i * 2 + 1] * fast_exp2((H->red_f[i * 2] - M) * kLog2e);
+    for (int i = 0; i < kWarps; ++i)
+      if (H->red_f[i * 2 + 1] != 0.0f) S += H->red_f[i * 2 + 1] * fast_exp2((H->red_f[i * 2] - M) * kLog2e);
     // NaN of either sign turns the sum NaN; +inf (and a NaN's key) lies at or above key(+inf)
     bad |= (ka >= kKeyPosInf || isnan(S)) ? 1u : 0u;
     H->row_amin = am;
     H->stats.kmax = ka;
     H->stats.kminf = kf == 0xFFFFFFFFu ? kf : kf + (kKeyNegInf + 1u);  // smallest finite key
     H->stats.bad = bad;
-    const bool none = !(M > kScanNoMax);
+    const bool none = !(M > -INFINITY);
     H->stats.m = none ? -INFINITY : M;
     H->stats.s = none ? 0.0f : S;
   }
