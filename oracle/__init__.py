@@ -25,12 +25,20 @@ reordering beyond what the definition states:
   exact tie / threshold readings are the plainest readings stated in each
   function's docstring.  ``processed_logprobs`` gives the log-probabilities of
   the distribution the draw samples from (after temperature, top-k, top-p).
+* ``oracle.verify``   - speculative verification of deterministic drafts over
+  a request's (spec + 1) rows (same page: the acceptance length of section
+  "the 1.5 % estimate"; draft logits are left for later in section
+  "batch-sharded sampling in one paragraph").
+* ``oracle.timing``   - the harness that times the sampler oracle on the
+  host's cores for the CPU baseline (no arithmetic of the method).
 
 Pins (see ``tests/test_oracle_*.py``): the Philox known-answer vectors of the
 Random123 distribution, brute-force enumeration on tiny vocabularies, closed
 forms (greedy == argmax, top_k=1, top_p -> 0, top_p=1 keeps all, sum of
 probabilities == 1), exact integer GEMMs, and chi-square tests of the draw
 frequencies; the processed logprobs against the library log-softmax (full
-vocabulary), point masses, and the frequencies of the oracle's own draws.
+vocabulary), point masses, and the frequencies of the oracle's own draws; the
+verification against an independent formulation and, by sampling, against
+the rejection rule it implements for a point-mass draft.
 No function here is "parity unpinned".
 """
