@@ -65,6 +65,7 @@ typedef enum {
 /* Limits of the library. */
 #define VSL_MAX_SLICES 16       /* S <= 16                                  */
 #define VSL_MAX_LOGPROBS 20     /* 0 <= n_logprobs <= 20 (and <= S * V_s)   */
+#define VSL_MAX_SPEC 64         /* speculative tokens per request in vsl_verify_drafts */
 
 /* Row flags written by vsl_sample (bit set = the row was not sampled).  A
  * flagged row gets token -1, logprob NaN, top-n ids -1 and top-n logprobs NaN;
@@ -208,6 +209,35 @@ VSL_API vsl_status vsl_sample_ex(const float* const* logits_slices, int32_t R, i
                          int32_t* token_ids, float* token_logprob, int32_t* topn_ids,
                          float* topn_logprob, uint32_t* row_flags, void* workspace,
                          size_t workspace_bytes, const vsl_sample_extras* extras, void* stream);
+
+/* vsl_verify_drafts - speculative verification of deterministic draft tokens
+ * over the rows one vsl_sample call drew.  Source: "Qwen4Exp batch-sharded
+ * sampling: inside vLLM PR #61018" (orcarouter.ai blog): the sampler's
+ * batch x (speculative tokens + 1) x vocab rows and sharded draft logits left
+ * for later (section "batch-sharded sampling in one paragraph"), acceptance
+ * length (section "the 1.5 % estimate").
+ * Request q owns rows q * (spec + 1) + j, j = 0 .. spec, row j holding the
+ * target's draw t_j for position j (vsl_sample's token, -1 if flagged); its
+ * drafts d_0 .. d_{spec-1} are single tokens (a point-mass draft).  Draft j is
+ * accepted while t_j == d_j and t_j >= 0; with a accepted the request emits
+ * d_0 .. d_{a-1}, then t_a (the correction, or the bonus token when a ==
+ * spec), then -1.  With vsl_sample's draw keyed by (seed, request, position,
+ * token) this is the rejection rule for a point-mass draft: d_j is accepted
+ * with probability p(d_j), p the distribution the row samples from, and a
+ * rejected position emits a token distributed as p without d_j.
+ *   token_ids     : device int32 [requests * (spec + 1)]  (vsl_sample's output)
+ *   token_logprob : device fp32 [requests * (spec + 1)]   (optional, NULL together with out_logprob)
+ *   draft_ids     : device int32 [requests][spec]         (may be NULL when spec == 0)
+ *   out_ids       : device int32 [requests][spec + 1]     (output) the emitted tokens, then -1
+ *   out_logprob   : device fp32 [requests][spec + 1]      (optional output) each emitted
+ *                   token's row logprob, NaN after the emitted tokens
+ *   accepted      : device int32 [requests]               (output) a, 0 <= a <= spec
+ *   1 <= requests, 0 <= spec <= VSL_MAX_SPEC.
+ * Errors: VSL_ERR_INVALID_ARG (null pointers, sizes, only one of the two
+ *         logprob pointers), VSL_ERR_UNSUPPORTED, VSL_ERR_CUDA. */
+VSL_API vsl_status vsl_verify_drafts(const int32_t* token_ids, const float* token_logprob,
+                                     const int32_t* draft_ids, int32_t requests, int32_t spec,
+                                     int32_t* out_ids, float* out_logprob, int32_t* accepted, void* stream);
 
 /* Reads and clears the device error word the kernels set when a bounded wait
  * gives up (a bug, never expected).  Synchronises the current device.

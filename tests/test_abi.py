@@ -70,6 +70,14 @@ def test_host_validation_rejects_bad_arguments_without_a_device():
     assert L.vsl_sample(*args(S=17)) == 3
     assert L.vsl_sample(*args(V_s=1 << 20, S=1)) == 3         # beyond the largest vocabulary
     assert L.vsl_sample_workspace_bytes(2048, 8, 18992, 20) == 0
+    # vsl_verify_drafts
+    L.vsl_verify_drafts.argtypes = [vp] * 3 + [ctypes.c_int32] * 2 + [vp] * 4
+    assert L.vsl_verify_drafts(None, None, fake, 4, 3, fake, None, fake, None) == 1     # no tokens
+    assert L.vsl_verify_drafts(fake, None, fake, 0, 3, fake, None, fake, None) == 1     # no requests
+    assert L.vsl_verify_drafts(fake, None, fake, 4, -1, fake, None, fake, None) == 1    # negative spec
+    assert L.vsl_verify_drafts(fake, None, fake, 4, 65, fake, None, fake, None) == 1    # spec > VSL_MAX_SPEC
+    assert L.vsl_verify_drafts(fake, None, None, 4, 3, fake, None, fake, None) == 1     # drafts missing
+    assert L.vsl_verify_drafts(fake, fake, fake, 4, 3, fake, None, fake, None) == 1     # one logprob pointer
     # vsl_sample_ex: the same checks, plus the optional outputs' alignment
     ex = lambda extras, **kw: L.vsl_sample_ex(*args(**kw)[:-1], extras, None)
     assert ex(None, R=0) == 1

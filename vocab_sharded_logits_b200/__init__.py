@@ -12,7 +12,7 @@ import torch
 
 __all__ = [
     "logits_local", "sample", "sample_launches", "sample_plan", "make_row_params", "SampleResult", "lib", "status_string",
-    "device_error", "VslError", "ROW_NONFINITE", "ROW_ALL_NEG_INF", "ROW_BAD_TEMPERATURE",
+    "device_error", "VslError", "verify_drafts", "VerifyResult", "MAX_SPEC", "ROW_NONFINITE", "ROW_ALL_NEG_INF", "ROW_BAD_TEMPERATURE",
     "ROW_BAD_TOP_P", "ROW_BAD_TOP_K", "ROW_SCALE_OVERFLOW", "MAX_SLICES", "MAX_LOGPROBS",
 ]
 
@@ -21,6 +21,7 @@ LIB_PATH = os.path.join(_PKG_DIR, "libvsl.so")
 
 MAX_SLICES = 16
 MAX_LOGPROBS = 20
+MAX_SPEC = 64
 ROW_NONFINITE = 1 << 0
 ROW_ALL_NEG_INF = 1 << 1
 ROW_BAD_TEMPERATURE = 1 << 2
@@ -68,6 +69,8 @@ def _load():
     l.vsl_sample_ex.restype = ctypes.c_int
     l.vsl_sample_ex.argtypes = [ctypes.POINTER(vp), i32, i32, i32, vp, u64, i32, vp, vp, vp, vp, vp, vp, sz,
                                 ctypes.POINTER(_Extras), vp]
+    l.vsl_verify_drafts.restype = ctypes.c_int
+    l.vsl_verify_drafts.argtypes = [vp, vp, vp, i32, i32, vp, vp, vp, vp]
     l.vsl_device_error.restype = ctypes.c_int
     l.vsl_device_error.argtypes = [ctypes.POINTER(u32)]
     l.vsl_status_string.restype = ctypes.c_char_p
@@ -218,6 +221,47 @@ def sample(logits_slices, params, seed, n_logprobs, out=None, stream=None, kept_
                                    _ptr(ws), ws_bytes, ctypes.byref(extras) if extras is not None else None,
                                    _stream_handle(stream, dev))
     _check(status, "vsl_sample")
+    return out
+
+
+class VerifyResult:
+    """Outputs of ``verify_drafts``: accepted drafts per request, the emitted
+    tokens [requests, spec + 1] and (when asked for) their logprobs."""
+
+    def __init__(self, accepted, out_ids, out_logprob=None):
+        self.accepted = accepted
+        self.out_ids = out_ids
+        self.out_logprob = out_logprob
+
+
+def verify_drafts(token_ids, draft_ids, token_logprob=None, out=None, stream=None):
+    """Speculative verification of deterministic drafts over ``sample``'s rows.
+
+    token_ids: int32 [requests * (spec + 1)] CUDA tensor (``sample``'s tokens, rows of a
+    request consecutive); draft_ids: int32 [requests, spec] CUDA tensor; token_logprob:
+    optional fp32 [requests * (spec + 1)].  Draft j is accepted while the target's draw
+    at position j equals it; a request emits its accepted drafts, then the target's
+    token at the first rejected position (or the bonus token), then -1.
+    """
+    requests, spec = draft_ids.shape
+    dev = token_ids.device
+    if token_ids.dtype != torch.int32 or token_ids.numel() != requests * (spec + 1) or not token_ids.is_contiguous():
+        raise ValueError("token_ids must be a contiguous int32 tensor of requests * (spec + 1) rows")
+    if draft_ids.dtype != torch.int32 or not draft_ids.is_contiguous() or draft_ids.device != dev:
+        raise ValueError("draft_ids must be a contiguous int32 [requests, spec] tensor on the tokens' device")
+    if token_logprob is not None and (token_logprob.dtype != torch.float32 or not token_logprob.is_contiguous()
+                                      or token_logprob.numel() != token_ids.numel() or token_logprob.device != dev):
+        raise ValueError("token_logprob must be a contiguous fp32 tensor like token_ids")
+    if out is None:
+        out = VerifyResult(torch.empty(requests, dtype=torch.int32, device=dev),
+                           torch.empty(requests, spec + 1, dtype=torch.int32, device=dev),
+                           torch.empty(requests, spec + 1, device=dev) if token_logprob is not None else None)
+    with _on_device(dev):
+        status = lib.vsl_verify_drafts(_ptr(token_ids), _ptr(token_logprob), _ptr(draft_ids) if spec else None,
+                                       requests, spec, _ptr(out.out_ids),
+                                       _ptr(out.out_logprob) if token_logprob is not None else None,
+                                       _ptr(out.accepted), _stream_handle(stream, dev))
+    _check(status, "vsl_verify_drafts")
     return out
 
 

@@ -118,6 +118,19 @@ vsl_status vsl_sample(const float* const* logits_slices, int32_t R, int32_t S, i
                        topn_logprob, row_flags, workspace, workspace_bytes, nullptr, stream);
 }
 
+vsl_status vsl_verify_drafts(const int32_t* token_ids, const float* token_logprob, const int32_t* draft_ids,
+                             int32_t requests, int32_t spec, int32_t* out_ids, float* out_logprob,
+                             int32_t* accepted, void* stream) {
+  if (token_ids == nullptr || out_ids == nullptr || accepted == nullptr) return VSL_ERR_INVALID_ARG;
+  if (requests <= 0 || spec < 0 || spec > VSL_MAX_SPEC) return VSL_ERR_INVALID_ARG;
+  if (spec > 0 && draft_ids == nullptr) return VSL_ERR_INVALID_ARG;
+  if ((out_logprob == nullptr) != (token_logprob == nullptr)) return VSL_ERR_INVALID_ARG;
+  if (static_cast<long long>(requests) * (spec + 1) > 0x7FFFFFFFLL) return VSL_ERR_UNSUPPORTED;
+  const cudaError_t e = vsl::launch_verify(token_ids, token_logprob, draft_ids, requests, spec, out_ids,
+                                           out_logprob, accepted, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? VSL_OK : VSL_ERR_CUDA;
+}
+
 vsl_status vsl_device_error(uint32_t* code_out) {
   if (cudaDeviceSynchronize() != cudaSuccess) return VSL_ERR_CUDA;
   uint32_t v = 0;

@@ -23,6 +23,11 @@ cudaError_t launch_sample(const float* const* logits, int R, int S, int V_s,
                           int32_t* token_ids, float* token_logprob, int32_t* topn_ids,
                           float* topn_logprob, uint32_t* row_flags, float* kept_theta, cudaStream_t stream);
 
+// Launch the speculative verification.  Arguments already validated.
+cudaError_t launch_verify(const int32_t* token_ids, const float* token_logprob, const int32_t* draft_ids,
+                          int requests, int spec, int32_t* out_ids, float* out_logprob, int32_t* accepted,
+                          cudaStream_t stream);
+
 // Sampler launch geometry for a vocabulary of V tokens on a device that
 // schedules clusters of at most maxc CTAs: CTAs per row (cluster size) and
 // elements per CTA.  Returns false if V cannot be handled.
