@@ -54,7 +54,8 @@ def _peaks():
 
 # The timed units of a step and the sources each is built from.  "sample" is
 # one call of the sampler (the streaming kernel and the cluster kernel).
-_KERNEL_SOURCES = {"logits_local_kernel": ["vsl_gemm.cu"], "sample": ["vsl_sample.cu", "vsl_stream.cuh"]}
+_KERNEL_SOURCES = {"logits_local_kernel": ["vsl_gemm.cu", "vsl_ptx.cuh"],
+                   "sample": ["vsl_sample.cu", "vsl_stream.cuh", "vsl_math.cuh", "vsl_ptx.cuh"]}
 
 
 def _source_sha(kernel):
@@ -574,6 +575,46 @@ def run_sampler_only(args, w):
     return 0
 
 
+def run_gemm_only(args, w):
+    """Times ``logits_local`` alone on the workload's bf16 inputs: ``--steps`` event
+    pairs around 10 back-to-back launches each (launch overhead hidden), after
+    ``--warmup`` launches, clocks sampled; one JSON line (a profiling aid)."""
+    import vocab_sharded_logits_b200 as vsl
+    dev = torch.device("cuda", 0)
+    hbm_peak, tf_peak, _, peak_kind = _peaks()
+    hidden, ws = W.gemm_inputs(w, dev)
+    out = [torch.empty(w.R, w.V_s, dtype=torch.float32, device=dev) for _ in range(w.S)]
+    for _ in range(args.warmup):
+        vsl.logits_local(hidden, ws, out=out)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(0)
+    clocks.start()
+    times = []
+    t_start = time.time()
+    i = 0
+    while i < args.steps or (clocks.proc is not None and clocks.count() - clocks.skip < 3
+                             and time.time() - t_start < 10):
+        e0, e1 = _events(2)
+        e0.record()
+        for _ in range(10):
+            vsl.logits_local(hidden, ws, out=out)
+        e1.record()
+        torch.cuda.synchronize()
+        if i < args.steps:
+            times.append(e0.elapsed_time(e1) / 10)
+        i += 1
+    clk = clocks.stop()
+    ms = statistics.median(times)
+    flops = 2.0 * w.R * w.H * w.V
+    nbytes = w.V * w.H * 2 + w.R * w.H * 2 + w.R * w.V * 4
+    print(json.dumps({"metric": f"logits_local TFLOP/s ({w.name})", "value": flops / ms / 1e9, "unit": "TFLOP/s",
+                      "ms": ms, "hbm_gbs": nbytes / (ms / 1e3) / 1e9, "tflops_frac_of_burst": flops / ms / 1e9 / tf_peak,
+                      "hbm_frac": nbytes / (ms / 1e3) / 1e9 / hbm_peak, "peak_source": peak_kind, "clocks": clk,
+                      "config": {"workload": w.name, "rows": w.R, "hidden": w.H, "vocab": w.V, "slices": w.S}}),
+          flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -587,6 +628,8 @@ def main():
     ap.add_argument("--no-per-config", action="store_true", help="measure the headline workload only")
     ap.add_argument("--sampler-only", action="store_true",
                     help="time the sampler alone on the workload's synthetic logits (profiling aid)")
+    ap.add_argument("--gemm-only", action="store_true",
+                    help="time the projection alone, 10 back-to-back launches per timing (profiling aid)")
     args = ap.parse_args()
     w = W.WORKLOADS[args.workload]
     if args.impl == "reference":
@@ -596,6 +639,8 @@ def main():
         return 1
     if args.sampler_only:
         return run_sampler_only(args, w)
+    if args.gemm_only:
+        return run_gemm_only(args, w)
     return run_gpu(args, w)
 
 
