@@ -194,16 +194,32 @@ VSL_API vsl_status vsl_sample(const float* const* logits_slices, int32_t R, int3
  *                0 or >= S * V_s, top_p >= 1) and NaN for a greedy or a
  *                flagged row.  The kept set the token is drawn from is exactly
  *                { i : x_i finite and x_i >= max(theta_k, theta_p) }.
+ *   processed_logprob      : device fp32 [R]: the token's log-probability under
+ *                the distribution it was drawn from (after temperature, top-k
+ *                and top-p): log q_i = (x_i - m) - log sum_{j in K} exp(x_j - m),
+ *                K the kept set above, m = max_K x; 0 for a greedy row, NaN for
+ *                a flagged row.  Needs kept_theta.
+ *   processed_topn_ids     : device int32 [R][n_logprobs] (with processed_logprob,
+ *   processed_topn_logprob : device fp32 [R][n_logprobs]   when n_logprobs > 0):
+ *                the n_logprobs largest log q (largest x of K, lower id first on
+ *                equal x) and their values, then -1 / -inf once K is exhausted
+ *                (a greedy row: its token with 0).  Computed by one more pass
+ *                over the logits after the draw.
  * Source: "Qwen4Exp batch-sharded sampling: inside vLLM PR #61018"
  * (orcarouter.ai blog), section "batch-sharded sampling in one paragraph": the
- * sampler's top-k and top-p work per request. */
+ * sampler's top-k and top-p work per request, logprobs through max_logprobs. */
 typedef struct {
   float* kept_theta;
+  float* processed_logprob;
+  int32_t* processed_topn_ids;
+  float* processed_topn_logprob;
 } vsl_sample_extras;
 
 /* vsl_sample_ex - vsl_sample with optional outputs (extras may be NULL, which
  * is vsl_sample).  Same arguments, ownership and errors as vsl_sample, plus
- * VSL_ERR_ALIGNMENT for a kept_theta that is not 8-byte aligned. */
+ * VSL_ERR_ALIGNMENT for a kept_theta that is not 8-byte aligned and
+ * VSL_ERR_INVALID_ARG for processed outputs without kept_theta or without
+ * their top-n buffers when n_logprobs > 0. */
 VSL_API vsl_status vsl_sample_ex(const float* const* logits_slices, int32_t R, int32_t S, int32_t V_s,
                          const vsl_row_params* params_dev, uint64_t seed, int32_t n_logprobs,
                          int32_t* token_ids, float* token_logprob, int32_t* topn_ids,

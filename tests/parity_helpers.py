@@ -20,9 +20,12 @@ def run_sampler(logits, params_np, seed, n, S_slices, device):
     T, k, p, req, pos = params_np
     slices = [t.contiguous() for t in torch.tensor_split(logits.to(device), S_slices, dim=1)]
     prm = vsl.make_row_params(T, k, p, req, pos, device)
-    out = vsl.sample(slices, prm, seed, n, kept_theta=True)
+    out = vsl.sample(slices, prm, seed, n, processed=True)
     torch.cuda.synchronize()
     return {
+        "p_token": out.processed_logprob.cpu().numpy(),
+        "p_topn_ids": out.processed_topn_ids.cpu().numpy(),
+        "p_topn_lp": out.processed_topn_logprob.cpu().numpy(),
         "token": out.token_ids.cpu().numpy(),
         "token_lp": out.token_logprob.cpu().numpy(),
         "topn_ids": out.topn_ids.cpu().numpy(),
@@ -39,9 +42,11 @@ def _expected_theta(v):
 def compare(gpu, logits_np, params_np, seed, n, rows):
     """Element-by-element comparison on ``rows``: flags, top-n ids (exact) and
     logprobs (1e-4), the kept-set thresholds theta_k and theta_p (bit-exact) and
-    the kept set they define (every element), and the token (exact).  Returns
-    counts of the allowed exceptions: near-ties of the draw (the token only) and
-    cut-ties of top-p (theta_p, the kept set and the token)."""
+    the kept set they define (every element), the token (exact), and the
+    processed logprobs (the token's and the top-n's: ids exact, values 1e-4).
+    Returns counts of the allowed exceptions: near-ties of the draw (the token
+    only) and cut-ties of top-p (theta_p, the kept set, the token and the
+    processed logprobs)."""
     T, k, p, req, pos = params_np
     stats = {"rows": 0, "near_tie": 0, "cut_tie": 0, "mismatch_allowed": 0, "kept_checked": 0}
     for r in rows:
@@ -52,8 +57,10 @@ def compare(gpu, logits_np, params_np, seed, n, rows):
         if o.flags:
             assert gpu["token"][r] == -1 and np.isnan(gpu["token_lp"][r])
             assert np.isnan(th).all(), (r, th)
+            assert np.isnan(gpu["p_token"][r])
             if n:
                 assert np.all(gpu["topn_ids"][r] == -1)
+                assert np.all(gpu["p_topn_ids"][r] == -1) and np.isnan(gpu["p_topn_lp"][r]).all()
             continue
         if n:
             assert np.array_equal(gpu["topn_ids"][r], o.topn_ids), (r, gpu["topn_ids"][r], o.topn_ids)
@@ -80,5 +87,14 @@ def compare(gpu, logits_np, params_np, seed, n, rows):
                 assert o.kept[tok]
         ref_lp = S.log_softmax(logits_np[r])[tok]
         assert abs(float(gpu["token_lp"][r]) - ref_lp) <= LOGPROB_TOL, (r, gpu["token_lp"][r], ref_lp)
+        if not o.cut_tie:
+            pr = S.processed_logprobs(logits_np[r], T[r], int(k[r]), p[r], n)
+            assert abs(float(gpu["p_token"][r]) - pr.logprob[tok]) <= LOGPROB_TOL, (r, gpu["p_token"][r], pr.logprob[tok])
+            if n:
+                assert np.array_equal(gpu["p_topn_ids"][r], pr.topn_ids), (r, gpu["p_topn_ids"][r], pr.topn_ids)
+                got, want = gpu["p_topn_lp"][r].astype(np.float64), pr.topn_logprob
+                assert np.array_equal(np.isinf(got), np.isinf(want)), r
+                fin = np.isfinite(want)
+                assert np.allclose(got[fin], want[fin], atol=LOGPROB_TOL, rtol=0), r
     REPORT.append((os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0], dict(stats)))
     return stats

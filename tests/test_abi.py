@@ -83,6 +83,9 @@ def test_host_validation_rejects_bad_arguments_without_a_device():
     assert ex(None, R=0) == 1
     assert ex(ctypes.byref(v._Extras(0x10004)), V_s=512) == 2         # kept_theta not 8-byte aligned
     assert ex(ctypes.byref(v._Extras(0x10008)), V_s=1 << 20) == 3     # aligned: the size check follows
+    assert ex(ctypes.byref(v._Extras(0, 0x10000)), V_s=512) == 1       # processed without kept_theta
+    assert ex(ctypes.byref(v._Extras(0x10008, 0x10000)), V_s=512) == 1 # processed top-n missing (n = 5)
+    assert ex(ctypes.byref(v._Extras(0, 0, 0x10000)), V_s=512) == 1    # processed top-n without the token's
 
 
 def test_binding_has_no_cpu_fallback(monkeypatch, tmp_path):

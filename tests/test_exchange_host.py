@@ -107,16 +107,21 @@ def _rank_leaves(rank, world, port, q):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     sys.path.insert(0, ROOT)
     from vocab_sharded_logits_b200 import exchange as X
-    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=10))
-    if rank == 1:
-        os._exit(3)  # leaves between steps, before the exchange, with nothing in flight
     import time
     t0 = time.time()
     try:
+        dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=10))
+        dist.barrier()  # every connection is up: the group has run one step together
+        if rank == 1:
+            os._exit(3)  # leaves between steps, before the exchange, with nothing in flight
+        t0 = time.time()
         X.exchange_slices(torch.zeros(4, 8))
         q.put(("no error", time.time() - t0))
     except Exception as e:  # the collective ends with an error
-        q.put((type(e).__name__, time.time() - t0))
+        if rank == 0:
+            q.put((type(e).__name__, time.time() - t0))
+    q.close()
+    q.join_thread()  # the queue's feeder thread has written the result before the process ends
     os._exit(0)
 
 

@@ -42,7 +42,8 @@ class VslError(RuntimeError):
 
 
 class _Extras(ctypes.Structure):
-    _fields_ = [("kept_theta", ctypes.c_void_p)]
+    _fields_ = [("kept_theta", ctypes.c_void_p), ("processed_logprob", ctypes.c_void_p),
+                ("processed_topn_ids", ctypes.c_void_p), ("processed_topn_logprob", ctypes.c_void_p)]
 
 
 class _Plan(ctypes.Structure):
@@ -167,16 +168,20 @@ class SampleResult:
     """Outputs of ``sample``: token ids, their raw logprobs, top-n ids / logprobs, row
     flags, and (when asked for) the kept-set thresholds ``kept_theta`` [R, 2]."""
 
-    def __init__(self, token_ids, token_logprob, topn_ids, topn_logprob, row_flags, kept_theta=None):
+    def __init__(self, token_ids, token_logprob, topn_ids, topn_logprob, row_flags, kept_theta=None,
+                 processed_logprob=None, processed_topn_ids=None, processed_topn_logprob=None):
         self.token_ids = token_ids
         self.token_logprob = token_logprob
         self.topn_ids = topn_ids
         self.topn_logprob = topn_logprob
         self.row_flags = row_flags
         self.kept_theta = kept_theta
+        self.processed_logprob = processed_logprob
+        self.processed_topn_ids = processed_topn_ids
+        self.processed_topn_logprob = processed_topn_logprob
 
 
-def sample(logits_slices, params, seed, n_logprobs, out=None, stream=None, kept_theta=False):
+def sample(logits_slices, params, seed, n_logprobs, out=None, stream=None, kept_theta=False, processed=False):
     """Per-row temperature / top-k / top-p / Gumbel-max draw / top-n raw logprobs.
 
     logits_slices: list of fp32 [R, V_s] CUDA tensors (row r = concatenation over slices).
@@ -184,6 +189,9 @@ def sample(logits_slices, params, seed, n_logprobs, out=None, stream=None, kept_
     kept_theta: also return each row's (theta_k, theta_p) on x = fl(l / T) (fp32 [R, 2]):
     the draw's kept set is every finite x >= max(theta_k, theta_p); -inf for a rule
     that is off, NaN for greedy and flagged rows.
+    processed: also return the processed logprobs (log-probabilities of the distribution
+    each token was drawn from: the token's [R], the top-n ids / values [R, n]); implies
+    kept_theta.
     """
     R, V_s = logits_slices[0].shape
     S = len(logits_slices)
@@ -202,14 +210,25 @@ def sample(logits_slices, params, seed, n_logprobs, out=None, stream=None, kept_
                            torch.empty(R, dtype=torch.int32, device=dev))
     if params.device != dev:
         raise ValueError("params must be on the logits' device")
+    kept_theta = kept_theta or processed
     if kept_theta and out.kept_theta is None:
         out.kept_theta = torch.empty(R, 2, dtype=torch.float32, device=dev)
+    if processed and out.processed_logprob is None:
+        n = max(n_logprobs, 1)
+        out.processed_logprob = torch.empty(R, dtype=torch.float32, device=dev)
+        out.processed_topn_ids = torch.empty(R, n, dtype=torch.int32, device=dev)[:, :n_logprobs]
+        out.processed_topn_logprob = torch.empty(R, n, dtype=torch.float32, device=dev)[:, :n_logprobs]
     extras = None
     if kept_theta:
         if out.kept_theta.dtype != torch.float32 or tuple(out.kept_theta.shape) != (R, 2) or \
                 not out.kept_theta.is_contiguous():
             raise ValueError("kept_theta must be a contiguous fp32 [R, 2] tensor")
         extras = _Extras(out.kept_theta.data_ptr())
+    if processed:
+        extras.processed_logprob = out.processed_logprob.data_ptr()
+        if n_logprobs > 0:
+            extras.processed_topn_ids = out.processed_topn_ids.data_ptr()
+            extras.processed_topn_logprob = out.processed_topn_logprob.data_ptr()
     ws_bytes = lib.vsl_sample_workspace_bytes(R, S, V_s, n_logprobs)
     with _on_device(dev):
         ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev) if ws_bytes else None

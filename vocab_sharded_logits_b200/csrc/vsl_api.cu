@@ -99,14 +99,23 @@ vsl_status vsl_sample_ex(const float* const* logits_slices, int32_t R, int32_t S
   }
   float* kept_theta = extras != nullptr ? extras->kept_theta : nullptr;
   if (kept_theta != nullptr && (reinterpret_cast<uintptr_t>(kept_theta) & 7u) != 0) return VSL_ERR_ALIGNMENT;
+  float* p_token = extras != nullptr ? extras->processed_logprob : nullptr;
+  int32_t* p_topn_ids = extras != nullptr ? extras->processed_topn_ids : nullptr;
+  float* p_topn = extras != nullptr ? extras->processed_topn_logprob : nullptr;
+  if (p_token == nullptr && (p_topn_ids != nullptr || p_topn != nullptr)) return VSL_ERR_INVALID_ARG;
+  if (p_token != nullptr && kept_theta == nullptr) return VSL_ERR_INVALID_ARG;
+  if (p_token != nullptr && n_logprobs > 0 && (p_topn_ids == nullptr || p_topn == nullptr)) return VSL_ERR_INVALID_ARG;
   if (V > vsl::sample_max_vocab()) return VSL_ERR_UNSUPPORTED;
   int maxc = 0, c = 0, part = 0;
   if (vsl::sample_max_cluster(&maxc) != cudaSuccess) return VSL_ERR_CUDA;
   if (!vsl::sample_geometry_for(V, maxc, &c, &part)) return VSL_ERR_UNSUPPORTED;
   if (workspace_bytes < vsl_sample_workspace_bytes(R, S, V_s, n_logprobs)) return VSL_ERR_WORKSPACE_TOO_SMALL;
-  const cudaError_t e = vsl::launch_sample(logits_slices, R, S, V_s, params_dev, seed, n_logprobs, token_ids,
-                                           token_logprob, topn_ids, topn_logprob, row_flags, kept_theta,
-                                           static_cast<cudaStream_t>(stream));
+  cudaError_t e = vsl::launch_sample(logits_slices, R, S, V_s, params_dev, seed, n_logprobs, token_ids,
+                                     token_logprob, topn_ids, topn_logprob, row_flags, kept_theta,
+                                     static_cast<cudaStream_t>(stream));
+  if (e == cudaSuccess && p_token != nullptr)
+    e = vsl::launch_processed(logits_slices, R, S, V_s, params_dev, n_logprobs, token_ids, topn_ids, row_flags,
+                              kept_theta, p_token, p_topn_ids, p_topn, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? VSL_OK : VSL_ERR_CUDA;
 }
 

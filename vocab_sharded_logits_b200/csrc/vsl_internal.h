@@ -23,6 +23,12 @@ cudaError_t launch_sample(const float* const* logits, int R, int S, int V_s,
                           int32_t* token_ids, float* token_logprob, int32_t* topn_ids,
                           float* topn_logprob, uint32_t* row_flags, float* kept_theta, cudaStream_t stream);
 
+// Launch the processed-logprobs pass (after the sampler, same stream).
+cudaError_t launch_processed(const float* const* logits, int R, int S, int V_s, const vsl_row_params* params,
+                             int n_logprobs, const int32_t* token_ids, const int32_t* topn_ids,
+                             const uint32_t* row_flags, const float* kept_theta, float* p_token,
+                             int32_t* p_topn_ids, float* p_topn, cudaStream_t stream);
+
 // Launch the speculative verification.  Arguments already validated.
 cudaError_t launch_verify(const int32_t* token_ids, const float* token_logprob, const int32_t* draft_ids,
                           int requests, int spec, int32_t* out_ids, float* out_logprob, int32_t* accepted,
