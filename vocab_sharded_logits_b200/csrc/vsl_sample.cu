@@ -230,6 +230,8 @@ struct __align__(16) SharedHeader {
   double exp_tab[256];
   int32_t drows[kThreads];        // deferred-row pass: the rows of one block of marks
   uint32_t row_amin;               // streaming kernel: smallest bit pattern of a nonzero |l| (top-k-off rows)
+  uint32_t kcut_above, kcut_window;  // streaming kernel: raw-key thresholds of the top-p window
+  double row_z;                    // streaming kernel: the float64 mass of every finite x of the row
 };
 
 constexpr size_t kScratchBytes = kHistBins * 4;  // 16 KB: raw histogram, later mass / narrowing bins
@@ -484,6 +486,49 @@ struct Best {
         take(cs, cx, cl, cw, cid);
         sd = csd;
         have_sd = true;
+      }
+    }
+  }
+};
+
+// Per-warp queue of kept tokens in shared memory (kDrawQueue entries per
+// warp, each a 32-bit payload and the token id).  A pass that finds kept
+// tokens scattered among many dropped ones queues them, and the warp works
+// on 32 queued tokens at a time, one per lane, so the per-token work (the
+// Philox words, the quotient, the exp) runs at full width instead of once per
+// warp step whenever any lane has a kept token.  Every lane of the warp
+// calls push and drain together (the count n is warp-uniform).
+constexpr int kDrawQueue = 160;  // a drain leaves < 32 entries; at most 128 are pushed before the next
+constexpr size_t kDrawQueueBytes = static_cast<size_t>(kWarps) * kDrawQueue * 8;
+struct DrawQueue {
+  uint64_t* q;  // this warp's entries: payload << 32 | id
+  uint32_t n;
+  __device__ __forceinline__ void init(void* base) {
+    q = reinterpret_cast<uint64_t*>(base) + (threadIdx.x >> 5) * kDrawQueue;
+    n = 0;
+  }
+  __device__ __forceinline__ void push(bool pred, uint64_t e) {
+    const uint32_t m = __ballot_sync(0xFFFFFFFFu, pred);
+    if (pred) q[n + __popc(m & ((1u << (threadIdx.x & 31)) - 1u))] = e;
+    n += __popc(m);
+  }
+  // Takes queued tokens 32 at a time while a full batch is queued (all:
+  // until the queue is empty), each through one(payload, Philox word, id).
+  template <typename F>
+  __device__ __forceinline__ void drain(bool all, uint32_t pos, uint32_t req, uint32_t k0, uint32_t k1, F&& one) {
+    while (n >= 32u || (all && n > 0u)) {
+      __syncwarp();
+      const uint32_t lane = threadIdx.x & 31;
+      const uint32_t take = min(n, 32u);
+      const uint32_t base = n - take;
+      const bool act = lane < take;
+      const uint64_t e = act ? q[base + lane] : 0ull;
+      __syncwarp();
+      n = base;
+      if (act) {
+        const uint32_t id = static_cast<uint32_t>(e);
+        const uint4 w = philox4x32_10(make_uint4(id >> 2, pos, req, 0u), k0, k1);
+        one(static_cast<uint32_t>(e >> 32), word_of(w, static_cast<int>(id & 3u)), static_cast<int32_t>(id));
       }
     }
   }
@@ -2219,7 +2264,7 @@ __device__ void finish_draw(const Ctx& cx, LeaderState& L, double sd, int32_t id
 // masses; the window sorted by (x desc, id asc) gives the cut as the smallest
 // x whose mass of strictly larger values is < top_p Z; the draw adds the
 // window's kept entries to the CTAs' bests.
-__device__ void exact_tail(const Ctx& cx, LeaderState& L) {
+__device__ void exact_tail(const Ctx& cx, LeaderState& L, double z_total = -1.0) {
   SharedHeader* H = cx.H;
   const int first = L.topn_count;  // the first-pass list [0, first), then the window
   const int count = min(static_cast<int>(H->list_count), kListCap) - first;
@@ -2241,7 +2286,8 @@ __device__ void exact_tail(const Ctx& cx, LeaderState& L) {
     for (int i = i0; i < i1; ++i) sum += exp_neg64(static_cast<double>(key_value(entry_key(buf[i]))) - m, H->exp_tab);
     double W;
     const double incl = block_scan_d(sum, &W, H);
-    const double pz = static_cast<double>(L.top_p) * (A + W + B);
+    // Z = A + W + B, or the total mass when the caller summed it over the whole row
+    const double pz = static_cast<double>(L.top_p) * (z_total >= 0.0 ? z_total : A + W + B);
     double run = A + (incl - sum);
     int cand = -1;
     for (int i = i0; i < i1; ++i) {

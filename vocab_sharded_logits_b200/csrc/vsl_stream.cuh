@@ -33,6 +33,7 @@ constexpr size_t kStreamRingBytes = static_cast<size_t>(kStreamStages) * kStream
 // the ring has landed by then).
 constexpr size_t kStreamBinsBytes = 1024;
 static_assert(kStreamRingBytes >= kScratchBytes, "the ring doubles as the leader's scratch");
+static_assert(kDrawQueueBytes <= kListCap * 8, "the third pass's draw queue lives in the list's first half");
 __host__ __device__ __forceinline__ size_t stream_smem_bytes() {
   return ((sizeof(SharedHeader) + 127) & ~size_t(127)) + kStreamBinsBytes + kStreamListBytes + kStreamRingBytes;
 }
@@ -329,6 +330,9 @@ __device__ bool stream_koff(const Ctx& cx, LeaderState& L, const SampleArgs& a, 
   for (int i = t; i < 2 * kXBins; i += kThreads) cnt[i] = 0;
   const float m = L.m;
   const float inv_w = xbin_scale(m, scale_x(key_value(L.kminf), T));
+  const double md = static_cast<double>(m);
+  const double* tab = H->exp_tab;
+  double zsum = 0.0;  // the float64 mass of every finite x: Z for the cut
   auto pass2 = [&](auto fast_tag) {
     constexpr bool kF = decltype(fast_tag)::value;
     stream_pass(a, cx.row, g0, n, ring, H->ring_bar, cg, [&](const float4* st4, int nq, uint32_t) {
@@ -342,15 +346,19 @@ __device__ bool stream_koff(const Ctx& cx, LeaderState& L, const SampleArgs& a, 
         for (int i = 0; i < 4; ++i) {
           if (!key_finite(fkey(v[i]))) continue;
           uint32_t qo;
-          const int j = xbin_q((kF ? scale_x_fast(v[i], T, y) : scale_x(v[i], T)), m, inv_w, qo);
+          const float x = kF ? scale_x_fast(v[i], T, y) : scale_x(v[i], T);
+          const int j = xbin_q(x, m, inv_w, qo);
           atomicAdd(&cnt[j], 1u);
           atomicAdd(&qs[j], qo);
+          zsum += exp_neg64(static_cast<double>(x) - md, tab);
         }
       }
     });
   };
   if (fast) pass2(std::true_type{});
   else pass2(std::false_type{});
+  const double zt = block_sum_d0(zsum, H);
+  if (t == 0) H->row_z = zt;
   // ---- the window (a cluster of one CTA)
   Ctx wc = cx;
   wc.scratch = reinterpret_cast<uint8_t*>(cnt);
@@ -362,18 +370,56 @@ __device__ bool stream_koff(const Ctx& cx, LeaderState& L, const SampleArgs& a, 
   px.step = inv_w;
   Plan e;
   if (!window_distributed(wc, px, e)) return false;
-  // ---- pass 3: float64 masses above / below the window, its members, the draw above it
-  if (t == 0) H->gbound = kKeyNegInf;
+  // ---- the raw-key thresholds of the window: x = fl(l / T) and its bin are
+  // monotone in l, so bin j < jlo (kept for certain) holds exactly for the
+  // keys >= ka and jlo <= j <= jhi (the window) for kw <= key < ka; each is
+  // found by a binary search over the row's finite keys with the same quotient
+  const int jlo = static_cast<int>(e.lo), jhi = static_cast<int>(e.hi);
+  auto thresholds = [&](auto fast_tag) {
+    constexpr bool kF = decltype(fast_tag)::value;
+    auto first_key = [&](auto pred) {  // the smallest key in [kminf, kmax] with pred(bin), else kmax + 1
+      uint32_t lo = L.kminf, hi = L.kmax + 1u;
+      while (lo < hi) {
+        const uint32_t mid = lo + (hi - lo) / 2u;
+        const float l = key_value(mid);
+        if (pred(xbin(kF ? scale_x_fast(l, T, y) : scale_x(l, T), m, inv_w))) hi = mid;
+        else lo = mid + 1u;
+      }
+      return lo;
+    };
+    const uint32_t ka = first_key([&](int jb) { return jb < jlo; });
+    const uint32_t kw = min(first_key([&](int jb) { return jb <= jhi; }), ka);
+    H->kcut_above = ka;
+    H->kcut_window = kw;
+  };
+  if (t == 0) {
+    if (fast) thresholds(std::true_type{});
+    else thresholds(std::false_type{});
+    H->gbound = kKeyNegInf;
+  }
   __syncthreads();
+  const uint32_t ka = H->kcut_above;
+  const uint32_t kw = H->kcut_window;
+  const double z_total = H->row_z;
+  // ---- pass 3: every key compared with the thresholds; the window's members
+  // listed (sort key ~x key, id); every token kept for certain queued, and the
+  // warp drains the queue 32 tokens at a time: its x, its float64 mass (the
+  // mass above the window, A) and the draw
   Best b;
   b.init(&H->gbound);
-  const double md = static_cast<double>(m);
-  const double* tab = H->exp_tab;
-  const int jlo = static_cast<int>(e.lo), jhi = static_cast<int>(e.hi);
-  double above = 0.0, below = 0.0;
+  double above = 0.0;
   float xmin_ab = INFINITY;  // smallest x above the window
+  DrawQueue dq;
+  dq.init(cnt);  // the fine bins' area is free once the window is found, until the window is sorted
   auto pass3 = [&](auto fast_tag) {
     constexpr bool kF = decltype(fast_tag)::value;
+    auto one = [&](uint32_t lbits, uint32_t wd, int32_t id) {
+      const float x = kF ? scale_x_fast(__uint_as_float(lbits), T, y) : scale_x(__uint_as_float(lbits), T);
+      above += exp_neg64(static_cast<double>(x) - md, tab);
+      xmin_ab = fminf(xmin_ab, x);
+      const float bl = b.bound_l2e();
+      if (bl == Best::kNoBound || !Best::rejects(bl, x, wd)) b.offer_passed(x, 0.0f, wd, id);
+    };
     stream_pass(a, cx.row, g0, n, ring, H->ring_bar, cg, [&](const float4* st4, int nq, uint32_t gid) {
 #pragma unroll
       for (int it = 0; it < kStreamChunk / 4 / kThreads; ++it) {
@@ -381,59 +427,44 @@ __device__ bool stream_koff(const Ctx& cx, LeaderState& L, const SampleArgs& a, 
         const bool valid = q < nq;
         const float4 v4 = valid ? st4[q] : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
         const float l[4] = {v4.x, v4.y, v4.z, v4.w};
-        float v[4];
         bool win[4], ab[4];
-        bool any_win = false, any_ab = false;
-        float xmax = -INFINITY;
+        bool any_win = false;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const bool fin = key_finite(fkey(l[i]));
-          v[i] = fin ? (kF ? scale_x_fast(l[i], T, y) : scale_x(l[i], T)) : -INFINITY;
-          const int j = fin ? xbin(v[i], m, inv_w) : kXBins;
-          win[i] = fin && j >= jlo && j <= jhi;
-          ab[i] = fin && j < jlo;
-          const double ev = exp_neg64(static_cast<double>(v[i]) - md, tab);
-          above += ab[i] ? ev : 0.0;
-          below += (fin && !ab[i] && !win[i]) ? ev : 0.0;
+          const uint32_t k = fkey(l[i]);  // -inf and padding lie below kw: the row's keys are finite above it
+          ab[i] = valid && k >= ka;
+          win[i] = valid && k >= kw && k < ka;
           any_win |= win[i];
-          any_ab |= ab[i];
-          if (ab[i]) {
-            xmax = fmaxf(xmax, v[i]);
-            xmin_ab = fminf(xmin_ab, v[i]);
-          }
         }
         const uint32_t gq = gid + 4u * static_cast<uint32_t>(q);
         if (__any_sync(0xFFFFFFFFu, any_win)) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            local_append(&H->list_count, wc.list, win[i], (static_cast<uint64_t>(~fkey(v[i])) << 32) | (gq + i));
+          for (int i = 0; i < 4; ++i) {
+            const float x = win[i] ? (kF ? scale_x_fast(l[i], T, y) : scale_x(l[i], T)) : 0.0f;
+            local_append(&H->list_count, wc.list, win[i], (static_cast<uint64_t>(~fkey(x)) << 32) | (gq + i));
+          }
         }
-        if (!any_ab) continue;
-        const float sb = b.bound_score();
-        if (sb > -INFINITY && xmax + kGMax < sb - score_tol(sb)) continue;
-        const uint4 w = philox4x32_10(make_uint4(gq >> 2, cx.pos, cx.req, 0u), k0, k1);
-        const float bl = b.bound_l2e();
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-          if (ab[i] && (bl == Best::kNoBound || !Best::rejects(bl, v[i], word_of(w, i))))
-            b.offer_passed(v[i], 0.0f, word_of(w, i), static_cast<int32_t>(gq + i));
+          dq.push(ab[i], (static_cast<uint64_t>(__float_as_uint(l[i])) << 32) | (gq + i));
+        dq.drain(false, cx.pos, cx.req, k0, k1, one);  // at most 31 + 128 queued
       }
     });
+    dq.drain(true, cx.pos, cx.req, k0, k1, one);
   };
   if (fast) pass3(std::true_type{});
   else pass3(std::false_type{});
   const double ta = block_sum_d0(above, H);
-  const double tb = block_sum_d0(below, H);
   const float tx = block_min_f0(xmin_ab, H);
   if (t == 0) {
     H->ex_above[0] = ta;
-    H->ex_below[0] = tb;
+    H->ex_below[0] = 0.0;  // unused: the cut takes the total mass
     H->ex_xmin[0] = tx;
     L.topn_count = 0;  // the window list starts at wc.list[0]
   }
   push_best(wc, b);
   __syncthreads();
-  exact_tail(wc, L);
+  exact_tail(wc, L, z_total);
   return true;
 }
 
