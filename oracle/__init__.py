@@ -29,6 +29,11 @@ reordering beyond what the definition states:
   a request's (spec + 1) rows (same page: the acceptance length of section
   "the 1.5 % estimate"; draft logits are left for later in section
   "batch-sharded sampling in one paragraph").
+* ``oracle.tile_stats`` - per block of 128 ids of a vocab slice, the maxima of
+  its four 32-id quarters, its sum of exp and its smallest finite logit: the
+  statistics the projection can emit tile by tile so that the sampler reads
+  only the tiles that can hold its candidates (a reading of the same section;
+  the record is the library's, stated in the module).
 * ``oracle.timing``   - the harness that times the sampler oracle on the
   host's cores for the CPU baseline (no arithmetic of the method).
 
