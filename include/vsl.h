@@ -116,6 +116,43 @@ VSL_API vsl_status vsl_logits_local(const void* hidden_bf16, const void* const* 
                             float* const* logits_slices, int32_t R, int32_t H, int32_t S,
                             int32_t V_s, void* stream);
 
+/* Tile statistics of the logits (optional; source: "Qwen4Exp batch-sharded
+ * sampling: inside vLLM PR #61018" (orcarouter.ai blog), section
+ * "batch-sharded sampling in one paragraph": the sampler's top-k / top-p and
+ * logprobs need, per row, the softmax statistics and the top candidates of
+ * the whole vocabulary; produced tile by tile where the projection writes the
+ * logits, they let vsl_sample read only the tiles that can hold a row's
+ * candidates).  For row r, slice s and block b of 128 ids (B = ceil(V_s / 128)
+ * blocks per slice) the record at float offset ((r * S + s) * B + b) * 8 of a
+ * device fp32 array of vsl_tile_stats_floats(R, S, V_s) floats (32-byte
+ * aligned, rows contiguous) holds:
+ *   [0..3] the largest logit of each 32-id quarter of the block (ids
+ *          s * V_s + 128 b + 32 q + [0, 32) below (s + 1) * V_s; -inf for a
+ *          quarter with no id; unspecified for a quarter holding a NaN)
+ *   [4]    sum over the block of exp(l - c), c the block's largest logit when
+ *          finite, else 0 (float32 with a fast exp; NaN if a logit is NaN,
+ *          +inf if one is +inf)
+ *   [5]    the block's smallest finite logit (+inf if none)
+ *   [6, 7] 0
+ * vsl_tile_stats_floats returns 0 for non-positive sizes. */
+VSL_API size_t vsl_tile_stats_floats(int32_t R, int32_t S, int32_t V_s);
+
+/* vsl_logits_local_ex - vsl_logits_local that also writes the tile
+ * statistics of the logits it produces from the same accumulators (tile_stats
+ * may be NULL: vsl_logits_local).  Extra error: VSL_ERR_ALIGNMENT for a
+ * tile_stats not 32-byte aligned. */
+VSL_API vsl_status vsl_logits_local_ex(const void* hidden_bf16, const void* const* w_slices_bf16,
+                                       float* const* logits_slices, int32_t R, int32_t H, int32_t S,
+                                       int32_t V_s, float* tile_stats, void* stream);
+
+/* vsl_tile_stats - the tile statistics of logits already in device memory
+ * (logits_slices as for vsl_sample; one read of every logit).
+ * Errors: VSL_ERR_INVALID_ARG, VSL_ERR_ALIGNMENT (slices not 16-byte or
+ * tile_stats not 32-byte aligned, V_s % 4 != 0), VSL_ERR_UNSUPPORTED,
+ * VSL_ERR_CUDA. */
+VSL_API vsl_status vsl_tile_stats(const float* const* logits_slices, int32_t R, int32_t S, int32_t V_s,
+                                  float* tile_stats, void* stream);
+
 /* Bytes of device workspace vsl_sample needs for these sizes (0 if none). */
 VSL_API size_t vsl_sample_workspace_bytes(int32_t R, int32_t S, int32_t V_s, int32_t n_logprobs);
 
@@ -205,6 +242,18 @@ VSL_API vsl_status vsl_sample(const float* const* logits_slices, int32_t R, int3
  *                equal x) and their values, then -1 / -inf once K is exhausted
  *                (a greedy row: its token with 0).  Computed by one more pass
  *                over the logits after the draw.
+ *   tile_stats : (input) device, the tile statistics of exactly these logits
+ *                (vsl_logits_local_ex or vsl_tile_stats), 32-byte aligned.
+ *                Rows that are greedy or have 0 < top_k <= 1024 then read the
+ *                records and only the 32-id quarters whose largest x can reach
+ *                their top max(n_logprobs, top_k) (greedy: max(n_logprobs, 1))
+ *                instead of the whole row: the R-th largest block maximum t0
+ *                is at most the row's R-th largest logit, so every candidate
+ *                lies in a quarter whose largest x is >= fl(t0 / T).  Token
+ *                ids, top-n ids, flags and kept_theta equal those of the call
+ *                without them; the raw logprobs take the row's log-sum-exp
+ *                from the records' sums (float32).  Ignored for top-k-off
+ *                rows and when S * B exceeds 4096 blocks.
  * Source: "Qwen4Exp batch-sharded sampling: inside vLLM PR #61018"
  * (orcarouter.ai blog), section "batch-sharded sampling in one paragraph": the
  * sampler's top-k and top-p work per request, logprobs through max_logprobs. */
@@ -213,11 +262,13 @@ typedef struct {
   float* processed_logprob;
   int32_t* processed_topn_ids;
   float* processed_topn_logprob;
+  const float* tile_stats;
 } vsl_sample_extras;
 
 /* vsl_sample_ex - vsl_sample with optional outputs (extras may be NULL, which
  * is vsl_sample).  Same arguments, ownership and errors as vsl_sample, plus
- * VSL_ERR_ALIGNMENT for a kept_theta that is not 8-byte aligned and
+ * VSL_ERR_ALIGNMENT for a kept_theta that is not 8-byte aligned or a
+ * tile_stats that is not 32-byte aligned, and
  * VSL_ERR_INVALID_ARG for processed outputs without kept_theta or without
  * their top-n buffers when n_logprobs > 0. */
 VSL_API vsl_status vsl_sample_ex(const float* const* logits_slices, int32_t R, int32_t S, int32_t V_s,

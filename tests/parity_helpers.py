@@ -14,13 +14,15 @@ LOGIT_TOL = 2e-2        # projection: bf16 inputs, fp32 accumulation vs float64
 REPORT = []
 
 
-def run_sampler(logits, params_np, seed, n, S_slices, device):
+def run_sampler(logits, params_np, seed, n, S_slices, device, tiles=False):
     """Runs the CUDA sampler on [R, V] fp32 logits split into S_slices slices,
-    with the kept-set thresholds requested."""
+    with the kept-set thresholds requested (tiles: with the tile statistics of
+    the logits, from the library's statistics kernel)."""
     T, k, p, req, pos = params_np
     slices = [t.contiguous() for t in torch.tensor_split(logits.to(device), S_slices, dim=1)]
     prm = vsl.make_row_params(T, k, p, req, pos, device)
-    out = vsl.sample(slices, prm, seed, n, processed=True)
+    stats = vsl.tile_stats(slices) if tiles else None
+    out = vsl.sample(slices, prm, seed, n, processed=True, tile_stats=stats)
     torch.cuda.synchronize()
     return {
         "p_token": out.processed_logprob.cpu().numpy(),

@@ -86,6 +86,19 @@ def test_host_validation_rejects_bad_arguments_without_a_device():
     assert ex(ctypes.byref(v._Extras(0, 0x10000)), V_s=512) == 1       # processed without kept_theta
     assert ex(ctypes.byref(v._Extras(0x10008, 0x10000)), V_s=512) == 1 # processed top-n missing (n = 5)
     assert ex(ctypes.byref(v._Extras(0, 0, 0x10000)), V_s=512) == 1    # processed top-n without the token's
+    assert ex(ctypes.byref(v._Extras(0, 0, 0, 0, 0x10010)), V_s=512) == 2  # tile statistics not 32-byte aligned
+    # tile statistics: sizes, and the checks of both producers
+    assert L.vsl_tile_stats_floats(4, 2, 300) == 4 * 2 * 3 * 8
+    assert L.vsl_tile_stats_floats(0, 2, 300) == 0
+    assert L.vsl_tile_stats(None, 4, 1, 512, fake, None) == 1
+    assert L.vsl_tile_stats(arr1, 4, 1, 512, None, None) == 1
+    assert L.vsl_tile_stats(arr1, 0, 1, 512, fake, None) == 1
+    assert L.vsl_tile_stats(arr1, 4, 17, 512, fake, None) == 3
+    assert L.vsl_tile_stats(arr1, 4, 1, 510, fake, None) == 2                # V_s % 4
+    assert L.vsl_tile_stats(arr1, 4, 1, 512, vp(0x10010), None) == 2         # records not 32-byte aligned
+    assert L.vsl_tile_stats((vp * 1)(0x10004), 4, 1, 512, fake, None) == 2   # slice not 16-byte aligned
+    assert L.vsl_logits_local_ex(fake, arr1, arr1, 4, 64, 1, 512, vp(0x10010), None) == 2
+    assert L.vsl_logits_local_ex(fake, arr1, arr1, 0, 64, 1, 512, fake, None) == 1
 
 
 def test_binding_has_no_cpu_fallback(monkeypatch, tmp_path):

@@ -11,7 +11,7 @@ import os
 import torch
 
 __all__ = [
-    "logits_local", "sample", "sample_launches", "sample_plan", "make_row_params", "SampleResult", "lib", "status_string",
+    "logits_local", "tile_stats", "tile_stats_shape", "sample", "sample_launches", "sample_plan", "make_row_params", "SampleResult", "lib", "status_string",
     "device_error", "VslError", "verify_drafts", "VerifyResult", "MAX_SPEC", "ROW_NONFINITE", "ROW_ALL_NEG_INF", "ROW_BAD_TEMPERATURE",
     "ROW_BAD_TOP_P", "ROW_BAD_TOP_K", "ROW_SCALE_OVERFLOW", "MAX_SLICES", "MAX_LOGPROBS",
 ]
@@ -43,7 +43,8 @@ class VslError(RuntimeError):
 
 class _Extras(ctypes.Structure):
     _fields_ = [("kept_theta", ctypes.c_void_p), ("processed_logprob", ctypes.c_void_p),
-                ("processed_topn_ids", ctypes.c_void_p), ("processed_topn_logprob", ctypes.c_void_p)]
+                ("processed_topn_ids", ctypes.c_void_p), ("processed_topn_logprob", ctypes.c_void_p),
+                ("tile_stats", ctypes.c_void_p)]
 
 
 class _Plan(ctypes.Structure):
@@ -59,6 +60,12 @@ def _load():
     vp, i32, u32, u64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_uint32, ctypes.c_uint64, ctypes.c_size_t
     l.vsl_logits_local.restype = ctypes.c_int
     l.vsl_logits_local.argtypes = [vp, ctypes.POINTER(vp), ctypes.POINTER(vp), i32, i32, i32, i32, vp]
+    l.vsl_logits_local_ex.restype = ctypes.c_int
+    l.vsl_logits_local_ex.argtypes = [vp, ctypes.POINTER(vp), ctypes.POINTER(vp), i32, i32, i32, i32, vp, vp]
+    l.vsl_tile_stats_floats.restype = sz
+    l.vsl_tile_stats_floats.argtypes = [i32, i32, i32]
+    l.vsl_tile_stats.restype = ctypes.c_int
+    l.vsl_tile_stats.argtypes = [ctypes.POINTER(vp), i32, i32, i32, vp, vp]
     l.vsl_sample_workspace_bytes.restype = sz
     l.vsl_sample_workspace_bytes.argtypes = [i32, i32, i32, i32]
     l.vsl_sample_launches.restype = i32
@@ -116,11 +123,43 @@ def _on_device(device):
     return torch.cuda.device(device)
 
 
-def logits_local(hidden, w_slices, out=None, stream=None):
+def tile_stats_shape(R, S, V_s):
+    """Shape of the tile statistics of R rows of S slices of V_s logits: [R, S * B, 8],
+    B = ceil(V_s / 128) (one record per block of 128 ids; ``include/vsl.h``)."""
+    return (R, S * (-(-V_s // 128)), 8)
+
+
+def _stats_tensor(stats, R, S, V_s, dev):
+    shape = tile_stats_shape(R, S, V_s)
+    if stats is True:
+        return torch.empty(shape, dtype=torch.float32, device=dev)
+    if stats.dtype != torch.float32 or tuple(stats.shape) != shape or not stats.is_contiguous() or stats.device != dev:
+        raise ValueError(f"tile statistics must be a contiguous fp32 {list(shape)} tensor on {dev}")
+    return stats
+
+
+def tile_stats(logits_slices, out=None, stream=None):
+    """Tile statistics of logits already in memory (fp32 [R, S * B, 8]; one read of the logits)."""
+    R, V_s = logits_slices[0].shape
+    S = len(logits_slices)
+    dev = logits_slices[0].device
+    for t in logits_slices:
+        if t.dtype != torch.float32 or not t.is_contiguous() or tuple(t.shape) != (R, V_s) or t.device != dev:
+            raise ValueError("logits slices must be contiguous fp32 [R, V_s] on one device")
+    out = _stats_tensor(True if out is None else out, R, S, V_s, dev)
+    with _on_device(dev):
+        status = lib.vsl_tile_stats(_ptr_array(logits_slices), R, S, V_s, _ptr(out), _stream_handle(stream, dev))
+    _check(status, "vsl_tile_stats")
+    return out
+
+
+def logits_local(hidden, w_slices, out=None, stream=None, tile_stats=None):
     """Vocab-slice projection with no gather: ``out[s] = hidden @ w_slices[s].T`` in fp32.
 
     hidden: bf16 [R, H] CUDA tensor; w_slices: list of bf16 [V_s, H] CUDA tensors.
-    Returns the list of fp32 [R, V_s] slices (``out`` if given).
+    Returns the list of fp32 [R, V_s] slices (``out`` if given).  With ``tile_stats``
+    (True, or an fp32 [R, S * B, 8] tensor to fill) the projection also writes the
+    tile statistics of its logits, and the call returns ``(slices, stats)``.
     """
     R, H = hidden.shape
     S = len(w_slices)
@@ -135,11 +174,12 @@ def logits_local(hidden, w_slices, out=None, stream=None):
     for t in [*w_slices, *out]:
         if t.device != hidden.device:
             raise ValueError("logits_local: every tensor must be on the hidden states' device")
+    stats = None if tile_stats is None or tile_stats is False else _stats_tensor(tile_stats, R, S, V_s, hidden.device)
     with _on_device(hidden.device):
-        status = lib.vsl_logits_local(_ptr(hidden), _ptr_array(w_slices), _ptr_array(out), R, H, S, V_s,
-                                      _stream_handle(stream, hidden.device))
+        status = lib.vsl_logits_local_ex(_ptr(hidden), _ptr_array(w_slices), _ptr_array(out), R, H, S, V_s,
+                                         _ptr(stats), _stream_handle(stream, hidden.device))
     _check(status, "vsl_logits_local")
-    return out
+    return out if stats is None else (out, stats)
 
 
 def make_row_params(temperature, top_k, top_p, request_id, position, device):
@@ -181,7 +221,8 @@ class SampleResult:
         self.processed_topn_logprob = processed_topn_logprob
 
 
-def sample(logits_slices, params, seed, n_logprobs, out=None, stream=None, kept_theta=False, processed=False):
+def sample(logits_slices, params, seed, n_logprobs, out=None, stream=None, kept_theta=False, processed=False,
+           tile_stats=None):
     """Per-row temperature / top-k / top-p / Gumbel-max draw / top-n raw logprobs.
 
     logits_slices: list of fp32 [R, V_s] CUDA tensors (row r = concatenation over slices).
@@ -192,6 +233,9 @@ def sample(logits_slices, params, seed, n_logprobs, out=None, stream=None, kept_
     processed: also return the processed logprobs (log-probabilities of the distribution
     each token was drawn from: the token's [R], the top-n ids / values [R, n]); implies
     kept_theta.
+    tile_stats: the tile statistics of exactly these logits (``logits_local(...,
+    tile_stats=True)`` or ``tile_stats``): greedy and top-k rows then read only the
+    quarters that can hold their candidates.
     """
     R, V_s = logits_slices[0].shape
     S = len(logits_slices)
@@ -219,11 +263,18 @@ def sample(logits_slices, params, seed, n_logprobs, out=None, stream=None, kept_
         out.processed_topn_ids = torch.empty(R, n, dtype=torch.int32, device=dev)[:, :n_logprobs]
         out.processed_topn_logprob = torch.empty(R, n, dtype=torch.float32, device=dev)[:, :n_logprobs]
     extras = None
+    if tile_stats is not None:
+        if not isinstance(tile_stats, torch.Tensor):
+            raise TypeError("tile_stats must be the statistics tensor of these logits")
+        tile_stats = _stats_tensor(tile_stats, R, S, V_s, dev)
+        extras = _Extras()
+        extras.tile_stats = tile_stats.data_ptr()
     if kept_theta:
         if out.kept_theta.dtype != torch.float32 or tuple(out.kept_theta.shape) != (R, 2) or \
                 not out.kept_theta.is_contiguous():
             raise ValueError("kept_theta must be a contiguous fp32 [R, 2] tensor")
-        extras = _Extras(out.kept_theta.data_ptr())
+        extras = extras if extras is not None else _Extras()
+        extras.kept_theta = out.kept_theta.data_ptr()
     if processed:
         extras.processed_logprob = out.processed_logprob.data_ptr()
         if n_logprobs > 0:

@@ -11,7 +11,7 @@ CSRC = os.path.join(PKG_DIR, "csrc")
 LIB_PATH = os.path.join(PKG_DIR, "libvsl.so")
 TEST_SRC = os.path.join(ROOT, "tests", "csrc", "vsl_test_probes.cu")
 TEST_LIB_PATH = os.path.join(ROOT, "tests", "libvsl_test.so")
-SOURCES = ["vsl_api.cu", "vsl_gemm.cu", "vsl_sample.cu", "vsl_verify.cu", "vsl_processed.cu"]
+SOURCES = ["vsl_api.cu", "vsl_gemm.cu", "vsl_sample.cu", "vsl_verify.cu", "vsl_processed.cu", "vsl_tiles.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = [*ARCH, "-lineinfo", "-O3", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden"]
 

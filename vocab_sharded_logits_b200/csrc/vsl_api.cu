@@ -19,6 +19,7 @@ uint32_t* device_error_word() {
 
 namespace {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 }  // namespace
 
 }  // namespace vsl
@@ -40,8 +41,32 @@ const char* vsl_status_string(vsl_status status) {
   return "unknown status";
 }
 
+size_t vsl_tile_stats_floats(int32_t R, int32_t S, int32_t V_s) {
+  if (R <= 0 || S <= 0 || V_s <= 0) return 0;
+  return static_cast<size_t>(R) * static_cast<size_t>(S) * ((static_cast<size_t>(V_s) + 127) / 128) * 8;
+}
+
+vsl_status vsl_tile_stats(const float* const* logits_slices, int32_t R, int32_t S, int32_t V_s, float* tile_stats,
+                          void* stream) {
+  if (logits_slices == nullptr || tile_stats == nullptr) return VSL_ERR_INVALID_ARG;
+  if (R <= 0 || S <= 0 || V_s <= 0) return VSL_ERR_INVALID_ARG;
+  if (S > VSL_MAX_SLICES) return VSL_ERR_UNSUPPORTED;
+  if (V_s % 4 != 0 || !vsl::aligned32(tile_stats)) return VSL_ERR_ALIGNMENT;
+  for (int s = 0; s < S; ++s) {
+    if (logits_slices[s] == nullptr) return VSL_ERR_INVALID_ARG;
+    if (!vsl::aligned16(logits_slices[s])) return VSL_ERR_ALIGNMENT;
+  }
+  const cudaError_t e = vsl::launch_tile_stats(logits_slices, R, S, V_s, tile_stats, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? VSL_OK : VSL_ERR_CUDA;
+}
+
 vsl_status vsl_logits_local(const void* hidden_bf16, const void* const* w_slices_bf16, float* const* logits_slices,
                             int32_t R, int32_t H, int32_t S, int32_t V_s, void* stream) {
+  return vsl_logits_local_ex(hidden_bf16, w_slices_bf16, logits_slices, R, H, S, V_s, nullptr, stream);
+}
+
+vsl_status vsl_logits_local_ex(const void* hidden_bf16, const void* const* w_slices_bf16, float* const* logits_slices,
+                               int32_t R, int32_t H, int32_t S, int32_t V_s, float* tile_stats, void* stream) {
   if (hidden_bf16 == nullptr || w_slices_bf16 == nullptr || logits_slices == nullptr) return VSL_ERR_INVALID_ARG;
   if (R <= 0 || H <= 0 || S <= 0 || V_s <= 0) return VSL_ERR_INVALID_ARG;
   if (S > VSL_MAX_SLICES) return VSL_ERR_UNSUPPORTED;
@@ -51,7 +76,8 @@ vsl_status vsl_logits_local(const void* hidden_bf16, const void* const* w_slices
     if (w_slices_bf16[s] == nullptr || logits_slices[s] == nullptr) return VSL_ERR_INVALID_ARG;
     if (!vsl::aligned16(w_slices_bf16[s]) || !vsl::aligned16(logits_slices[s])) return VSL_ERR_ALIGNMENT;
   }
-  const cudaError_t e = vsl::launch_logits_local(hidden_bf16, w_slices_bf16, logits_slices, R, H, S, V_s,
+  if (tile_stats != nullptr && !vsl::aligned32(tile_stats)) return VSL_ERR_ALIGNMENT;
+  const cudaError_t e = vsl::launch_logits_local(hidden_bf16, w_slices_bf16, logits_slices, R, H, S, V_s, tile_stats,
                                                  static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? VSL_OK : VSL_ERR_CUDA;
 }
@@ -105,13 +131,15 @@ vsl_status vsl_sample_ex(const float* const* logits_slices, int32_t R, int32_t S
   if (p_token == nullptr && (p_topn_ids != nullptr || p_topn != nullptr)) return VSL_ERR_INVALID_ARG;
   if (p_token != nullptr && kept_theta == nullptr) return VSL_ERR_INVALID_ARG;
   if (p_token != nullptr && n_logprobs > 0 && (p_topn_ids == nullptr || p_topn == nullptr)) return VSL_ERR_INVALID_ARG;
+  const float* tile_stats = extras != nullptr ? extras->tile_stats : nullptr;
+  if (tile_stats != nullptr && !vsl::aligned32(tile_stats)) return VSL_ERR_ALIGNMENT;
   if (V > vsl::sample_max_vocab()) return VSL_ERR_UNSUPPORTED;
   int maxc = 0, c = 0, part = 0;
   if (vsl::sample_max_cluster(&maxc) != cudaSuccess) return VSL_ERR_CUDA;
   if (!vsl::sample_geometry_for(V, maxc, &c, &part)) return VSL_ERR_UNSUPPORTED;
   if (workspace_bytes < vsl_sample_workspace_bytes(R, S, V_s, n_logprobs)) return VSL_ERR_WORKSPACE_TOO_SMALL;
   cudaError_t e = vsl::launch_sample(logits_slices, R, S, V_s, params_dev, seed, n_logprobs, token_ids,
-                                     token_logprob, topn_ids, topn_logprob, row_flags, kept_theta,
+                                     token_logprob, topn_ids, topn_logprob, row_flags, kept_theta, tile_stats,
                                      static_cast<cudaStream_t>(stream));
   if (e == cudaSuccess && p_token != nullptr)
     e = vsl::launch_processed(logits_slices, R, S, V_s, params_dev, n_logprobs, token_ids, topn_ids, row_flags,

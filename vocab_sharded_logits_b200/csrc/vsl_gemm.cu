@@ -24,6 +24,14 @@
 //     the next tile's MMAs run; for each batch row a warp writes 32 consecutive
 //     floats (128 coalesced bytes).  They hand the accumulator back through an
 //     mbarrier.
+//   * Optionally the epilogue also writes each batch row's tile statistics
+//     for the 128 vocab rows of the tile (the block): the maximum of each
+//     warp's 32 (its quarter, an integer max of order-preserving keys across
+//     the warp), the block's sum of exp(l - c) and its smallest finite value.
+//     A warp sums its quarter's exps per batch row with a butterfly that
+//     leaves each pair of lanes one row's total (16 shuffles per 16 rows); the
+//     four warps then combine their quarters through shared memory, meeting
+//     at an mbarrier (bounded wait) per 16 rows.
 // Every wait is bounded; a wait that gives up sets the device error word and
 // the CTA drains its own copies, frees its tensor memory and returns.
 #include <cuda.h>
@@ -51,8 +59,29 @@ struct GemmArgs {
   int n_tiles;       // batch tiles
   int k_iters;       // K slabs
   int w_evict_first; // W read once (single batch tile): stream it through L2
+  float* stats;      // optional tile statistics [R][S * m_tiles][8] (nullptr: none)
   uint32_t* err;
 };
+
+constexpr uint32_t kKeyNegInfG = 0x007FFFFFu;  // order-preserving key of -inf
+constexpr uint32_t kKeyPosInfG = 0xFF800000u;  // ... and of +inf
+constexpr int kStatCols = 16;                  // batch rows per epilogue chunk
+// per chunk buffer: [warp quarter][column] max key, min-finite key, sum
+constexpr size_t kStatStageBytes = 4 * kStatCols * 3 * 4;
+
+__device__ __forceinline__ uint32_t okey(float v) {
+  uint32_t b = __float_as_uint(v);
+  b = (b == 0x80000000u) ? 0u : b;
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float okey_value(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 // Shared-memory matrix descriptor for a K-major tile whose rows are 128 bytes,
 // stored as TMA writes it with 128-byte swizzle: 8-row groups 1024 bytes apart.
@@ -81,7 +110,84 @@ __host__ __device__ constexpr int tmem_cols() {
 template <int BN, int STAGES>
 constexpr size_t gemm_smem_bytes() {
   return 1024 /*alignment slack*/ + static_cast<size_t>(STAGES) * (kBM + BN) * kBK * 2 +
-         (2 * STAGES + 5) * 8 + 16;
+         (2 * STAGES + 7) * 8 + 16 + 2 * kStatStageBytes;
+}
+
+// Tile statistics of one epilogue chunk: 16 batch rows (columns n0 ..) of the
+// 128-row vocab block, this warp holding vocab rows 32 q + lane of it in
+// r[0..15].  Called by the four epilogue warps for every chunk, in the same
+// order; returns false if the meeting with the other warps timed out.
+__device__ __forceinline__ bool epilogue_stats(const GemmArgs& a, const uint32_t (&r)[16], bool m_ok, int q, int lane,
+                                            int n0, int slice, int block, uint32_t* stage_all, uint64_t* bars,
+                                            uint32_t chunk) {
+  constexpr float kLog2e = 1.4426950408889634f;
+  uint32_t* stage = stage_all + (chunk & 1u) * (kStatStageBytes / 4);
+  uint32_t* st_max = stage;                        // [4][16]
+  uint32_t* st_min = stage + 4 * kStatCols;        // [4][16]
+  float* st_sum = reinterpret_cast<float*>(stage + 8 * kStatCols);
+  float e[16];
+  uint32_t my_max = 0, my_min = 0xFFFFFFFFu;  // of column `lane` (lanes 0..15)
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const float v = __uint_as_float(r[j]);
+    const uint32_t k = m_ok ? okey(v) : kKeyNegInfG;
+    const uint32_t kq = __reduce_max_sync(0xFFFFFFFFu, k);
+    const uint32_t kf = __reduce_min_sync(0xFFFFFFFFu, m_ok ? k - (kKeyNegInfG + 1u) : 0xFFFFFFFFu);
+    const float cq = (kq > kKeyNegInfG && kq < kKeyPosInfG) ? okey_value(kq) : 0.0f;
+    e[j] = m_ok ? ex2_approx((v - cq) * kLog2e) : 0.0f;
+    my_max = lane == j ? kq : my_max;
+    my_min = lane == j ? kf : my_min;
+  }
+  // butterfly: after the steps over lane bits 4, 3, 2, 1 a lane holds column
+  // 8 b4 + 4 b3 + 2 b2 + b1 summed over 16 lanes; bit 0 pairs the halves
+#pragma unroll
+  for (int h = 8; h >= 1; h >>= 1) {
+    const bool up = (lane & (2 * h)) != 0;
+#pragma unroll
+    for (int u = 0; u < h; ++u) {
+      const float send = up ? e[u] : e[u + h];
+      const float keep = up ? e[u + h] : e[u];
+      e[u] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, 2 * h);
+    }
+  }
+  const float tot = e[0] + __shfl_xor_sync(0xFFFFFFFFu, e[0], 1);
+  const int col = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
+  if ((lane & 1) == 0) st_sum[q * kStatCols + col] = tot;
+  if (lane < kStatCols) {
+    st_max[q * kStatCols + lane] = my_max;
+    st_min[q * kStatCols + lane] = my_min;
+  }
+  __syncwarp();
+  const uint32_t bar = smem_u32(&bars[chunk & 1u]);
+  if (lane == 0) mbar_arrive(bar);
+  if (!mbar_wait_bounded(bar, (chunk >> 1) & 1u)) return false;
+  // warp q writes the records of columns 4 q .. 4 q + 3
+  if (lane < 4) {
+    const int cc = 4 * q + lane;
+    const int n = n0 + cc;
+    uint32_t kq[4], kb = 0, kf = 0xFFFFFFFFu;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      kq[w] = st_max[w * kStatCols + cc];
+      kb = max(kb, kq[w]);
+      kf = min(kf, st_min[w * kStatCols + cc]);
+    }
+    const float c = (kb > kKeyNegInfG && kb < kKeyPosInfG) ? okey_value(kb) : 0.0f;
+    float sum = 0.0f;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const float sw = st_sum[w * kStatCols + cc];
+      const float cw = (kq[w] > kKeyNegInfG && kq[w] < kKeyPosInfG) ? okey_value(kq[w]) : 0.0f;
+      sum += sw == 0.0f ? 0.0f : sw * ex2_approx((cw - c) * kLog2e);
+    }
+    if (n < a.R) {
+      float4* rec = reinterpret_cast<float4*>(
+          a.stats + ((static_cast<size_t>(n) * a.S + slice) * a.m_tiles + block) * 8);
+      rec[0] = make_float4(okey_value(kq[0]), okey_value(kq[1]), okey_value(kq[2]), okey_value(kq[3]));
+      rec[1] = make_float4(sum, kf == 0xFFFFFFFFu ? INFINITY : okey_value(kf + kKeyNegInfG + 1u), 0.0f, 0.0f);
+    }
+  }
+  return true;
 }
 
 template <int BN, int STAGES>
@@ -98,8 +204,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) logits_local_kernel(const __g
   uint64_t* acc_full = empty + STAGES;   // [2]: MMA -> epilogue
   uint64_t* acc_empty = acc_full + 2;    // [2]: epilogue (4 warps) -> MMA
   uint64_t* done = acc_empty + 2;        // every MMA of the CTA has completed
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  uint64_t* stat_bar = done + 1;         // [2]: the epilogue's 4 warps staged a chunk's statistics
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(stat_bar + 2);
   volatile uint32_t* abort_flag = tmem_slot + 1;
+  uint32_t* stat_stage = tmem_slot + 4;  // [2][kStatStageBytes / 4]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -115,6 +223,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) logits_local_kernel(const __g
       mbar_init(smem_u32(&acc_empty[b]), 4);
     }
     mbar_init(smem_u32(done), 1);
+    mbar_init(smem_u32(&stat_bar[0]), 4);
+    mbar_init(smem_u32(&stat_bar[1]), 4);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -197,6 +307,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) logits_local_kernel(const __g
     // ---------------- epilogue: TMEM -> registers -> global fp32, one tile behind the MMAs
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     int i = 0;
+    uint32_t chunk = 0;      // statistics chunks so far (stage buffer and mbarrier phase)
+    bool stat_ok = true;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++i) {
       const int b = i & 1;
       const bool ok = mbar_wait_bounded(smem_u32(&acc_full[b]), (i >> 1) & 1);
@@ -224,6 +336,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) logits_local_kernel(const __g
           for (int j = 0; j < 16; ++j) {
             const int n = n0 + c + j;
             if (n < a.R) out[static_cast<size_t>(n) * a.V_s + m] = __uint_as_float(r[j]);
+          }
+        }
+        if (a.stats != nullptr && stat_ok) {
+          stat_ok = epilogue_stats(a, r, m_ok, q, lane, n0 + c, slice, mt % a.m_tiles, stat_stage, stat_bar, chunk);
+          ++chunk;
+          if (!stat_ok) {
+            if (lane == 0) atomicOr(a.err, kErrGemmEpilogue);
+            *abort_flag = 1;
           }
         }
       }
@@ -317,9 +437,10 @@ cudaError_t launch_bn(GemmArgs& args, const void* hidden, const void* const* w, 
 }  // namespace
 
 cudaError_t launch_logits_local(const void* hidden, const void* const* w_slices, float* const* logits,
-                                int R, int H, int S, int V_s, cudaStream_t stream) {
+                                int R, int H, int S, int V_s, float* stats, cudaStream_t stream) {
   if (!get_encoder()) return cudaErrorNotSupported;
   GemmArgs args{};
+  args.stats = stats;
   for (int s = 0; s < S; ++s) args.out[s] = logits[s];
   args.R = R;
   args.H = H;

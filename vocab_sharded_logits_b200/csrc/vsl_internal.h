@@ -12,16 +12,22 @@ namespace vsl {
 // Device address of the library's error word on the current device.
 uint32_t* device_error_word();
 
-// Launch the vocab-slice projection.  Arguments already validated.
+// Launch the vocab-slice projection (stats: optional tile statistics, or
+// nullptr).  Arguments already validated.
 cudaError_t launch_logits_local(const void* hidden, const void* const* w_slices,
                                 float* const* logits, int R, int H, int S, int V_s,
-                                cudaStream_t stream);
+                                float* stats, cudaStream_t stream);
+
+// Launch the tile statistics of logits in memory.  Arguments already validated.
+cudaError_t launch_tile_stats(const float* const* logits, int R, int S, int V_s, float* stats,
+                              cudaStream_t stream);
 
 // Launch the sampler.  Arguments already validated.
 cudaError_t launch_sample(const float* const* logits, int R, int S, int V_s,
                           const vsl_row_params* params, uint64_t seed, int n_logprobs,
                           int32_t* token_ids, float* token_logprob, int32_t* topn_ids,
-                          float* topn_logprob, uint32_t* row_flags, float* kept_theta, cudaStream_t stream);
+                          float* topn_logprob, uint32_t* row_flags, float* kept_theta,
+                          const float* tile_stats, cudaStream_t stream);
 
 // Launch the processed-logprobs pass (after the sampler, same stream).
 cudaError_t launch_processed(const float* const* logits, int R, int S, int V_s, const vsl_row_params* params,

@@ -117,6 +117,8 @@ struct SampleArgs {
   float* topn_logprob;
   uint32_t* row_flags;
   float* kept_theta;  // optional [R][2]: theta_k, theta_p of each row (nullptr: not written)
+  const float* tile_stats;  // streaming kernel: optional records [R][S * tile_blocks][8] (nullptr: none)
+  int tile_blocks;          // blocks of 128 ids per slice
   uint32_t* err;
   unsigned long long seed;
   int R, S, V_s, V, C, part, n_logprobs;
@@ -3116,7 +3118,7 @@ int sample_launches(int R, long long V) {
 cudaError_t launch_sample(const float* const* logits, int R, int S, int V_s, const vsl_row_params* params,
                           uint64_t seed, int n_logprobs, int32_t* token_ids, float* token_logprob,
                           int32_t* topn_ids, float* topn_logprob, uint32_t* row_flags, float* kept_theta,
-                          cudaStream_t stream) {
+                          const float* tile_stats, cudaStream_t stream) {
   DeviceState* d = nullptr;
   cudaError_t e = current_device_state(&d);
   if (e != cudaSuccess) return e;
@@ -3142,6 +3144,14 @@ cudaError_t launch_sample(const float* const* logits, int R, int S, int V_s, con
   const int sms = d->sms;
   SampleArgs sa = a;
   stream_geometry(R, a.V, sms, &sa.C, &sa.part);
+  const int tile_blocks = (V_s + 127) / 128;
+  if (tile_stats != nullptr && static_cast<long long>(S) * tile_blocks <= kStreamCap) {
+    // tile mode: each greedy / top-k row reads its records and a few quarters on one CTA
+    sa.tile_stats = tile_stats;
+    sa.tile_blocks = tile_blocks;
+    sa.C = 1;
+    sa.part = a.V;
+  }
   a.C = c;
   a.part = part;
   const void* fs = reinterpret_cast<const void*>(stream_kernel);

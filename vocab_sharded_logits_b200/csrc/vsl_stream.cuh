@@ -220,6 +220,121 @@ __device__ __forceinline__ void stream_scan(const float4* st4, int nq, uint32_t 
     }
 }
 
+// Tile mode (a greedy or top-k row on one CTA, with the tile statistics of its
+// logits): the row's statistics come from its records, the cut from the block
+// maxima, and only the 32-id quarters whose largest raw value reaches the cut
+// are read.  The R-th largest block maximum t0 is at most the row's R-th
+// largest logit (R blocks hold a value >= t0), and x = fl(l / T) is
+// non-decreasing in l, so every top-R logit and every value that scales to the
+// same x as the R-th lies in a quarter whose maximum is >= the cut
+// stream_floor(t0).  Lists every logit >= the cut and returns the cut;
+// `qkeys` (the idle ring, 4 * S * B keys) holds the quarter maxima.  A list
+// that overflows shows in the list count (the row is deferred).
+struct TileScan {
+  ScanStats st;
+  uint32_t cut;
+};
+__device__ __forceinline__ TileScan stream_tiles(const Ctx& cx, const SampleArgs& a, uint32_t R, uint32_t* qkeys) {
+  constexpr float kLog2e = 1.4426950408889634f;
+  ScanStats st{0u, 0xFFFFFFFFu, 0xFFFFFFFFu, kScanNoMax, 0.0f};
+  SharedHeader* H = cx.H;
+  const int B = a.tile_blocks;
+  const int SB = a.S * B;
+  const float4* rec = reinterpret_cast<const float4*>(a.tile_stats) + static_cast<size_t>(cx.row) * SB * 2;
+  // records: statistics, the block maxima as list entries, the quarter maxima
+  for (int i = threadIdx.x; i < SB; i += kThreads) {
+    const float4 qm = __ldg(rec + 2 * i);
+    const float4 sm = __ldg(rec + 2 * i + 1);
+    const uint4 k = make_uint4(fkey(qm.x), fkey(qm.y), fkey(qm.z), fkey(qm.w));
+    reinterpret_cast<uint4*>(qkeys)[i] = k;
+    const uint32_t kb = max(max(k.x, k.y), max(k.z, k.w));
+    cx.list[i] = (static_cast<uint64_t>(~kb) << 32) | static_cast<uint32_t>(i);
+    const uint32_t kmin = fkey(sm.y);
+    st.kmf = min(st.kmf, key_finite(kmin) ? kmin - (kKeyNegInf + 1u) : 0xFFFFFFFFu);
+    // the block's sum runs against its maximum c (0 when that is not finite)
+    if (kb > st.kmax) {
+      st.kmax = kb;
+      if (key_finite(kb)) {
+        const float mn = key_value(kb);
+        st.s = st.s == 0.0f ? 0.0f : st.s * fast_exp2((st.m - mn) * kLog2e);
+        st.m = mn;
+      }
+    }
+    if (key_finite(kb)) st.s += sm.x * fast_exp2((key_value(kb) - st.m) * kLog2e);
+    else if (sm.x != 0.0f) st.s += sm.x;  // NaN or +inf: the row is flagged
+  }
+  if (threadIdx.x == 0) H->list_count = static_cast<uint32_t>(SB);
+  __syncthreads();
+  uint32_t left;
+  const uint32_t cut = stream_compact(cx, R, 0u, 64, left);  // 0 (every quarter) when SB <= R
+  __syncthreads();
+  if (threadIdx.x == 0) H->list_count = 0;
+  __syncthreads();
+  // each warp compacts the indices of its quarters that reach the cut in place
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int NQ = 4 * SB;
+  const int per = ((NQ + kWarps - 1) / kWarps + 31) & ~31;
+  const int q0 = min(warp * per, NQ), q1 = min(q0 + per, NQ);
+  uint32_t nsel = 0;
+  for (int j = q0; j < q1; j += 32) {
+    const bool pick = j + lane < q1 && qkeys[j + lane] >= cut;
+    const uint32_t m = __ballot_sync(0xFFFFFFFFu, pick);
+    if (pick) qkeys[q0 + nsel + __popc(m & ((1u << lane) - 1u))] = static_cast<uint32_t>(j + lane);
+    nsel += __popc(m);
+    __syncwarp();
+  }
+  // gather: 8 lanes per quarter (one float4 each), 4 quarters per load, 4 loads in flight
+  const uint32_t below = (1u << lane) - 1u;
+  for (uint32_t u = 0; u < nsel; u += 16) {
+    float4 v[4];
+    uint32_t gid[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const uint32_t qi = u + 4u * w + (lane >> 3);
+      gid[w] = 0xFFFFFFFFu;
+      v[w] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (qi < nsel) {
+        const uint32_t j = qkeys[q0 + qi];
+        const int blk = static_cast<int>(j >> 2);
+        const int sl = blk / B;
+        const int col = (blk - sl * B) * 128 + static_cast<int>(j & 3u) * 32 + 4 * (lane & 7);
+        if (col < a.V_s) {
+          gid[w] = static_cast<uint32_t>(sl * a.V_s + col);
+          v[w] = ldg_stream4(a.slices[sl] + static_cast<size_t>(cx.row) * a.V_s + col);
+        }
+      }
+    }
+    uint32_t mask[4][4], total = 0;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const float e[4] = {v[w].x, v[w].y, v[w].z, v[w].w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        mask[w][i] = __ballot_sync(0xFFFFFFFFu, gid[w] != 0xFFFFFFFFu && fkey(e[i]) >= cut);
+        total += __popc(mask[w][i]);
+      }
+    }
+    if (total == 0) continue;
+    uint32_t base = 0;
+    if (lane == 0) base = atomicAdd(&H->list_count, total);
+    base = __shfl_sync(0xFFFFFFFFu, base, 0);
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const float e[4] = {v[w].x, v[w].y, v[w].z, v[w].w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t idx = base + __popc(mask[w][i] & below);
+        if (((mask[w][i] >> lane) & 1u) && idx < static_cast<uint32_t>(kStreamCap))
+          cx.list[idx] = (static_cast<uint64_t>(~fkey(e[i])) << 32) | (gid[w] + i);
+        base += __popc(mask[w][i]);
+      }
+    }
+  }
+  __syncthreads();
+  return TileScan{st, cut};
+}
+
 // One more streaming pass over this CTA's part [g0, g0 + n), continuing the
 // ring where the previous pass left it (`cg`: chunks streamed so far, which
 // fixes each stage's mbarrier phase).  `body(st4, nq, gid)` scans one stage
@@ -505,6 +620,7 @@ __global__ void __launch_bounds__(kThreads, 2) stream_kernel(const __grid_consta
   const bool k_on = !greedy && prm.top_k > 0 && prm.top_k < a.V;
   uint32_t R = a.n_logprobs > 0 ? static_cast<uint32_t>(a.n_logprobs) : 1u;
   if (k_on) R = max(R, static_cast<uint32_t>(prm.top_k));
+  const bool tiles = a.tile_stats != nullptr && a.C == 1 && (greedy || k_on);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStreamStages; ++s) mbar_init(smem_u32(&H->ring_bar[s]), 1);
@@ -517,7 +633,7 @@ __global__ void __launch_bounds__(kThreads, 2) stream_kernel(const __grid_consta
   const uint64_t pol = policy_evict_first();
   const int g0 = static_cast<int>(cx.g0);
   int s_issue = 0;
-  if (threadIdx.x == 0)
+  if (threadIdx.x == 0 && !tiles)
     for (int c = 0; c < min(nch, kStreamStages - 1); ++c) stream_issue(a, cx.row, g0, n, c, s_issue, ring, H->ring_bar, pol);
 
   constexpr float kLog2e = 1.4426950408889634f;
@@ -543,7 +659,12 @@ __global__ void __launch_bounds__(kThreads, 2) stream_kernel(const __grid_consta
   // row is deferred.
   int next_issue = min(nch, kStreamStages - 1);  // thread 0: chunks issued so far
   int step = 1;
-  for (int c = 0; c < nch;) {
+  if (tiles) {
+    const TileScan ts = stream_tiles(cx, a, R, reinterpret_cast<uint32_t*>(ring));
+    st = ts.st;
+    thr = ts.cut;
+  }
+  for (int c = 0; c < (tiles ? 0 : nch);) {
     const int cur = step;  // this round's chunks (a compaction below may widen the next rounds)
     // refill every stage whose chunk all threads have scanned (the last barrier has passed)
     if (threadIdx.x == 0)
