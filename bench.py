@@ -304,6 +304,49 @@ def _events(n):
     return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
 
 
+def _tile_rows(T, k, V):
+    """Rows the sampler's tile mode takes: greedy, or 0 < top_k <= 1024 (below V)."""
+    T = np.asarray(T, np.float32)
+    k = np.asarray(k, np.int64)
+    return (T == 0) | ((k > 0) & (k < V) & (k <= 1024))
+
+
+def _uses_tiles(w, T, k):
+    """The step requests tile statistics when some row can use them (and the
+    vocabulary has at most 4096 blocks of 128)."""
+    return bool(_tile_rows(T, k, w.V).any()) and w.S * (-(-w.V_s // 128)) <= 4096
+
+
+def _sampler_read_bytes(w, T, k, stats):
+    """Algorithmic bytes one sampler call reads: every row outside the tile mode
+    reads its V logits; a tile-mode row reads its records (S * B * 32 bytes)
+    and the 32-logit quarters whose largest x reaches fl(t0 / T), t0 the R-th
+    largest block maximum, R = max(n, k) (greedy: max(n, 1)).  Counted from the
+    records with torch on the device (the kernel's cut can sit a few floats
+    lower, where the temperature maps neighbours to one x: an undercount of a
+    few quarters at most)."""
+    tile = _tile_rows(T, k, w.V)
+    full = int((~tile).sum()) * w.V * 4
+    if stats is None or not tile.any():
+        return w.R * w.V * 4
+    dev = stats.device
+    rows = torch.from_numpy(np.flatnonzero(tile)).to(dev)
+    st = stats[rows]
+    SB = st.shape[1]
+    Tt = torch.as_tensor(np.asarray(T, np.float32)[tile], device=dev)
+    kt = torch.as_tensor(np.asarray(k, np.int64)[tile], device=dev)
+    n = max(w.n_logprobs, 1)
+    r_sel = torch.where(Tt == 0, torch.full_like(kt, n), torch.clamp(kt, min=w.n_logprobs))
+    qmax = st[..., :4]
+    bmax = qmax.amax(-1).sort(dim=1, descending=True).values
+    t0 = bmax.gather(1, (r_sel - 1).clamp(max=SB - 1)[:, None]).squeeze(1)
+    t0 = torch.where(r_sel > SB, torch.full_like(t0, -float("inf")), t0)
+    scale = torch.where(Tt == 0, torch.ones_like(Tt), Tt)
+    sel = (qmax / scale[:, None, None]) >= (t0 / scale)[:, None, None]
+    quarters = int(sel.sum())
+    return full + int(tile.sum()) * SB * 32 + quarters * 128
+
+
 def measure_config(w, dev, world, rank, steps, warmup, peaks):
     """One workload on this rank: the timed steps (projection + sampler, events per
     kernel on the launching stream), the sampler alone with L2 flushed, the end-to-end
@@ -324,10 +367,23 @@ def measure_config(w, dev, world, rank, steps, warmup, peaks):
     out = vsl.SampleResult(torch.empty(w.R, dtype=torch.int32, device=dev), torch.empty(w.R, device=dev),
                            torch.empty(w.R, n, dtype=torch.int32, device=dev), torch.empty(w.R, n, device=dev),
                            torch.empty(w.R, dtype=torch.int32, device=dev))
+    # tile statistics, when some row can use them: the projection writes them
+    # every step and the sampler reads them; for the peaked workload, whose
+    # sampler reads its own synthetic logits, the records of those logits
+    # (written once) stand in for the epilogue's
+    tiles = _uses_tiles(w, T, k)
+    stats = torch.empty(vsl.tile_stats_shape(w.R, w.S, w.V_s), device=dev) if tiles else None
+    samp_stats = vsl.tile_stats(samp_in) if tiles and samp_in is not logits else stats
+
+    def project(hid, stream):
+        vsl.logits_local(hid, ws, out=logits, stream=stream, tile_stats=stats)
+
+    def sample(prm, seed, res, stream):
+        vsl.sample(samp_in, prm, seed, n, out=res, stream=stream, tile_stats=samp_stats)
 
     def step(seed):
-        vsl.logits_local(hidden, ws, out=logits, stream=stream)
-        vsl.sample(samp_in, params, seed, n, out=out, stream=stream)
+        project(hidden, stream)
+        sample(params, seed, out, stream)
 
     for i in range(warmup):
         step(i)
@@ -340,9 +396,9 @@ def measure_config(w, dev, world, rank, steps, warmup, peaks):
     for i in range(steps):
         a, b, c = ev[i]
         a.record(stream)
-        vsl.logits_local(hidden, ws, out=logits, stream=stream)
+        project(hidden, stream)
         b.record(stream)
-        vsl.sample(samp_in, params, 1000 + i, n, out=out, stream=stream)
+        sample(params, 1000 + i, out, stream)
         c.record(stream)
     t1.record(stream)
     torch.cuda.synchronize()
@@ -357,7 +413,7 @@ def measure_config(w, dev, world, rank, steps, warmup, peaks):
         flush.fill_(float(i))
         e0, e1 = _events(2)
         e0.record(stream)
-        vsl.sample(samp_in, params, 2000 + i, n, out=out, stream=stream)
+        sample(params, 2000 + i, out, stream)
         e1.record(stream)
         torch.cuda.synchronize()
         s_times.append(e0.elapsed_time(e1))
@@ -396,8 +452,8 @@ def measure_config(w, dev, world, rank, steps, warmup, peaks):
                 dev_in[b].copy_(pin_in[b], non_blocking=True)
                 ev_in[b].record(copy_stream)
             stream.wait_event(ev_in[b])
-            vsl.logits_local(hid, ws, out=logits, stream=stream)
-            vsl.sample(samp_in, prm, first_seed + i, n, out=res, stream=stream)
+            project(hid, stream)
+            sample(prm, first_seed + i, res, stream)
             ev_done[b].record(stream)
             with torch.cuda.stream(copy_stream):
                 copy_stream.wait_event(ev_done[b])
@@ -419,7 +475,7 @@ def measure_config(w, dev, world, rank, steps, warmup, peaks):
 
     gemm_bytes = w.V * w.H * 2 + w.R * w.H * 2 + w.R * w.V * 4
     gemm_flops = 2.0 * w.R * w.H * w.V
-    samp_bytes = w.R * w.V * 4
+    samp_bytes = _sampler_read_bytes(w, T, k, samp_stats)
     ridge = tf_peak * 1e12 / (hbm_peak * 1e9)
     gemm_hbm = gemm_flops / gemm_bytes < ridge
     gemm_tf = gemm_flops / (gemm_ms / 1e3) / 1e12
@@ -434,13 +490,16 @@ def measure_config(w, dev, world, rank, steps, warmup, peaks):
         "gemm_frac": (gemm_gbs / hbm_peak) if gemm_hbm else (gemm_tf / tf_peak),
         "gemm_frac_of": "measured HBM copy GB/s" if gemm_hbm else "measured bf16 burst TF/s",
         "sample_ms_in_step": samp_ms, "sample_ms_cold_l2": samp_cold_ms,
+        "sampler_mode": "tile statistics" if tiles else "full rows",
+        "sampler_read_bytes": samp_bytes,
         "sampler_hbm_gbs_cold_l2": samp_gbs_cold, "sampler_frac_cold_l2": samp_gbs_cold / hbm_peak,
+        "sampler_full_rows_equiv_gbs": w.R * w.V * 4 / (samp_cold_ms / 1e3) / 1e9,
         "sampler_rows_per_s_cold_l2": w.R / (samp_cold_ms / 1e3),
     }
     state = {"samp_in": samp_in, "params": params, "T": T, "k": k, "p": p, "req": req + rank * w.requests,
              "pos": pos, "total_ms": total_ms, "gemm_ms": gemm_ms, "samp_ms": samp_ms, "e2e_ms": e2e_ms,
              "h2d": in_bytes, "d2h": out_words * 4, "gemm_bytes": gemm_bytes, "gemm_flops": gemm_flops,
-             "samp_bytes": samp_bytes, "gemm_hbm": gemm_hbm, "out": out}
+             "samp_bytes": samp_bytes, "gemm_hbm": gemm_hbm, "out": out, "samp_stats": samp_stats}
     return summary, state
 
 
@@ -463,7 +522,7 @@ def run_gpu(args, w):
         torch.cuda.synchronize()
 
     # the GPU's draw on the headline's logits for the bench-side parity count
-    parity_out = vsl.sample(st["samp_in"], st["params"], PARITY_SEED, w.n_logprobs)
+    parity_out = vsl.sample(st["samp_in"], st["params"], PARITY_SEED, w.n_logprobs, tile_stats=st["samp_stats"])
     gpu_tokens = parity_out.token_ids.cpu().numpy()
     logits_host = None
     if rank == 0 and world == 1 and not args.skip_cpu:
@@ -542,10 +601,11 @@ def run_sampler_only(args, w):
     del logits
     T, k, p, req, pos = W.row_params(w)
     params = vsl.make_row_params(T, k, p, req, pos, dev)
-    out = vsl.sample(slices, params, 0, w.n_logprobs)
+    stats = vsl.tile_stats(slices) if args.tile_stats else None
+    out = vsl.sample(slices, params, 0, w.n_logprobs, tile_stats=stats)
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
     for i in range(args.warmup):
-        vsl.sample(slices, params, i, w.n_logprobs, out=out)
+        vsl.sample(slices, params, i, w.n_logprobs, out=out, tile_stats=stats)
     clocks = ClockSampler(0)
     clocks.start()
     times = []
@@ -556,7 +616,7 @@ def run_sampler_only(args, w):
         flush.fill_(float(i))
         e0, e1 = _events(2)
         e0.record()
-        vsl.sample(slices, params, 100 + i, w.n_logprobs, out=out)
+        vsl.sample(slices, params, 100 + i, w.n_logprobs, out=out, tile_stats=stats)
         e1.record()
         torch.cuda.synchronize()
         if i < args.steps:
@@ -564,14 +624,15 @@ def run_sampler_only(args, w):
         i += 1
     clk = clocks.stop()
     ms = statistics.median(times)
-    nbytes = w.R * w.V * 4
+    nbytes = _sampler_read_bytes(w, T, k, stats)
     print(json.dumps({"metric": f"sampler rows/sec ({w.name}, V={w.V}, L2 flushed)", "value": w.R / (ms / 1e3),
                       "unit": "rows/s", "ms": ms, "hbm_gbs": nbytes / (ms / 1e3) / 1e9,
                       "roofline": {"bound": "hbm", "achieved": nbytes / (ms / 1e3) / 1e9, "peak": hbm_peak,
                                    "unit": "GB/s", "frac": nbytes / (ms / 1e3) / 1e9 / hbm_peak,
                                    "peak_source": peak_kind},
-                      "clocks": clk,
-                      "config": {"workload": w.name, "rows": w.R, "vocab": w.V, "slices": w.S}}), flush=True)
+                      "clocks": clk, "read_bytes": nbytes,
+                      "config": {"workload": w.name, "rows": w.R, "vocab": w.V, "slices": w.S,
+                                 "tile_statistics": bool(args.tile_stats)}}), flush=True)
     return 0
 
 
@@ -628,6 +689,8 @@ def main():
     ap.add_argument("--no-per-config", action="store_true", help="measure the headline workload only")
     ap.add_argument("--sampler-only", action="store_true",
                     help="time the sampler alone on the workload's synthetic logits (profiling aid)")
+    ap.add_argument("--tile-stats", action="store_true",
+                    help="with --sampler-only: give the sampler the tile statistics of its logits")
     ap.add_argument("--gemm-only", action="store_true",
                     help="time the projection alone, 10 back-to-back launches per timing (profiling aid)")
     args = ap.parse_args()

@@ -20,18 +20,21 @@
 //     one of two 128 x BN fp32 accumulators in tensor memory (tile i uses
 //     accumulator i mod 2), releasing each ring slot with tcgen05.commit.
 //   * Warps 2..5 read the accumulator of the previous tile with tcgen05.ld
-//     (one TMEM lane = one vocab row per thread) and store fp32 logits while
-//     the next tile's MMAs run; for each batch row a warp writes 32 consecutive
-//     floats (128 coalesced bytes).  They hand the accumulator back through an
-//     mbarrier.
+//     (one TMEM lane = one vocab row per thread), 16 batch rows at a time,
+//     while the next tile's MMAs run, and hand the accumulator back through an
+//     mbarrier once its last columns are in registers.  Each chunk of 16 batch
+//     rows x 128 vocab rows is staged in shared memory in the output's layout
+//     ([batch row][vocab]) and written with one TMA store (clipped at the
+//     slice's edges).
 //   * Optionally the epilogue also writes each batch row's tile statistics
-//     for the 128 vocab rows of the tile (the block): the maximum of each
-//     warp's 32 (its quarter, an integer max of order-preserving keys across
-//     the warp), the block's sum of exp(l - c) and its smallest finite value.
-//     A warp sums its quarter's exps per batch row with a butterfly that
-//     leaves each pair of lanes one row's total (16 shuffles per 16 rows); the
-//     four warps then combine their quarters through shared memory, meeting
-//     at an mbarrier (bounded wait) per 16 rows.
+//     for the 128 vocab rows of the tile (the block) from the staged chunk:
+//     each of the 128 epilogue threads reads 16 consecutive logits of one
+//     (batch row, quarter, half) from shared memory (maximum, smallest finite
+//     value, sum of exp(l - c)), and three shuffle steps among the 8 threads of
+//     a batch row give the quarter maxima and the block's sum and minimum.
+//   * The four epilogue warps meet at two mbarriers per chunk (bounded waits):
+//     the chunk is staged, and the buffer is free again (read by the
+//     statistics and by the store).
 // Every wait is bounded; a wait that gives up sets the device error word and
 // the CTA drains its own copies, frees its tensor memory and returns.
 #include <cuda.h>
@@ -61,22 +64,17 @@ struct GemmArgs {
   int w_evict_first; // W read once (single batch tile): stream it through L2
   float* stats;      // optional tile statistics [R][S * m_tiles][8] (nullptr: none)
   uint32_t* err;
+  CUtensorMap tmap_out[VSL_MAX_SLICES];  // fp32 [R][V_s] outputs, box 128 x 16
 };
 
-constexpr uint32_t kKeyNegInfG = 0x007FFFFFu;  // order-preserving key of -inf
-constexpr uint32_t kKeyPosInfG = 0xFF800000u;  // ... and of +inf
-constexpr int kStatCols = 16;                  // batch rows per epilogue chunk
-// per chunk buffer: [warp quarter][column] max key, min-finite key, sum
-constexpr size_t kStatStageBytes = 4 * kStatCols * 3 * 4;
+constexpr int kChunk = 16;                                      // batch rows per epilogue chunk
+constexpr uint32_t kChunkBytes = kChunk * kBM * 4;              // one staged chunk (8 KB)
+// staged chunk buffers: two, except for BN = 64, whose CTAs must fit two per SM
+template <int BN>
+__host__ __device__ constexpr int chunk_buffers() {
+  return BN == 64 ? 1 : 2;
+}
 
-__device__ __forceinline__ uint32_t okey(float v) {
-  uint32_t b = __float_as_uint(v);
-  b = (b == 0x80000000u) ? 0u : b;
-  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-}
-__device__ __forceinline__ float okey_value(uint32_t k) {
-  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
-}
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -110,84 +108,57 @@ __host__ __device__ constexpr int tmem_cols() {
 template <int BN, int STAGES>
 constexpr size_t gemm_smem_bytes() {
   return 1024 /*alignment slack*/ + static_cast<size_t>(STAGES) * (kBM + BN) * kBK * 2 +
-         (2 * STAGES + 7) * 8 + 16 + 2 * kStatStageBytes;
+         static_cast<size_t>(chunk_buffers<BN>()) * kChunkBytes + (2 * STAGES + 9) * 8 + 16;
 }
 
-// Tile statistics of one epilogue chunk: 16 batch rows (columns n0 ..) of the
-// 128-row vocab block, this warp holding vocab rows 32 q + lane of it in
-// r[0..15].  Called by the four epilogue warps for every chunk, in the same
-// order; returns false if the meeting with the other warps timed out.
-__device__ __forceinline__ bool epilogue_stats(const GemmArgs& a, const uint32_t (&r)[16], bool m_ok, int q, int lane,
-                                            int n0, int slice, int block, uint32_t* stage_all, uint64_t* bars,
-                                            uint32_t chunk) {
+// Tile statistics of one staged chunk (16 batch rows x 128 vocab rows,
+// [row][vocab], -inf past the slice's end) by the 128 epilogue threads: thread
+// e takes batch row e / 8 and the 16 logits of its half (e & 1) of quarter
+// (e >> 1) & 3; the 8 threads of a row are consecutive lanes.
+__device__ __forceinline__ void chunk_stats(const GemmArgs& a, const float* stage, int e, int lane, int n_first,
+                                            int slice, int block) {
   constexpr float kLog2e = 1.4426950408889634f;
-  uint32_t* stage = stage_all + (chunk & 1u) * (kStatStageBytes / 4);
-  uint32_t* st_max = stage;                        // [4][16]
-  uint32_t* st_min = stage + 4 * kStatCols;        // [4][16]
-  float* st_sum = reinterpret_cast<float*>(stage + 8 * kStatCols);
-  float e[16];
-  uint32_t my_max = 0, my_min = 0xFFFFFFFFu;  // of column `lane` (lanes 0..15)
+  const int row = e >> 3, sub = e & 7;
+  const float4* src = reinterpret_cast<const float4*>(stage + row * kBM + sub * 16);
+  // the four float4 in an order rotated by sub (fewer bank conflicts among the
+  // 8 threads of a phase); the statistics do not depend on the order
+  float v[16];
 #pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    const float v = __uint_as_float(r[j]);
-    const uint32_t k = m_ok ? okey(v) : kKeyNegInfG;
-    const uint32_t kq = __reduce_max_sync(0xFFFFFFFFu, k);
-    const uint32_t kf = __reduce_min_sync(0xFFFFFFFFu, m_ok ? k - (kKeyNegInfG + 1u) : 0xFFFFFFFFu);
-    const float cq = (kq > kKeyNegInfG && kq < kKeyPosInfG) ? okey_value(kq) : 0.0f;
-    e[j] = m_ok ? ex2_approx((v - cq) * kLog2e) : 0.0f;
-    my_max = lane == j ? kq : my_max;
-    my_min = lane == j ? kf : my_min;
+  for (int j = 0; j < 4; ++j) {
+    const float4 x = src[(j + sub) & 3];
+    v[4 * j] = x.x;
+    v[4 * j + 1] = x.y;
+    v[4 * j + 2] = x.z;
+    v[4 * j + 3] = x.w;
   }
-  // butterfly: after the steps over lane bits 4, 3, 2, 1 a lane holds column
-  // 8 b4 + 4 b3 + 2 b2 + b1 summed over 16 lanes; bit 0 pairs the halves
+  float mx = v[0], mn = INFINITY;
 #pragma unroll
-  for (int h = 8; h >= 1; h >>= 1) {
-    const bool up = (lane & (2 * h)) != 0;
-#pragma unroll
-    for (int u = 0; u < h; ++u) {
-      const float send = up ? e[u] : e[u + h];
-      const float keep = up ? e[u + h] : e[u];
-      e[u] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, 2 * h);
-    }
+  for (int i = 0; i < 16; ++i) {
+    mx = fmaxf(mx, v[i]);
+    mn = fminf(mn, isfinite(v[i]) ? v[i] : INFINITY);
   }
-  const float tot = e[0] + __shfl_xor_sync(0xFFFFFFFFu, e[0], 1);
-  const int col = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
-  if ((lane & 1) == 0) st_sum[q * kStatCols + col] = tot;
-  if (lane < kStatCols) {
-    st_max[q * kStatCols + lane] = my_max;
-    st_min[q * kStatCols + lane] = my_min;
-  }
-  __syncwarp();
-  const uint32_t bar = smem_u32(&bars[chunk & 1u]);
-  if (lane == 0) mbar_arrive(bar);
-  if (!mbar_wait_bounded(bar, (chunk >> 1) & 1u)) return false;
-  // warp q writes the records of columns 4 q .. 4 q + 3
-  if (lane < 4) {
-    const int cc = 4 * q + lane;
-    const int n = n0 + cc;
-    uint32_t kq[4], kb = 0, kf = 0xFFFFFFFFu;
+  mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 1));  // the quarter's maximum
+  mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, 1));
+  float bm = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 2));
+  bm = fmaxf(bm, __shfl_xor_sync(0xFFFFFFFFu, bm, 4));  // the block's maximum
+  mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, 2));
+  mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, 4));
+  const float c = isfinite(bm) ? bm : 0.0f;
+  float sum = 0.0f;
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      kq[w] = st_max[w * kStatCols + cc];
-      kb = max(kb, kq[w]);
-      kf = min(kf, st_min[w * kStatCols + cc]);
-    }
-    const float c = (kb > kKeyNegInfG && kb < kKeyPosInfG) ? okey_value(kb) : 0.0f;
-    float sum = 0.0f;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      const float sw = st_sum[w * kStatCols + cc];
-      const float cw = (kq[w] > kKeyNegInfG && kq[w] < kKeyPosInfG) ? okey_value(kq[w]) : 0.0f;
-      sum += sw == 0.0f ? 0.0f : sw * ex2_approx((cw - c) * kLog2e);
-    }
-    if (n < a.R) {
-      float4* rec = reinterpret_cast<float4*>(
-          a.stats + ((static_cast<size_t>(n) * a.S + slice) * a.m_tiles + block) * 8);
-      rec[0] = make_float4(okey_value(kq[0]), okey_value(kq[1]), okey_value(kq[2]), okey_value(kq[3]));
-      rec[1] = make_float4(sum, kf == 0xFFFFFFFFu ? INFINITY : okey_value(kf + kKeyNegInfG + 1u), 0.0f, 0.0f);
-    }
+  for (int i = 0; i < 16; ++i) sum += ex2_approx((v[i] - c) * kLog2e);
+  sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 1);
+  sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 2);
+  sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 4);
+  const int g = lane & ~7;
+  const float q0 = __shfl_sync(0xFFFFFFFFu, mx, g), q1 = __shfl_sync(0xFFFFFFFFu, mx, g + 2);
+  const float q2 = __shfl_sync(0xFFFFFFFFu, mx, g + 4), q3 = __shfl_sync(0xFFFFFFFFu, mx, g + 6);
+  const int n = n_first + row;
+  if (sub == 0 && n < a.R) {
+    float4* rec = reinterpret_cast<float4*>(a.stats + ((static_cast<size_t>(n) * a.S + slice) * a.m_tiles + block) * 8);
+    rec[0] = make_float4(q0, q1, q2, q3);
+    rec[1] = make_float4(sum, mn, 0.0f, 0.0f);
   }
-  return true;
 }
 
 template <int BN, int STAGES>
@@ -197,17 +168,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1) logits_local_kernel(const __g
   constexpr uint32_t kABytes = kBM * kBK * 2;
   constexpr uint32_t kBBytes = BN * kBK * 2;
   constexpr uint32_t kAccCols = static_cast<uint32_t>(tmem_cols<BN>());
+  constexpr int NB = chunk_buffers<BN>();
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * kABytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * (kABytes + kBBytes));
+  float* chunk_buf = reinterpret_cast<float*>(smem + STAGES * (kABytes + kBBytes));  // [NB][16][128]
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * (kABytes + kBBytes) + NB * kChunkBytes);
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;   // [2]: MMA -> epilogue
   uint64_t* acc_empty = acc_full + 2;    // [2]: epilogue (4 warps) -> MMA
   uint64_t* done = acc_empty + 2;        // every MMA of the CTA has completed
-  uint64_t* stat_bar = done + 1;         // [2]: the epilogue's 4 warps staged a chunk's statistics
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(stat_bar + 2);
+  uint64_t* chunk_full = done + 1;       // [2]: the 4 epilogue warps staged a chunk in buffer b
+  uint64_t* chunk_free = chunk_full + 2; // [2]: buffer b was read by the statistics and the store
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(chunk_free + 2);
   volatile uint32_t* abort_flag = tmem_slot + 1;
-  uint32_t* stat_stage = tmem_slot + 4;  // [2][kStatStageBytes / 4]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -223,8 +196,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) logits_local_kernel(const __g
       mbar_init(smem_u32(&acc_empty[b]), 4);
     }
     mbar_init(smem_u32(done), 1);
-    mbar_init(smem_u32(&stat_bar[0]), 4);
-    mbar_init(smem_u32(&stat_bar[1]), 4);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&chunk_full[b]), 4);
+      mbar_init(smem_u32(&chunk_free[b]), 4);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -304,14 +279,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1) logits_local_kernel(const __g
     umma_commit(smem_u32(done));
     mbar_wait_bounded(smem_u32(done), 0);
   } else if (warp >= 2) {
-    // ---------------- epilogue: TMEM -> registers -> global fp32, one tile behind the MMAs
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    // ---------------- epilogue: TMEM -> registers -> staged chunk -> TMA store, one tile behind the MMAs
+    const int q = warp & 3;              // TMEM lane quarter this warp may access
+    const int e = threadIdx.x - 64;      // 0..127
+    const bool leader = threadIdx.x == 64;
+    if (leader)
+      for (int s = 0; s < a.S; ++s) prefetch_tmap(&a.tmap_out[s]);
     int i = 0;
-    uint32_t chunk = 0;      // statistics chunks so far (stage buffer and mbarrier phase)
-    bool stat_ok = true;
-    for (int t = blockIdx.x; t < total; t += gridDim.x, ++i) {
-      const int b = i & 1;
-      const bool ok = mbar_wait_bounded(smem_u32(&acc_full[b]), (i >> 1) & 1);
+    uint32_t chunk = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++i) {
+      const int ab = i & 1;
+      ok = mbar_wait_bounded(smem_u32(&acc_full[ab]), (i >> 1) & 1);
       if (!ok) {
         if (lane == 0) atomicOr(a.err, kErrGemmEpilogue);
         *abort_flag = 1;
@@ -321,37 +300,53 @@ __global__ void __launch_bounds__(kGemmThreads, 1) logits_local_kernel(const __g
       if (!__all_sync(0xFFFFFFFFu, ok && !*abort_flag)) break;
       const int mt = t / a.n_tiles;
       const int slice = mt / a.m_tiles;
-      const int m = (mt % a.m_tiles) * kBM + q * 32 + lane;  // vocab row of this thread
+      const int block = mt % a.m_tiles;
+      const int m0 = block * kBM;
+      const bool m_ok = m0 + q * 32 + lane < a.V_s;  // this thread's vocab row exists
       const int n0 = (t % a.n_tiles) * BN;
-      float* out = a.out[slice];
-      const bool m_ok = m < a.V_s;
-      const uint32_t acc = tmem + static_cast<uint32_t>(b) * kAccCols + (static_cast<uint32_t>(q * 32) << 16);
+      const uint32_t acc = tmem + static_cast<uint32_t>(ab) * kAccCols + (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll 1
-      for (int c = 0; c < BN; c += 16) {
+      for (int c = 0; c < BN && ok; c += kChunk, ++chunk) {
         uint32_t r[16];
         tmem_ld_x16(acc + c, r);
         tmem_ld_wait();
-        if (m_ok) {
+        if (c + kChunk >= BN) {
+          // the accumulator's reads are complete: hand it back to the MMA warp
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&acc_empty[ab]));
+        }
+        const uint32_t b = chunk % NB, use = chunk / NB;
+        float* stage = chunk_buf + b * (kChunk * kBM);
+        // the buffer's previous chunk has been read by the statistics and the store
+        if (chunk >= static_cast<uint32_t>(NB) && !mbar_wait_bounded(smem_u32(&chunk_free[b]), (use - 1) & 1u)) {
+          ok = false;
+          break;
+        }
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int n = n0 + c + j;
-            if (n < a.R) out[static_cast<size_t>(n) * a.V_s + m] = __uint_as_float(r[j]);
-          }
+        for (int j = 0; j < 16; ++j) stage[j * kBM + q * 32 + lane] = m_ok ? __uint_as_float(r[j]) : -INFINITY;
+        fence_proxy_async_smem();  // the TMA store reads what the generic proxy wrote
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&chunk_full[b]));
+        if (!mbar_wait_bounded(smem_u32(&chunk_full[b]), use & 1u)) {
+          ok = false;
+          break;
         }
-        if (a.stats != nullptr && stat_ok) {
-          stat_ok = epilogue_stats(a, r, m_ok, q, lane, n0 + c, slice, mt % a.m_tiles, stat_stage, stat_bar, chunk);
-          ++chunk;
-          if (!stat_ok) {
-            if (lane == 0) atomicOr(a.err, kErrGemmEpilogue);
-            *abort_flag = 1;
-          }
+        if (leader && n0 + c < a.R) {  // a box that starts past the last row writes nothing: not issued
+          tma_store_2d(&a.tmap_out[slice], m0, n0 + c, smem_u32(stage));
+          bulk_commit_group();
         }
+        if (a.stats != nullptr) chunk_stats(a, stage, e, lane, n0 + c, slice, block);
+        if (leader) bulk_wait_read_all();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&chunk_free[b]));
       }
-      // the accumulator's reads are complete: hand it back to the MMA warp
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&acc_empty[b]));
+      if (!ok) {
+        if (lane == 0) atomicOr(a.err, kErrGemmEpilogue);
+        *abort_flag = 1;
+      }
     }
+    if (leader) bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();
@@ -391,11 +386,25 @@ bool encode_bf16_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t co
   return r == CUDA_SUCCESS;
 }
 
+// 2-D fp32 row-major [rows][cols] map with a box of 128 columns x 16 rows (epilogue stores).
+bool encode_f32_out(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 4};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kBM), static_cast<cuuint32_t>(kChunk)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 template <int BN, int STAGES>
 cudaError_t launch_bn(GemmArgs& args, const void* hidden, const void* const* w, int S, int H, int R,
                       int V_s, cudaStream_t stream) {
   for (int s = 0; s < S; ++s)
     if (!encode_bf16_2d(&args.tmap_w[s], w[s], V_s, H, kBM)) return cudaErrorInvalidValue;
+  for (int s = 0; s < S; ++s)
+    if (!encode_f32_out(&args.tmap_out[s], args.out[s], R, V_s)) return cudaErrorInvalidValue;
   if (!encode_bf16_2d(&args.tmap_h, hidden, R, H, BN)) return cudaErrorInvalidValue;
   args.n_tiles = (R + BN - 1) / BN;
   args.w_evict_first = args.n_tiles == 1;
