@@ -25,7 +25,9 @@ tests can check them:
          largest logit when that is finite, else 0 (so a block of -inf sums
          to 0; a NaN makes bsum NaN and +inf makes it +inf);
   [5]    bmin, the smallest finite logit of the block (+inf if none);
-  [6, 7] 0.
+  [6]    amin, the smallest |l| over the block's logits that are not NaN
+         and not 0 (+inf if none; an infinite logit counts as +inf);
+  [7]    0.
 Everything is float64 here; the library stores float32 (the maxima and minima
 exactly, bsum rounded).
 """
@@ -56,6 +58,8 @@ def block_record(vals):
     with np.errstate(invalid="ignore", over="ignore"):
         rec[4] = np.sum(np.exp(vals - c))
     rec[5] = finite.min() if finite.size else np.inf
+    mag = np.abs(vals[~np.isnan(vals) & (vals != 0.0)])
+    rec[6] = mag.min() if mag.size else np.inf
     return rec
 
 

@@ -24,7 +24,9 @@ def test_arithmetic_progression_closed_form(n):
     # c is the largest value a + d (n - 1): terms exp(-d k), k = 0 .. n - 1
     assert rec[4] == pytest.approx(geometric(n, d), rel=1e-14)
     assert rec[5] == a
-    assert rec[6] == 0.0 and rec[7] == 0.0
+    # every term is negative (a + d (n - 1) < 0): the smallest |l| is the last one
+    assert rec[6] == -(a + d * (n - 1))
+    assert rec[7] == 0.0
 
 
 def test_decreasing_progression_quarters():
@@ -39,10 +41,18 @@ def test_constant_block_sums_to_its_size():
     assert block_record(np.full(77, 4.5))[4] == 77.0
 
 
+def test_smallest_nonzero_magnitude():
+    vals = np.array([0.0, -0.0, -2.5, 1e-30, -3e-38, np.nan, 7.0] + [0.0] * 20)
+    assert block_record(vals)[6] == 3e-38
+    assert block_record(np.zeros(40))[6] == np.inf
+    assert block_record(np.array([0.0, -np.inf, 0.0]))[6] == np.inf      # only an infinity: +inf
+    assert block_record(np.array([0.0, -np.inf, -5.0]))[6] == 5.0
+
+
 def test_negative_infinity_entries():
     vals = np.full(128, -np.inf)
     rec = block_record(vals)
-    assert np.all(rec[:4] == -np.inf) and rec[4] == 0.0 and rec[5] == np.inf
+    assert np.all(rec[:4] == -np.inf) and rec[4] == 0.0 and rec[5] == np.inf and rec[6] == np.inf
     vals[40] = 2.0
     vals[100] = -7.0
     rec = block_record(vals)
