@@ -311,24 +311,38 @@ def _tile_rows(T, k, V):
     return (T == 0) | ((k > 0) & (k < V) & (k <= 1024))
 
 
-def _uses_tiles(w, T, k):
+def _large_batch(w, sms):
+    """More rows than SMs: the streaming kernel gives each row one CTA and also
+    takes the top-k-off rows (which then read the records too)."""
+    return w.R > sms
+
+
+def _uses_tiles(w, T, k, sms):
     """The step requests tile statistics when some row can use them (and the
     vocabulary has at most 4096 blocks of 128)."""
-    return bool(_tile_rows(T, k, w.V).any()) and w.S * (-(-w.V_s // 128)) <= 4096
+    some = bool(_tile_rows(T, k, w.V).any()) or _large_batch(w, sms)
+    return some and w.S * (-(-w.V_s // 128)) <= 4096
 
 
-def _sampler_read_bytes(w, T, k, stats):
-    """Algorithmic bytes one sampler call reads: every row outside the tile mode
-    reads its V logits; a tile-mode row reads its records (S * B * 32 bytes)
-    and the 32-logit quarters whose largest x reaches fl(t0 / T), t0 the R-th
-    largest block maximum, R = max(n, k) (greedy: max(n, 1)).  Counted from the
-    records with torch on the device (the kernel's cut can sit a few floats
-    lower, where the temperature maps neighbours to one x: an undercount of a
-    few quarters at most)."""
+def _sampler_read_bytes(w, T, k, stats, sms):
+    """Algorithmic bytes one sampler call reads.  Without records every row
+    reads its V logits.  With them, a greedy or top-k row reads its records
+    (S * B * 32 bytes) and the 32-logit quarters whose largest x reaches
+    fl(t0 / T), t0 the R-th largest block maximum, R = max(n, k) (greedy:
+    max(n, 1)); a top-k-off row of a large batch its records and its V logits
+    once (the top-p passes; its few top-n quarters are not counted); any other
+    row its V logits.  The quarters are counted from the records with torch on
+    the device (the kernel's cut can sit a few floats lower, where the
+    temperature maps neighbours to one x: an undercount of a few quarters at
+    most)."""
     tile = _tile_rows(T, k, w.V)
-    full = int((~tile).sum()) * w.V * 4
-    if stats is None or not tile.any():
+    if stats is None:
         return w.R * w.V * 4
+    SB = w.S * (-(-w.V_s // 128))
+    koff = int((~tile).sum())
+    full = koff * (w.V * 4 + (SB * 32 if _large_batch(w, sms) else 0))
+    if not tile.any():
+        return full
     dev = stats.device
     rows = torch.from_numpy(np.flatnonzero(tile)).to(dev)
     st = stats[rows]
@@ -371,7 +385,8 @@ def measure_config(w, dev, world, rank, steps, warmup, peaks):
     # every step and the sampler reads them; for the peaked workload, whose
     # sampler reads its own synthetic logits, the records of those logits
     # (written once) stand in for the epilogue's
-    tiles = _uses_tiles(w, T, k)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    tiles = _uses_tiles(w, T, k, sms)
     stats = torch.empty(vsl.tile_stats_shape(w.R, w.S, w.V_s), device=dev) if tiles else None
     samp_stats = vsl.tile_stats(samp_in) if tiles and samp_in is not logits else stats
 
@@ -475,7 +490,7 @@ def measure_config(w, dev, world, rank, steps, warmup, peaks):
 
     gemm_bytes = w.V * w.H * 2 + w.R * w.H * 2 + w.R * w.V * 4
     gemm_flops = 2.0 * w.R * w.H * w.V
-    samp_bytes = _sampler_read_bytes(w, T, k, samp_stats)
+    samp_bytes = _sampler_read_bytes(w, T, k, samp_stats, sms)
     ridge = tf_peak * 1e12 / (hbm_peak * 1e9)
     gemm_hbm = gemm_flops / gemm_bytes < ridge
     gemm_tf = gemm_flops / (gemm_ms / 1e3) / 1e12
@@ -624,7 +639,7 @@ def run_sampler_only(args, w):
         i += 1
     clk = clocks.stop()
     ms = statistics.median(times)
-    nbytes = _sampler_read_bytes(w, T, k, stats)
+    nbytes = _sampler_read_bytes(w, T, k, stats, torch.cuda.get_device_properties(dev).multi_processor_count)
     print(json.dumps({"metric": f"sampler rows/sec ({w.name}, V={w.V}, L2 flushed)", "value": w.R / (ms / 1e3),
                       "unit": "rows/s", "ms": ms, "hbm_gbs": nbytes / (ms / 1e3) / 1e9,
                       "roofline": {"bound": "hbm", "achieved": nbytes / (ms / 1e3) / 1e9, "peak": hbm_peak,

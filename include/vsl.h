@@ -133,7 +133,9 @@ VSL_API vsl_status vsl_logits_local(const void* hidden_bf16, const void* const* 
  *          finite, else 0 (float32 with a fast exp; NaN if a logit is NaN,
  *          +inf if one is +inf)
  *   [5]    the block's smallest finite logit (+inf if none)
- *   [6, 7] 0
+ *   [6]    the block's smallest |l| over logits that are neither 0 nor NaN
+ *          (+inf if none; an infinite logit counts as +inf)
+ *   [7]    0
  * vsl_tile_stats_floats returns 0 for non-positive sizes. */
 VSL_API size_t vsl_tile_stats_floats(int32_t R, int32_t S, int32_t V_s);
 

@@ -25,8 +25,8 @@ def check_records(got, want):
     nan_block = np.isnan(want[..., 4])
     q = got[..., :4][~nan_block]
     assert np.array_equal(q, want[..., :4][~nan_block]), np.argwhere(got[..., :4][~nan_block] != want[..., :4][~nan_block])[:5]
-    assert np.array_equal(got[..., 5], want[..., 5])
-    assert np.all(got[..., 6:] == 0)
+    assert np.array_equal(got[..., 5:7], want[..., 5:7])
+    assert np.all(got[..., 7] == 0)
     s, w = got[..., 4], want[..., 4]
     assert np.array_equal(np.isnan(s), np.isnan(w))
     fin = np.isfinite(w)
@@ -92,7 +92,7 @@ def test_projection_statistics_full_size(cuda_device, name):
     again = vsl.tile_stats(out)
     torch.cuda.synchronize()
     a, b = stats.cpu().numpy(), again.cpu().numpy()
-    assert np.array_equal(a[..., :4], b[..., :4]) and np.array_equal(a[..., 5:], b[..., 5:])
+    assert np.array_equal(a[..., :4], b[..., :4]) and np.array_equal(a[..., 5:], b[..., 5:])  # maxima, minima, word 7
     assert np.all(np.abs(a[..., 4] - b[..., 4]) <= 2 * SUM_RTOL * np.abs(b[..., 4]))
     rows = [0, w.R // 2, w.R - 1]
     want = ref_tile_stats([o[rows].cpu().numpy() for o in out])
@@ -106,7 +106,7 @@ def _same_as_without(a, b):
         assert np.allclose(a[key], b[key], atol=2e-5, rtol=0, equal_nan=True), key
 
 
-@pytest.mark.parametrize("name", ["decode", "spec", "peaked", "tiny"])
+@pytest.mark.parametrize("name", ["decode", "spec", "peaked", "tiny", "large"])
 def test_tile_mode_small_vocab_all_rows(cuda_device, name):
     w = W.scaled(W.WORKLOADS[name], V=8 * 1500, requests=max(4, 64 // W.WORKLOADS[name].rows_per_request)) \
         if name != "tiny" else W.WORKLOADS[name]
@@ -170,3 +170,22 @@ def test_tile_mode_large_batch_mixed(cuda_device):
     rows = sorted(np.random.default_rng(4).choice(w.R, 40, replace=False).tolist())
     compare(got, logits.cpu().numpy(), params, 3, w.n_logprobs, rows)
     assert vsl.device_error() == (0, 0)
+
+
+@pytest.mark.parametrize("V,S", [(12000, 4), (151936, 8)])
+def test_tile_mode_large_batch_top_k_off(cuda_device, V, S):
+    """Top-k-off rows of a large batch take their statistics, smallest nonzero
+    |l| (the division's domain check) and top-n candidates from the records
+    and stream their row for the top-p passes only: the same results as
+    without the records, and the oracle's."""
+    from test_sample_gpu import _koff_rows
+    R = 300
+    rng = np.random.default_rng(V + 5)
+    logits, params = _koff_rows(V, R, rng)
+    t = torch.from_numpy(logits)
+    got = run_sampler(t, params, 4243, 20, S, cuda_device, tiles=True)
+    ref = run_sampler(t, params, 4243, 20, S, cuda_device)
+    _same_as_without(got, ref)
+    rows = range(R) if V <= 12000 else sorted(set(range(12)) | set(rng.choice(R, 28, replace=False).tolist()))
+    st = compare(got, logits, params, 4243, 20, rows)
+    assert st["mismatch_allowed"] <= 2

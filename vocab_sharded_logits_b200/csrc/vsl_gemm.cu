@@ -30,8 +30,9 @@
 //     for the 128 vocab rows of the tile (the block) from the staged chunk:
 //     each of the 128 epilogue threads reads 16 consecutive logits of one
 //     (batch row, quarter, half) from shared memory (maximum, smallest finite
-//     value, sum of exp(l - c)), and three shuffle steps among the 8 threads of
-//     a batch row give the quarter maxima and the block's sum and minimum.
+//     value, smallest nonzero |l|, sum of exp(l - c)), and three shuffle steps
+//     among the 8 threads of a batch row give the quarter maxima and the
+//     block's sum and minima.
 //   * The four epilogue warps meet at two mbarriers per chunk (bounded waits):
 //     the chunk is staged, and the buffer is free again (read by the
 //     statistics and by the store).
@@ -131,11 +132,12 @@ __device__ __forceinline__ void chunk_stats(const GemmArgs& a, const float* stag
     v[4 * j + 2] = x.z;
     v[4 * j + 3] = x.w;
   }
-  float mx = v[0], mn = INFINITY;
+  float mx = v[0], mn = INFINITY, am = INFINITY;
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     mx = fmaxf(mx, v[i]);
     mn = fminf(mn, isfinite(v[i]) ? v[i] : INFINITY);
+    am = fminf(am, v[i] != 0.0f ? fabsf(v[i]) : INFINITY);  // fminf drops a NaN
   }
   mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 1));  // the quarter's maximum
   mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, 1));
@@ -143,6 +145,8 @@ __device__ __forceinline__ void chunk_stats(const GemmArgs& a, const float* stag
   bm = fmaxf(bm, __shfl_xor_sync(0xFFFFFFFFu, bm, 4));  // the block's maximum
   mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, 2));
   mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, 4));
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1) am = fminf(am, __shfl_xor_sync(0xFFFFFFFFu, am, o));
   const float c = isfinite(bm) ? bm : 0.0f;
   float sum = 0.0f;
 #pragma unroll
@@ -157,7 +161,7 @@ __device__ __forceinline__ void chunk_stats(const GemmArgs& a, const float* stag
   if (sub == 0 && n < a.R) {
     float4* rec = reinterpret_cast<float4*>(a.stats + ((static_cast<size_t>(n) * a.S + slice) * a.m_tiles + block) * 8);
     rec[0] = make_float4(q0, q1, q2, q3);
-    rec[1] = make_float4(sum, mn, 0.0f, 0.0f);
+    rec[1] = make_float4(sum, mn, am, 0.0f);
   }
 }
 

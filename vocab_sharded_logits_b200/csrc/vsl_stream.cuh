@@ -251,6 +251,7 @@ __device__ __forceinline__ TileScan stream_tiles(const Ctx& cx, const SampleArgs
     cx.list[i] = (static_cast<uint64_t>(~kb) << 32) | static_cast<uint32_t>(i);
     const uint32_t kmin = fkey(sm.y);
     st.kmf = min(st.kmf, key_finite(kmin) ? kmin - (kKeyNegInf + 1u) : 0xFFFFFFFFu);
+    st.amin = min(st.amin, __float_as_uint(sm.z) & 0x7FFFFFFFu);  // smallest nonzero |l| (+inf: none)
     // the block's sum runs against its maximum c (0 when that is not finite)
     if (kb > st.kmax) {
       st.kmax = kb;
@@ -620,7 +621,9 @@ __global__ void __launch_bounds__(kThreads, 2) stream_kernel(const __grid_consta
   const bool k_on = !greedy && prm.top_k > 0 && prm.top_k < a.V;
   uint32_t R = a.n_logprobs > 0 ? static_cast<uint32_t>(a.n_logprobs) : 1u;
   if (k_on) R = max(R, static_cast<uint32_t>(prm.top_k));
-  const bool tiles = a.tile_stats != nullptr && a.C == 1 && (greedy || k_on);
+  // tile mode: every row this kernel takes on one CTA (a top-k-off row of a
+  // large batch then replaces its first pass with the records and the top-n quarters)
+  const bool tiles = a.tile_stats != nullptr && a.C == 1 && (greedy || k_on || take_koff);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStreamStages; ++s) mbar_init(smem_u32(&H->ring_bar[s]), 1);
@@ -705,7 +708,7 @@ __global__ void __launch_bounds__(kThreads, 2) stream_kernel(const __grid_consta
     c += cur;
   }
 
-  int cg = nch;  // chunks streamed so far (the ring's position)
+  int cg = tiles ? 0 : nch;  // chunks streamed so far (the ring's position)
   // ---- CTA statistics (the cluster kernel's CtaStats layout)
   // (m, s) pairs merge by rescaling to the larger m; empty sums add 0
 #pragma unroll

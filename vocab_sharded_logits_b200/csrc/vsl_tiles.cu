@@ -6,7 +6,8 @@
 // top-k / top-p and logprobs need, per row, the softmax statistics and the
 // top candidates of the whole vocabulary.  Per block of 128 ids of a slice the
 // record holds the four 32-id quarter maxima, the sum of exp(l - c) (c the
-// block's largest logit when finite, else 0) and the smallest finite logit;
+// block's largest logit when finite, else 0), the smallest finite logit and
+// the smallest nonzero |l|;
 // a sampler that has them reads only the quarters that can hold its top
 // candidates.
 //
@@ -66,12 +67,14 @@ __global__ void __launch_bounds__(kTileWarps * 32) tile_stats_kernel(const __gri
     v[2] = x.z;
     v[3] = x.w;
   }
-  uint32_t kq = 0, kf = 0xFFFFFFFFu;
+  uint32_t kq = 0, kf = 0xFFFFFFFFu, am = 0xFFFFFFFFu;
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
     const uint32_t k = order_key(v[u]);
     kq = max(kq, k);
     kf = min(kf, k - (kNegInfKey + 1u));  // -inf and negative NaN wrap above every finite key
+    const uint32_t ab = __float_as_uint(v[u]) & 0x7FFFFFFFu;  // |l|: nonzero and not NaN
+    am = min(am, (ab != 0u && ab <= 0x7F800000u) ? ab : 0xFFFFFFFFu);
   }
 #pragma unroll
   for (int o = 1; o < 8; o <<= 1) kq = max(kq, __shfl_xor_sync(0xFFFFFFFFu, kq, o));  // the quarter's 8 lanes
@@ -79,6 +82,7 @@ __global__ void __launch_bounds__(kTileWarps * 32) tile_stats_kernel(const __gri
 #pragma unroll
   for (int o = 8; o < 32; o <<= 1) kb = max(kb, __shfl_xor_sync(0xFFFFFFFFu, kb, o));
   kf = __reduce_min_sync(0xFFFFFFFFu, kf);
+  am = __reduce_min_sync(0xFFFFFFFFu, am);
   const float c = (kb > kNegInfKey && kb < kPosInfKey) ? key_float(kb) : 0.0f;
   constexpr float kLog2e = 1.4426950408889634f;
   float e = 0.0f;
@@ -94,7 +98,7 @@ __global__ void __launch_bounds__(kTileWarps * 32) tile_stats_kernel(const __gri
     float4* rec = reinterpret_cast<float4*>(a.stats + (static_cast<size_t>(row) * a.S * a.B + i) * 8);
     const float bmin = kf == 0xFFFFFFFFu ? INFINITY : key_float(kf + kNegInfKey + 1u);
     rec[0] = make_float4(q0, q1, q2, q3);
-    rec[1] = make_float4(e, bmin, 0.0f, 0.0f);
+    rec[1] = make_float4(e, bmin, am == 0xFFFFFFFFu ? INFINITY : __uint_as_float(am), 0.0f);
   }
 }
 
