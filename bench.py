@@ -660,8 +660,9 @@ def run_gemm_only(args, w):
     hbm_peak, tf_peak, _, peak_kind = _peaks()
     hidden, ws = W.gemm_inputs(w, dev)
     out = [torch.empty(w.R, w.V_s, dtype=torch.float32, device=dev) for _ in range(w.S)]
+    stats = torch.empty(vsl.tile_stats_shape(w.R, w.S, w.V_s), device=dev) if args.tile_stats else None
     for _ in range(args.warmup):
-        vsl.logits_local(hidden, ws, out=out)
+        vsl.logits_local(hidden, ws, out=out, tile_stats=stats)
     torch.cuda.synchronize()
     clocks = ClockSampler(0)
     clocks.start()
@@ -673,7 +674,7 @@ def run_gemm_only(args, w):
         e0, e1 = _events(2)
         e0.record()
         for _ in range(10):
-            vsl.logits_local(hidden, ws, out=out)
+            vsl.logits_local(hidden, ws, out=out, tile_stats=stats)
         e1.record()
         torch.cuda.synchronize()
         if i < args.steps:
@@ -686,7 +687,8 @@ def run_gemm_only(args, w):
     print(json.dumps({"metric": f"logits_local TFLOP/s ({w.name})", "value": flops / ms / 1e9, "unit": "TFLOP/s",
                       "ms": ms, "hbm_gbs": nbytes / (ms / 1e3) / 1e9, "tflops_frac_of_burst": flops / ms / 1e9 / tf_peak,
                       "hbm_frac": nbytes / (ms / 1e3) / 1e9 / hbm_peak, "peak_source": peak_kind, "clocks": clk,
-                      "config": {"workload": w.name, "rows": w.R, "hidden": w.H, "vocab": w.V, "slices": w.S}}),
+                      "config": {"workload": w.name, "rows": w.R, "hidden": w.H, "vocab": w.V, "slices": w.S,
+                                 "tile_statistics": bool(args.tile_stats)}}),
           flush=True)
     return 0
 
@@ -705,7 +707,8 @@ def main():
     ap.add_argument("--sampler-only", action="store_true",
                     help="time the sampler alone on the workload's synthetic logits (profiling aid)")
     ap.add_argument("--tile-stats", action="store_true",
-                    help="with --sampler-only: give the sampler the tile statistics of its logits")
+                    help="with --sampler-only: give the sampler the tile statistics of its logits; with "
+                         "--gemm-only: the projection also writes them")
     ap.add_argument("--gemm-only", action="store_true",
                     help="time the projection alone, 10 back-to-back launches per timing (profiling aid)")
     args = ap.parse_args()
