@@ -500,18 +500,28 @@ struct Best {
 // Philox words, the quotient, the exp) runs at full width instead of once per
 // warp step whenever any lane has a kept token.  Every lane of the warp
 // calls push and drain together (the count n is warp-uniform).
+// A queue may also carry each token's Philox word (kWords: the pass computed
+// it once per float4 group, for rows where most groups hold a kept token).
 constexpr int kDrawQueue = 160;  // a drain leaves < 32 entries; at most 128 are pushed before the next
-constexpr size_t kDrawQueueBytes = static_cast<size_t>(kWarps) * kDrawQueue * 8;
+constexpr size_t kDrawQueueBytes = static_cast<size_t>(kWarps) * kDrawQueue * 12;
+template <bool kWords>
 struct DrawQueue {
-  uint64_t* q;  // this warp's entries: payload << 32 | id
+  uint64_t* q;   // this warp's entries: payload << 32 | id
+  uint32_t* wq;  // (kWords) their Philox words
   uint32_t n;
   __device__ __forceinline__ void init(void* base) {
     q = reinterpret_cast<uint64_t*>(base) + (threadIdx.x >> 5) * kDrawQueue;
+    wq = reinterpret_cast<uint32_t*>(reinterpret_cast<uint64_t*>(base) + kWarps * kDrawQueue) +
+         (threadIdx.x >> 5) * kDrawQueue;
     n = 0;
   }
-  __device__ __forceinline__ void push(bool pred, uint64_t e) {
+  __device__ __forceinline__ void push(bool pred, uint64_t e, uint32_t word = 0u) {
     const uint32_t m = __ballot_sync(0xFFFFFFFFu, pred);
-    if (pred) q[n + __popc(m & ((1u << (threadIdx.x & 31)) - 1u))] = e;
+    if (pred) {
+      const uint32_t i = n + __popc(m & ((1u << (threadIdx.x & 31)) - 1u));
+      q[i] = e;
+      if (kWords) wq[i] = word;
+    }
     n += __popc(m);
   }
   // Takes queued tokens 32 at a time while a full batch is queued (all:
@@ -525,12 +535,14 @@ struct DrawQueue {
       const uint32_t base = n - take;
       const bool act = lane < take;
       const uint64_t e = act ? q[base + lane] : 0ull;
+      const uint32_t wd = (kWords && act) ? wq[base + lane] : 0u;
       __syncwarp();
       n = base;
       if (act) {
         const uint32_t id = static_cast<uint32_t>(e);
-        const uint4 w = philox4x32_10(make_uint4(id >> 2, pos, req, 0u), k0, k1);
-        one(static_cast<uint32_t>(e >> 32), word_of(w, static_cast<int>(id & 3u)), static_cast<int32_t>(id));
+        uint32_t word = wd;
+        if (!kWords) word = word_of(philox4x32_10(make_uint4(id >> 2, pos, req, 0u), k0, k1), static_cast<int>(id & 3u));
+        one(static_cast<uint32_t>(e >> 32), word, static_cast<int32_t>(id));
       }
     }
   }

@@ -517,18 +517,29 @@ __device__ bool stream_koff(const Ctx& cx, LeaderState& L, const SampleArgs& a, 
   const uint32_t ka = H->kcut_above;
   const uint32_t kw = H->kcut_window;
   const double z_total = H->row_z;
+  // tokens kept for certain (the fine bins above the window): when more than
+  // a quarter of the row is kept, nearly every float4 group holds one, and
+  // one Philox call per group (its four words, queued with the tokens) costs
+  // less than one per queued token
+  uint32_t kept_here = 0, kept_total = 0;
+  for (int j = t; j < jlo; j += kThreads) kept_here += cnt[j];
+  block_scan_u(kept_here, &kept_total, H);
+  const bool dense = 4ull * kept_total > static_cast<unsigned long long>(n);
   // ---- pass 3: every key compared with the thresholds; the window's members
-  // listed (sort key ~x key, id); every token kept for certain queued, and the
-  // warp drains the queue 32 tokens at a time: its x, its float64 mass (the
-  // mass above the window, A) and the draw
+  // listed (sort key ~x key, id); every token kept for certain queued (with
+  // its Philox word on a densely kept row), and the warp drains the queue 32
+  // tokens at a time: its x, its float64 mass (the mass above the window, A)
+  // and the draw
   Best b;
   b.init(&H->gbound);
   double above = 0.0;
   float xmin_ab = INFINITY;  // smallest x above the window
-  DrawQueue dq;
-  dq.init(cnt);  // the fine bins' area is free once the window is found, until the window is sorted
-  auto pass3 = [&](auto fast_tag) {
+  // the fine bins' area is free once the window is found, until the window is sorted
+  auto pass3 = [&](auto fast_tag, auto words_tag) {
     constexpr bool kF = decltype(fast_tag)::value;
+    constexpr bool kW = decltype(words_tag)::value;
+    DrawQueue<kW> dq;
+    dq.init(cnt);
     auto one = [&](uint32_t lbits, uint32_t wd, int32_t id) {
       const float x = kF ? scale_x_fast(__uint_as_float(lbits), T, y) : scale_x(__uint_as_float(lbits), T);
       above += exp_neg64(static_cast<double>(x) - md, tab);
@@ -544,13 +555,14 @@ __device__ bool stream_koff(const Ctx& cx, LeaderState& L, const SampleArgs& a, 
         const float4 v4 = valid ? st4[q] : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
         const float l[4] = {v4.x, v4.y, v4.z, v4.w};
         bool win[4], ab[4];
-        bool any_win = false;
+        bool any_win = false, any_ab = false;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const uint32_t k = fkey(l[i]);  // -inf and padding lie below kw: the row's keys are finite above it
           ab[i] = valid && k >= ka;
           win[i] = valid && k >= kw && k < ka;
           any_win |= win[i];
+          any_ab |= ab[i];
         }
         const uint32_t gq = gid + 4u * static_cast<uint32_t>(q);
         if (__any_sync(0xFFFFFFFFu, any_win)) {
@@ -560,16 +572,23 @@ __device__ bool stream_koff(const Ctx& cx, LeaderState& L, const SampleArgs& a, 
             local_append(&H->list_count, wc.list, win[i], (static_cast<uint64_t>(~fkey(x)) << 32) | (gq + i));
           }
         }
+        uint4 w = make_uint4(0u, 0u, 0u, 0u);
+        if (kW && any_ab) w = philox4x32_10(make_uint4(gq >> 2, cx.pos, cx.req, 0u), k0, k1);
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-          dq.push(ab[i], (static_cast<uint64_t>(__float_as_uint(l[i])) << 32) | (gq + i));
+          dq.push(ab[i], (static_cast<uint64_t>(__float_as_uint(l[i])) << 32) | (gq + i), word_of(w, i));
         dq.drain(false, cx.pos, cx.req, k0, k1, one);  // at most 31 + 128 queued
       }
     });
     dq.drain(true, cx.pos, cx.req, k0, k1, one);
   };
-  if (fast) pass3(std::true_type{});
-  else pass3(std::false_type{});
+  if (dense) {
+    if (fast) pass3(std::true_type{}, std::true_type{});
+    else pass3(std::false_type{}, std::true_type{});
+  } else {
+    if (fast) pass3(std::true_type{}, std::false_type{});
+    else pass3(std::false_type{}, std::false_type{});
+  }
   const double ta = block_sum_d0(above, H);
   const float tx = block_min_f0(xmin_ab, H);
   if (t == 0) {
