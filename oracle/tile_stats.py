@@ -30,13 +30,6 @@ tests can check them:
   [7]    0.
 Everything is float64 here; the library stores float32 (the maxima and minima
 exactly, bsum rounded).
-
-Tile masses (optional, given each row's temperature T > 0): for every (row,
-slice, block) the float64 sum over the block's finite logits of
-exp(x_j - x_b), x = fl(l / T) in float32 (IEEE division, as the sampler's x)
-and x_b the block's largest such x; 0 for a block without a finite logit.  A
-row's Z = sum_j exp(x_j - m) (m = max x) is then sum_b exp(x_b - m) * mass_b.
-Stored as float64 [R, S * B].
 """
 import numpy as np
 
@@ -83,34 +76,6 @@ def tile_stats(slices):
         for s in range(S):
             for b in range(B):
                 out[r, s * B + b] = block_record(slices[s][r, b * BLOCK:min((b + 1) * BLOCK, V_s)])
-    return out
-
-
-def block_mass(vals, T):
-    """The tile mass of one block (its logits in id order) at temperature T > 0."""
-    l32 = np.asarray(vals, np.float32)
-    fin = np.isfinite(l32)
-    if not fin.any():
-        return 0.0
-    with np.errstate(over="ignore"):
-        x = (l32[fin] / np.float32(T)).astype(np.float32).astype(np.float64)
-    return float(np.sum(np.exp(x - x.max())))
-
-
-def tile_mass(slices, T):
-    """Tile masses [R, S * B] (float64) of every (row, slice, block); T: [R] temperatures
-    (rows with T <= 0 get 0)."""
-    slices = [np.asarray(s, np.float32) for s in slices]
-    R, V_s = slices[0].shape
-    S = len(slices)
-    B = blocks_per_slice(V_s)
-    out = np.zeros((R, S * B))
-    for r in range(R):
-        if not (np.float32(T[r]) > 0):
-            continue
-        for s in range(S):
-            for b in range(B):
-                out[r, s * B + b] = block_mass(slices[s][r, b * BLOCK:min((b + 1) * BLOCK, V_s)], T[r])
     return out
 
 

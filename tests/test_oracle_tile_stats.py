@@ -4,8 +4,7 @@ import numpy as np
 import pytest
 from scipy.special import logsumexp
 
-from oracle.sampler import scale
-from oracle.tile_stats import BLOCK, blocks_per_slice, block_mass, block_record, row_logsumexp, tile_mass, tile_stats
+from oracle.tile_stats import BLOCK, blocks_per_slice, block_record, row_logsumexp, tile_stats
 
 
 def geometric(n, d):
@@ -103,46 +102,3 @@ def test_merged_sums_equal_library_logsumexp():
             assert row_logsumexp(st[r]) == pytest.approx(logsumexp(row[r]), abs=1e-12)
             # the maxima of the quarters give the row maximum
             assert st[r, :, :4].max() == row[r].max()
-
-
-@pytest.mark.parametrize("T", [1.0, 2.0, 0.25])
-def test_block_mass_closed_form(T):
-    # l = T (a + d k) with T a power of two: x = a + d k exactly, the block's
-    # largest x is the last one, and the mass is the geometric sum
-    a, d = -1.5, 0.03125
-    for n in (128, 77, 1):
-        vals = np.float32(T) * (a + d * np.arange(n, dtype=np.float32))
-        assert block_mass(vals, T) == pytest.approx(geometric(n, d), rel=1e-14)
-
-
-def test_block_mass_special_values():
-    assert block_mass(np.full(128, -np.inf, np.float32), 0.7) == 0.0
-    vals = np.full(128, -np.inf, np.float32)
-    vals[3] = 5.0
-    assert block_mass(vals, 0.7) == 1.0              # one finite logit: exp(0)
-    vals[9] = 5.0
-    assert block_mass(vals, 0.7) == 2.0              # ties at the maximum
-
-
-def test_tile_masses_give_the_row_mass():
-    """sum_b exp(x_b - m) mass_b equals sum_j exp(x_j - m) computed directly
-    (x the float32 quotient), for random rows, temperatures and ragged slices."""
-    rng = np.random.default_rng(3)
-    S, V_s = 3, 300
-    slices = [rng.normal(0.0, 2.5, (4, V_s)).astype(np.float32) for _ in range(S)]
-    slices[1][2, 40:200] = -np.inf
-    T = np.array([0.37, 1.0, 1.7, 0.0], np.float32)
-    tm = tile_mass(slices, T)
-    B = blocks_per_slice(V_s)
-    assert tm.shape == (4, S * B) and np.all(tm[3] == 0.0)
-    row = np.concatenate(slices, axis=1)
-    for r in range(3):
-        x = scale(row[r], T[r]).astype(np.float64)
-        fin = np.isfinite(x)
-        m = x[fin].max()
-        direct = np.sum(np.exp(x[fin] - m))
-        xb = np.array([scale(np.float32(s[r, b * BLOCK:(b + 1) * BLOCK][np.isfinite(s[r, b * BLOCK:(b + 1) * BLOCK])].max()
-                                        if np.isfinite(s[r, b * BLOCK:(b + 1) * BLOCK]).any() else -np.inf), T[r])
-                       for s in slices for b in range(B)], np.float64)
-        merged = np.sum(np.where(tm[r] > 0, np.exp(np.where(np.isfinite(xb), xb, m) - m) * tm[r], 0.0))
-        assert merged == pytest.approx(direct, rel=1e-13)
