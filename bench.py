@@ -438,8 +438,10 @@ def measure_config(w, dev, world, rank, steps, warmup, peaks):
     # end to end through the public API with host buffers: every step copies its
     # inputs (hidden states + row parameters, one packed pinned buffer) to the
     # device and reads its results (one packed buffer of the five outputs) back,
-    # on a copy stream, double-buffered, so step i + 1's inputs cross PCIe while
-    # step i computes: the way a serving loop feeds the GPU
+    # double-buffered, the uploads and the read-backs on two copy streams of
+    # their own (on one stream step i + 1's upload would queue behind step i's
+    # read-back, which waits for step i's kernels), so step i + 1's inputs cross
+    # PCIe while step i computes: the way a serving loop feeds the GPU
     in_bytes, out_words = _e2e_sizes(w.R, w.H, n)
     pin_in = [torch.empty(in_bytes, dtype=torch.uint8).pin_memory() for _ in range(2)]
     for b in range(2):
@@ -449,31 +451,33 @@ def measure_config(w, dev, world, rank, steps, warmup, peaks):
     dev_in = [torch.empty(in_bytes, dtype=torch.uint8, device=dev) for _ in range(2)]
     dev_out = [torch.empty(out_words, dtype=torch.int32, device=dev) for _ in range(2)]
     bufs = [_e2e_views(dev_in[b], dev_out[b], w.R, w.H, n) for b in range(2)]
-    copy_stream = torch.cuda.Stream(dev)
+    up_stream = torch.cuda.Stream(dev)
+    down_stream = torch.cuda.Stream(dev)
     ev_in = [torch.cuda.Event() for _ in range(2)]    # inputs of buffer b are on the device
     ev_done = [torch.cuda.Event() for _ in range(2)]  # the step using buffer b has computed
     ev_out = [torch.cuda.Event() for _ in range(2)]   # results of buffer b are on the host
 
     def e2e_run(first_seed, nsteps, start=None):
         if start is not None:
-            copy_stream.wait_event(start)  # no copy of the timed steps starts before the clock
+            up_stream.wait_event(start)  # no copy of the timed steps starts before the clock
+            down_stream.wait_event(start)
         for b in range(2):
-            ev_out[b].record(copy_stream)
+            ev_out[b].record(down_stream)
         for i in range(nsteps):
             b = i & 1
             hid, prm, res = bufs[b]
-            with torch.cuda.stream(copy_stream):
-                copy_stream.wait_event(ev_out[b])  # buffer b's previous step has been read back
+            with torch.cuda.stream(up_stream):
+                up_stream.wait_event(ev_out[b])  # buffer b's previous step has been read back
                 dev_in[b].copy_(pin_in[b], non_blocking=True)
-                ev_in[b].record(copy_stream)
+                ev_in[b].record(up_stream)
             stream.wait_event(ev_in[b])
             project(hid, stream)
             sample(prm, first_seed + i, res, stream)
             ev_done[b].record(stream)
-            with torch.cuda.stream(copy_stream):
-                copy_stream.wait_event(ev_done[b])
+            with torch.cuda.stream(down_stream):
+                down_stream.wait_event(ev_done[b])
                 pin_out[b].copy_(dev_out[b], non_blocking=True)
-                ev_out[b].record(copy_stream)
+                ev_out[b].record(down_stream)
         for b in range(2):
             stream.wait_event(ev_out[b])  # every result is on the host
 
