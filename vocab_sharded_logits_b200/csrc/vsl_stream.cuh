@@ -242,32 +242,51 @@ __device__ __forceinline__ TileScan stream_tiles(const Ctx& cx, const SampleArgs
   const int SB = a.S * B;
   const float4* rec = reinterpret_cast<const float4*>(a.tile_stats) + static_cast<size_t>(cx.row) * SB * 2;
   // records: statistics, the block maxima as list entries, the quarter maxima
-  for (int i = threadIdx.x; i < SB; i += kThreads) {
-    const float4 qm = __ldg(rec + 2 * i);
-    const float4 sm = __ldg(rec + 2 * i + 1);
-    const uint4 k = make_uint4(fkey(qm.x), fkey(qm.y), fkey(qm.z), fkey(qm.w));
-    reinterpret_cast<uint4*>(qkeys)[i] = k;
-    const uint32_t kb = max(max(k.x, k.y), max(k.z, k.w));
-    cx.list[i] = (static_cast<uint64_t>(~kb) << 32) | static_cast<uint32_t>(i);
-    const uint32_t kmin = fkey(sm.y);
-    st.kmf = min(st.kmf, key_finite(kmin) ? kmin - (kKeyNegInf + 1u) : 0xFFFFFFFFu);
-    st.amin = min(st.amin, __float_as_uint(sm.z) & 0x7FFFFFFFu);  // smallest nonzero |l| (+inf: none)
-    // the block's sum runs against its maximum c (0 when that is not finite)
-    if (kb > st.kmax) {
-      st.kmax = kb;
-      if (key_finite(kb)) {
-        const float mn = key_value(kb);
-        st.s = st.s == 0.0f ? 0.0f : st.s * fast_exp2((st.m - mn) * kLog2e);
-        st.m = mn;
+  // (four records per thread loaded before any is used: their latencies overlap)
+  constexpr int kRecBatch = 4;
+  for (int base = threadIdx.x; base < SB; base += kRecBatch * kThreads) {
+    float4 qmb[kRecBatch], smb[kRecBatch];
+#pragma unroll
+    for (int u = 0; u < kRecBatch; ++u) {
+      const int i = base + u * kThreads;
+      if (i < SB) {
+        qmb[u] = __ldg(rec + 2 * i);
+        smb[u] = __ldg(rec + 2 * i + 1);
       }
     }
-    if (key_finite(kb)) st.s += sm.x * fast_exp2((key_value(kb) - st.m) * kLog2e);
-    else if (sm.x != 0.0f) st.s += sm.x;  // NaN or +inf: the row is flagged
+#pragma unroll
+    for (int u = 0; u < kRecBatch; ++u) {
+      const int i = base + u * kThreads;
+      if (i >= SB) break;
+      const float4 qm = qmb[u];
+      const float4 sm = smb[u];
+      const uint4 k = make_uint4(fkey(qm.x), fkey(qm.y), fkey(qm.z), fkey(qm.w));
+      reinterpret_cast<uint4*>(qkeys)[i] = k;
+      const uint32_t kb = max(max(k.x, k.y), max(k.z, k.w));
+      cx.list[i] = (static_cast<uint64_t>(~kb) << 32) | static_cast<uint32_t>(i);
+      const uint32_t kmin = fkey(sm.y);
+      st.kmf = min(st.kmf, key_finite(kmin) ? kmin - (kKeyNegInf + 1u) : 0xFFFFFFFFu);
+      st.amin = min(st.amin, __float_as_uint(sm.z) & 0x7FFFFFFFu);  // smallest nonzero |l| (+inf: none)
+      // the block's sum runs against its maximum c (0 when that is not finite)
+      if (kb > st.kmax) {
+        st.kmax = kb;
+        if (key_finite(kb)) {
+          const float mn = key_value(kb);
+          st.s = st.s == 0.0f ? 0.0f : st.s * fast_exp2((st.m - mn) * kLog2e);
+          st.m = mn;
+        }
+      }
+      if (key_finite(kb)) st.s += sm.x * fast_exp2((key_value(kb) - st.m) * kLog2e);
+      else if (sm.x != 0.0f) st.s += sm.x;  // NaN or +inf: the row is flagged
+    }
   }
   if (threadIdx.x == 0) H->list_count = static_cast<uint32_t>(SB);
   __syncthreads();
   uint32_t left;
-  const uint32_t cut = stream_compact(cx, R, 0u, 64, left);  // 0 (every quarter) when SB <= R
+  // two 256-bin narrowings: a cut at most ~2^-14 of the block maxima's key range
+  // below t0 is still a valid cut and adds next to no quarter (0: every quarter
+  // when SB <= R)
+  const uint32_t cut = stream_compact(cx, R, 0u, 2, left);
   __syncthreads();
   if (threadIdx.x == 0) H->list_count = 0;
   __syncthreads();
@@ -285,13 +304,15 @@ __device__ __forceinline__ TileScan stream_tiles(const Ctx& cx, const SampleArgs
     nsel += __popc(m);
     __syncwarp();
   }
-  // gather: 8 lanes per quarter (one float4 each), 4 quarters per load, 4 loads in flight
+  // gather: 8 lanes per quarter (one float4 each), 4 quarters per load, kGather
+  // loads in flight per lane
+  constexpr int kGather = 8;
   const uint32_t below = (1u << lane) - 1u;
-  for (uint32_t u = 0; u < nsel; u += 16) {
-    float4 v[4];
-    uint32_t gid[4];
+  for (uint32_t u = 0; u < nsel; u += 4u * kGather) {
+    float4 v[kGather];
+    uint32_t gid[kGather];
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
+    for (int w = 0; w < kGather; ++w) {
       const uint32_t qi = u + 4u * w + (lane >> 3);
       gid[w] = 0xFFFFFFFFu;
       v[w] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -306,29 +327,25 @@ __device__ __forceinline__ TileScan stream_tiles(const Ctx& cx, const SampleArgs
         }
       }
     }
-    uint32_t mask[4][4], total = 0;
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
+    for (int w = 0; w < kGather; ++w) {
       const float e[4] = {v[w].x, v[w].y, v[w].z, v[w].w};
+      uint32_t mask[4], total = 0;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        mask[w][i] = __ballot_sync(0xFFFFFFFFu, gid[w] != 0xFFFFFFFFu && fkey(e[i]) >= cut);
-        total += __popc(mask[w][i]);
+        mask[i] = __ballot_sync(0xFFFFFFFFu, gid[w] != 0xFFFFFFFFu && fkey(e[i]) >= cut);
+        total += __popc(mask[i]);
       }
-    }
-    if (total == 0) continue;
-    uint32_t base = 0;
-    if (lane == 0) base = atomicAdd(&H->list_count, total);
-    base = __shfl_sync(0xFFFFFFFFu, base, 0);
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      const float e[4] = {v[w].x, v[w].y, v[w].z, v[w].w};
+      if (total == 0) continue;
+      uint32_t base = 0;
+      if (lane == 0) base = atomicAdd(&H->list_count, total);
+      base = __shfl_sync(0xFFFFFFFFu, base, 0);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const uint32_t idx = base + __popc(mask[w][i] & below);
-        if (((mask[w][i] >> lane) & 1u) && idx < static_cast<uint32_t>(kStreamCap))
+        const uint32_t idx = base + __popc(mask[i] & below);
+        if (((mask[i] >> lane) & 1u) && idx < static_cast<uint32_t>(kStreamCap))
           cx.list[idx] = (static_cast<uint64_t>(~fkey(e[i])) << 32) | (gid[w] + i);
-        base += __popc(mask[w][i]);
+        base += __popc(mask[i]);
       }
     }
   }
