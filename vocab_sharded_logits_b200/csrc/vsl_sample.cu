@@ -1213,6 +1213,11 @@ __device__ void op_xhist(const Ctx& cx, const Plan& p, uint32_t collect_lo = 0xF
   uint32_t* counter = collect_counter(cx);
   if (collect && cx.rank != 0 && threadIdx.x == 0) cx.H->list_aux = 0;
   __syncthreads();
+  // x = fl(l / T): the fused quotient where it is exact (T in [2^-20, 2^20] and
+  // l zero or 2^-60 <= |l| <= 2^100, checked per logit), else the IEEE division
+  // out of line (a rare, divergent branch)
+  const float yT = __frcp_rn(cx.T);
+  const bool t_ok = cx.T >= 0x1p-20f && cx.T <= 0x1p20f;
   const int nq = (cx.n4 + kThreads - 1) / kThreads * kThreads;  // whole warps: the appends are warp-wide
   for (int q = threadIdx.x; q < nq; q += kThreads) {
     const bool valid = q < cx.n4;
@@ -1237,7 +1242,12 @@ __device__ void op_xhist(const Ctx& cx, const Plan& p, uint32_t collect_lo = 0xF
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const bool fin = key_finite(fkey(v[i]));
-      const float x = fin ? scale_x(v[i], cx.T) : -INFINITY;
+      const float al = fabsf(v[i]);
+      float x = -INFINITY;
+      if (fin) {
+        if (t_ok && (al == 0.0f || (al >= 0x1p-60f && al <= 0x1p100f))) x = scale_x_fast(v[i], cx.T, yT);
+        else x = div_ieee(v[i], cx.T);
+      }
       v[i] = x;
       if (fin) {
         uint32_t qo;
