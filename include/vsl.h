@@ -182,7 +182,10 @@ VSL_API int32_t vsl_sample_launches(int32_t R, int32_t S, int32_t V_s);
  *   deferred_grid  : the grid of its pass over the rows the streaming kernel
  *                    marked: min(R, 2 * sms / cluster) clusters
  * sms is the device's SM count and max_cluster the largest cluster size it
- * schedules for the cluster kernel (a power of two).  Returns VSL_OK,
+ * schedules for the cluster kernel (a power of two).  The plan is that of a
+ * call without tile statistics; with them (S * B <= 4096) the streaming
+ * kernel runs one CTA per row (stream_cluster 1, stream_part S * V_s,
+ * stream_grid R), the rest unchanged.  Returns VSL_OK,
  * VSL_ERR_INVALID_ARG (null out, non-positive sizes), VSL_ERR_ALIGNMENT
  * (V_s % 4 != 0) or VSL_ERR_UNSUPPORTED (a vocabulary beyond the limits). */
 typedef struct {
