@@ -1622,10 +1622,27 @@ __device__ uint32_t list_rank_key(const Ctx& cx, int count, uint32_t r, int max_
 }
 
 // Writes the top-n (key desc, id asc) of a raw list that holds the row's top n.
-__device__ void list_topn(const Ctx& cx, const LeaderState& L, int count) {
+constexpr int kRankAllMax = 64;  // see sort_entries
+__device__ void sort_entries(const uint64_t* in, int count, uint64_t* out);
+
+// scratch_free: the caller no longer needs cx.scratch, so a list of more than
+// kRankAllMax entries is sorted there by the bitonic network instead of being
+// ranked entry against entry.
+__device__ void list_topn(const Ctx& cx, const LeaderState& L, int count, bool scratch_free = false) {
   const SampleArgs& a = *cx.a;
   const int n = a.n_logprobs;
   if (n <= 0) return;
+  if (scratch_free && count > kRankAllMax && count <= 2 * kThreads) {
+    uint64_t* buf = reinterpret_cast<uint64_t*>(cx.scratch);
+    sort_entries(cx.list, count, buf);
+    for (int j = threadIdx.x; j < min(n, count); j += kThreads) {
+      const uint64_t e = buf[j];
+      a.topn_ids[static_cast<size_t>(cx.row) * n + j] = entry_id(e);
+      a.topn_logprob[static_cast<size_t>(cx.row) * n + j] = key_value(entry_key(e)) - L.lse;
+    }
+    __syncthreads();
+    return;
+  }
   if (count <= 2 * kThreads) {
     // sort keys are distinct: an entry of rank r < n (entries smaller than it) is the (r+1)-th
     const int t = static_cast<int>(threadIdx.x);
@@ -1821,8 +1838,13 @@ __device__ void list_gumbel(const Ctx& cx, LeaderState& L, int count, bool x_key
 // entries every thread ranks its entries against all of them in one pass of
 // broadcast reads and stores each at its rank; a longer list is copied and
 // sorted by the bitonic network.
+// Lists of at most kRankAllMax entries are sorted by ranking every entry
+// against all (one pass, broadcast reads); longer ones by the bitonic network
+// (register steps, warp shuffles, shared memory only for the largest strides):
+// at 240 entries the ranking took ~9k cycles, the network far fewer barriers'
+// worth.  The output buffer holds up to the next power of two of count.
 __device__ void sort_entries(const uint64_t* in, int count, uint64_t* out) {
-  if (count <= 2 * kThreads) {
+  if (count <= kRankAllMax) {
     const int t = static_cast<int>(threadIdx.x);
     const uint64_t e0 = t < count ? in[t] : ~0ull;
     const uint64_t e1 = t + kThreads < count ? in[t + kThreads] : ~0ull;
@@ -2336,7 +2358,7 @@ __device__ void exact_tail(const Ctx& cx, LeaderState& L, double z_total = -1.0)
   float l;
   list_best(win, L, count, true, theta_p, sd, id, l);
   finish_draw(cx, L, sd, id);
-  list_topn(cx, L, first);
+  list_topn(cx, L, first, true);  // the sorted window in the scratch is no longer read
 }
 
 // Leader: merges the statistics every CTA pushed, validates data and parameters,
