@@ -166,3 +166,25 @@ def test_oracle_timing_harness_matches_the_oracle_on_every_row():
         orc.close()
     assert [t for _, t, _, _, _ in sorted(one)] == want
     assert [t for _, t, _, _, _ in sorted(many)] == want
+
+
+def test_tile_mode_row_selection():
+    """Which rows take the sampler's tile mode in the bench's accounting, and
+    when the step requests tile statistics (host logic, no device)."""
+    import bench
+    import workloads as W
+    V = 151936
+    T = [0.0, 0.8, 0.8, 0.8, 1.0]
+    k = [0, 40, 0, 2000, V]
+    assert bench._tile_rows(T, k, V).tolist() == [True, True, False, False, False]
+    sms = 148
+    for name, want in [("decode", True), ("spec", True), ("large", True), ("peaked", True), ("tiny", True)]:
+        w = W.WORKLOADS[name]
+        Tw, kw, _, _, _ = W.row_params(w)
+        assert bench._uses_tiles(w, Tw, kw, sms) == want, name
+    # a small batch of top-k-off rows only: the records would go unused
+    w = W.scaled(W.WORKLOADS["large"], requests=4)
+    Tw, kw, _, _, _ = W.row_params(w)
+    assert not bench._large_batch(w, sms) and not bench._uses_tiles(w, Tw, kw, sms)
+    # without records every row reads its V logits
+    assert bench._sampler_read_bytes(w, Tw, kw, None, sms) == w.R * w.V * 4
