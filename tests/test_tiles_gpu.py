@@ -206,3 +206,27 @@ def test_tile_mode_large_batch_top_k_off(cuda_device, V, S):
     rows = range(R) if V <= 12000 else sorted(set(range(12)) | set(rng.choice(R, 28, replace=False).tolist()))
     st = compare(got, logits, params, 4243, 20, rows)
     assert st["mismatch_allowed"] <= 2
+
+
+@pytest.mark.parametrize("S,V_s", [(16, 32768), (15, 34952)])
+def test_tile_mode_at_the_record_limit(cuda_device, S, V_s):
+    """4,096 blocks of 128 (the quarter maxima fill the streaming kernel's ring
+    exactly) and 4,110 (above the limit: the sampler ignores the records), at
+    vocabularies of about 524k: the same results as without the records, and
+    the oracle's.  Such vocabularies need clusters of 16 CTAs; a device that
+    does not schedule them rejects the size and the test is skipped."""
+    R = 6
+    rng = np.random.default_rng(S)
+    logits = rng.normal(0.0, 1.5, (R, S * V_s)).astype(np.float32)
+    params = (np.array([0.0, 0.8, 1.0, 0.7, 1.2, 0.9], np.float32), np.array([0, 40, 1000, 20, 1, 64], np.int32),
+              np.array([1.0, 0.9, 0.95, 1.0, 0.5, 0.8], np.float32), np.arange(R), np.arange(R))
+    t = torch.from_numpy(logits)
+    try:
+        ref = run_sampler(t, params, 5, 20, S, cuda_device)
+    except vsl.VslError as e:
+        if e.status == 3:
+            pytest.skip("the device does not schedule the clusters this vocabulary needs")
+        raise
+    got = run_sampler(t, params, 5, 20, S, cuda_device, tiles=True)
+    _same_as_without(got, ref)
+    compare(got, logits, params, 5, 20, range(R))
